@@ -1,0 +1,10 @@
+"""CPU binary64 oracle for exact fused linear cross-entropy.
+
+Test infrastructure: imported only by the tests, the smoke check and the
+benchmark's CPU-baseline leg.  It shares no code with the CUDA path.
+"""
+from .flce_oracle import (IGNORE_INDEX, backward, chunked, forward, forward_backward,
+                          objective, row_outputs, supervised_rows, vocab_outputs)
+
+__all__ = ["IGNORE_INDEX", "backward", "chunked", "forward", "forward_backward",
+           "objective", "row_outputs", "supervised_rows", "vocab_outputs"]
