@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of exact fused linear cross-entropy (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload packed]
+    python bench.py --impl reference ...      # the CPU oracle arm
+
+One step = flce_forward + flce_backward over one synthetic batch of the
+workload (inputs resident in HBM).  Credited work is 8*C*D*V FLOP per step
+(forward 2CDV, backward 6CDV).  With N > 1 (torchrun) each rank runs its own
+independent batch (weak scaling; the loss has no cross-rank exchange), and the
+time is the max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused linear-CE fwd+bwd TFLOP/s (8·C·D·V) & % bf16 TC peak; peak MiB"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["lm_head_projection_supervised_b200/csrc/gemm.cuh",
+                "lm_head_projection_supervised_b200/csrc/ptx.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="flce", choices=["flce", "reference"])
+    p.add_argument("--workload", default="packed")
+    p.add_argument("--cpu-rows", type=int, default=768,
+                   help="supervised rows in the CPU-oracle baseline sample")
+    p.add_argument("--ref-rows", type=int, default=64,
+                   help="supervised rows per step of the reference (oracle) arm")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_kind):
+    """DRAM bytes per launch of `kernel_kind` from the committed ncu summary,
+    or None when absent or taken on a different version of the kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_kind)
+    if not e or e.get("source_hash") != source_hash(GEMM_SOURCES):
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the timed region runs
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample of supervised rows
+# ---------------------------------------------------------------------------
+_DECODED = {}
+
+
+def oracle_sample_run(inp, rows_wanted, seed=0):
+    """Times the oracle's dense forward + backward on a seeded sample of
+    supervised rows (inputs decoded to float64 outside the timed call)."""
+    import numpy as np
+    import torch
+    from oracle import flce_oracle as orc
+    idx, C = orc.supervised_rows(inp.labels, inp.mask)
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(idx, size=min(rows_wanted, C), replace=False))
+    key = id(inp)
+    if key not in _DECODED:
+        _DECODED.clear()
+        _DECODED[key] = (inp.W64(), inp.b64())
+    W64, b64 = _DECODED[key]
+    H64 = inp.H64()[rows]
+    y = inp.labels[rows]
+    mk = inp.mask[rows]
+    t0 = time.perf_counter()
+    orc.forward_backward(H64, W64, b64, y, mk, lam=inp.lam, row_block=256)
+    dt = time.perf_counter() - t0
+    Cs = orc.supervised_rows(y, mk)[1]
+    return dt, Cs, torch.get_num_threads()
+
+
+def run_reference(args, inp, spec):
+    """The oracle as the reference arm: each step is a bounded row sample."""
+    from oracle import flce_oracle as orc  # noqa: F401
+    times, Cs, cores = [], 0, 0
+    for i in range(args.warmup + args.steps):
+        dt, Cs, cores = oracle_sample_run(inp, args.ref_rows, seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+    step_s = statistics.mean(times)
+    value = 8.0 * Cs * inp.D * inp.V / step_s / 1e12
+    sample = (f"{Cs} supervised rows of {spec.name} per step (full V={inp.V}, D={inp.D}), "
+              "fp64 dense forward+backward")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(spec, inp, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(spec, inp, n):
+    import numpy as np
+    C = int(np.count_nonzero((inp.labels != -100) & (inp.mask != 0)))
+    w_mb = inp.V * inp.D * 2 / 1e6
+    l2 = (f"inputs larger than L2 (W alone is {w_mb:.0f} MB > 126 MB); no flush" if w_mb > 126
+          else f"W is {w_mb:.0f} MB, may stay L2-resident between steps (not flushed)")
+    return {"workload": f"{spec.name}: N={inp.N} D={inp.D} V={inp.V} {spec.dtype}"
+                        f"{' +bias' if inp.b is not None else ''}, C={C}",
+            "N": inp.N, "D": inp.D, "V": inp.V, "C": C, "dtype": spec.dtype,
+            "labels": spec.label_dist, "parallelism": f"replicas{n}", "l2": l2}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from lm_head_projection_supervised_b200 import workloads as wl
+    spec = wl.SPECS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = wl.make_inputs(spec)
+        run_reference(args, inp, spec)
+        return
+
+    import numpy as np
+    import torch
+    from lm_head_projection_supervised_b200 import binding
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    inp = wl.make_inputs(spec, seed=wl.SEED_BASE + spec.k + 1000 * rank)
+    cfg = workload_config(spec, inp, world)
+    C = cfg["C"]
+    flop_step = 8.0 * C * inp.D * inp.V
+
+    # CPU baseline first (rank 0, one GPU): no GPU work has started yet.
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, Cs, cores = oracle_sample_run(inp, args.cpu_rows)
+        cpu_baseline = {"value": 8.0 * Cs * inp.D * inp.V / dt / 1e12, "unit": UNIT,
+                        "cores": cores, "kind": "oracle",
+                        "sample": f"{Cs} supervised rows of {spec.name} (full V={inp.V}, "
+                                  f"D={inp.D}), fp64 dense forward+backward, {dt:.1f} s"}
+
+    tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float16
+    torch.cuda.reset_peak_memory_stats(dev)
+    H = torch.from_numpy(inp.H.view(np.int16)).view(tdt).to(dev)
+    W = torch.from_numpy(inp.W.view(np.int16)).view(tdt).to(dev)
+    b = None if inp.b is None else torch.from_numpy(inp.b.view(np.int16)).view(tdt).to(dev)
+    y = torch.from_numpy(inp.labels).to(dev)
+    mk = torch.from_numpy(inp.mask).to(dev)
+    in_mib = sum(t.numel() * t.element_size() for t in (H, W, y, mk) + ((b,) if b is not None
+                                                                            else ())) / 2**20
+    ws = binding.Workspace(inp.N, inp.D, inp.V, tdt, dev)
+    dH = torch.empty((inp.N, inp.D), dtype=torch.float32, device=dev)
+    dW = torch.empty((inp.V, inp.D), dtype=torch.float32, device=dev)
+    db = None if b is None else torch.empty(inp.V, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        loss, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
+        binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws, out=(dH, dW, db))
+        return loss
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    n_warm = max(args.warmup, 3)
+    for _ in range(n_warm):
+        step()
+    torch.cuda.synchronize(dev)
+    st = binding.device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {binding.status_string(st)}")
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    binding.profile_begin()
+    for k in range(args.steps):
+        e0, e1, e2 = evs[k]
+        e0.record(stream)
+        loss, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
+        e1.record(stream)
+        binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws, out=(dH, dW, db))
+        e2.record(stream)
+    torch.cuda.synchronize(dev)
+    prof = binding.profile_end()
+    barrier()
+    clocks = sampler.stop()
+    st = binding.device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {binding.status_string(st)}")
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    fwd_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    t_max = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flop_step * args.steps / (total_ms * 1e-3) / 1e12
+    peak_mib = torch.cuda.max_memory_allocated(dev) / 2**20
+    launches = sum(n for _, n in prof.values())
+
+    # e2e: host buffers, copies inside the timed region, loss read back
+    e2e = None
+    if not args.no_e2e:
+        hostH, hostW = H.cpu().pin_memory(), W.cpu().pin_memory()
+        hosty, hostm = y.cpu().pin_memory(), mk.cpu().pin_memory()
+        hostb = None if b is None else b.cpu().pin_memory()
+        loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hostH, hostW, hosty, hostm) +
+                  ((hostb,) if hostb is not None else ()))
+        barrier()
+        torch.cuda.synchronize(dev)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            H.copy_(hostH, non_blocking=True)
+            W.copy_(hostW, non_blocking=True)
+            y.copy_(hosty, non_blocking=True)
+            mk.copy_(hostm, non_blocking=True)
+            if b is not None:
+                b.copy_(hostb, non_blocking=True)
+            loss = step()
+            loss_host.copy_(loss, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = s0.elapsed_time(s1)
+        te = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * flop_step * args.steps / (float(te.item()) * 1e-3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4,
+               "loss": float(loss_host.item())}
+
+    # roofline of the dominant kernel (largest share of device time)
+    peaks, peak_src = load_peaks()
+    n_panels = -(-inp.V // 4096)
+    algo_flops = {  # algorithmic FLOP per launch
+        "fwd_gemm": 2.0 * C * inp.D * inp.V,
+        "grad_gemm": 2.0 * C * inp.D * inp.V / n_panels,
+        "wh_gemm": 4.0 * C * inp.D * inp.V / n_panels,
+    }
+    dom = max(algo_flops, key=lambda k: prof[k][0])
+    ms_tot, n_l = prof[dom]
+    avg_ms = ms_tot / max(n_l, 1)
+    achieved = algo_flops[dom] / (avg_ms * 1e-3) / 1e12
+    # fp16 and bf16 share the dense tensor-core rate on this part
+    peak = peaks.get("bf16_tflops_sustained")
+    tb = ncu_traffic(dom)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_note": f"sustained dense bf16, {peak_src} (kernel timed inside a long step)",
+                "traffic": tb, "avg_launch_ms": avg_ms, "launches": n_l,
+                "kernel_share": {k: round(v[0] / max(1e-9, sum(x[0] for x in prof.values())), 4)
+                                 for k, v in prof.items()}}
+
+    burst = peaks.get("bf16_tflops")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": n_warm, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype, "data": "synthetic",
+            "config": cfg, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "fwd_tflops": 2.0 * C * inp.D * inp.V / (fwd_ms * 1e-3) / 1e12,
+            "bwd_tflops": 6.0 * C * inp.D * inp.V / (bwd_ms * 1e-3) / 1e12,
+            "pct_bf16_peak": 100.0 * (value / world) / burst,
+            "pct_bf16_peak_sustained": 100.0 * (value / world) / peaks.get(
+                "bf16_tflops_sustained"),
+            "peak_note": f"bf16 peak {burst} TFLOP/s burst, {peak_src}",
+            "peak_mib": peak_mib, "input_mib": in_mib,
+            "logits_mib_avoided": inp.N * inp.V * 2 / 2**20,
+            "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roofline, "cpu_baseline": cpu_baseline}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

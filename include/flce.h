@@ -1,0 +1,143 @@
+/*
+ * flce.h -- exact fused linear cross-entropy on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation is the one stated in "分块交叉熵 / Output projection / exact
+ * cross entropy" (glenzli.com), §01 equation:
+ *
+ *   Z_ij = H_i W_j^T + b_j                       (never stored: tiles live on chip)
+ *   a_i  = 1[mask_i] * 1[y_i != ignore_index],   C = sum_i a_i
+ *   L    = (1/C) sum_{i: a_i=1} ( (m_i - Z_{i,y_i}) + log s_i )       (§02)
+ *
+ * with m_i = max_j Z_ij and s_i = sum_j exp(Z_ij - m_i) over the full
+ * vocabulary (the running statistics of §02), and the gradients of §04:
+ *
+ *   p_ij = exp((Z_ij - m_i) - log s_i)
+ *   G_ij = (lambda a_i / C) (p_ij - 1[j = y_i])
+ *   dH = G W,   dW = G^T H,   db = sum_i G_i
+ *
+ * C = 0 gives the zero sentinel loss and zero gradients (§01).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All arrays are DEVICE pointers, dense, row-major, owned by the caller.
+ *    The library never allocates, frees or writes its inputs.  It never
+ *    synchronises the stream, except in flce_device_status().
+ *  - 16-bit tensors (H, W, b) are bf16 or fp16 per `dtype`; both operands of
+ *    one call have the same type.  H and W must be 16-byte aligned and D a
+ *    multiple of 8 (rows of 16-byte multiples, needed by the TMA engine).
+ *  - labels are int64 [N]; mask is uint8 [N] (nonzero = position takes part)
+ *    or NULL (all positions take part).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and runs asynchronously.  Argument errors are returned before
+ *    anything is enqueued.  Errors found on the device (a supervised label
+ *    outside [0, V), a pipeline wait that ran past its time limit, a
+ *    non-finite statistic) are recorded in an error word inside the
+ *    workspace, make the loss NaN, and are reported by flce_device_status().
+ *  - The workspace is caller-allocated device memory of at least
+ *    flce_workspace_bytes(N, D, V, dtype) bytes, 256-byte aligned.  Calls are
+ *    stateless: the workspace carries nothing from one call to the next, but
+ *    two calls in flight at the same time must not share one workspace.
+ *  - Only the current CUDA device is used; it must be compute capability
+ *    10.0 (sm_100a).
+ */
+#ifndef FLCE_H_
+#define FLCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FLCE_API __attribute__((visibility("default")))
+#else
+#define FLCE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_NULL = 1,        /* a required pointer is NULL                        */
+  FLCE_ERR_SHAPE = 2,       /* N, D or V out of range                            */
+  FLCE_ERR_DTYPE = 3,       /* dtype is not FLCE_BF16 / FLCE_FP16                */
+  FLCE_ERR_ALIGN = 4,       /* pointer or D not aligned as required              */
+  FLCE_ERR_WORKSPACE = 5,   /* workspace smaller than flce_workspace_bytes()     */
+  FLCE_ERR_CUDA = 6,        /* a CUDA runtime call failed                        */
+  FLCE_ERR_LABEL = 7,       /* device: a supervised label is outside [0, V)      */
+  FLCE_ERR_TIMEOUT = 8,     /* device: a pipeline wait ran past its time limit   */
+  FLCE_ERR_NONFINITE = 9,   /* device: a non-finite per-row statistic            */
+  FLCE_ERR_DEVICE = 10      /* current device is not sm_100 / cannot run kernels */
+} flce_status;
+
+typedef enum { FLCE_BF16 = 0, FLCE_FP16 = 1 } flce_dtype;
+
+/* A cudaStream_t, passed without the CUDA headers. */
+typedef void* flce_stream;
+
+/* Bytes of device workspace needed for problem size (N, D, V).  Returns 0
+ * when the sizes are out of range (same limits as FLCE_ERR_SHAPE). */
+FLCE_API size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype);
+
+/*
+ * Supervised-row compaction (a_i and C of §01; "filter: keep only labels !=
+ * -100" of "ChunkedLinearCrossEntropy (Qwen3.5 training memory peak)").
+ *
+ * Writes idx[0..C) = the supervised rows in ascending order (int32, device,
+ * capacity N) and *C_out (int32, device).  Labels of supervised rows outside
+ * [0, V) set FLCE_ERR_LABEL in the workspace error word.
+ */
+FLCE_API flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                         int64_t N, int64_t V, int32_t* idx, int32_t* C_out,
+                         void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * Forward (§01 objective, §02 running statistics).
+ *
+ *   H [N x D], W [V x D], b [V] or NULL (absent bias means b = 0)
+ *   loss  : device float scalar, the mean over the C supervised rows; 0 when C = 0
+ *   m     : device float [N], per-row max logit; -inf for unsupervised rows
+ *   logs  : device float [N], per-row log s;     -inf for unsupervised rows
+ *
+ * m and logs are the saved statistics that flce_backward() consumes.
+ */
+FLCE_API flce_status flce_forward(const void* H, const void* W, const void* b,
+                         const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                         int64_t N, int64_t D, int64_t V, int dtype,
+                         float* loss, float* m, float* logs,
+                         void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * Backward (§04 reconstruction and accumulation).
+ *
+ *   m, logs   : the statistics written by flce_forward() for the same inputs
+ *   lambda    : upstream gradient dJ/dL (host float), used when lambda_dev is NULL
+ *   lambda_dev: optional device float scalar holding lambda (lets an autograd
+ *               caller pass its gradient without a host round trip)
+ *   dH [N x D], dW [V x D] : float32 outputs, fully overwritten; rows of dH
+ *               for unsupervised positions are zero
+ *   db [V]    : float32 output, required iff b is not NULL
+ *
+ * dH, dW and db are deterministic: every output element is reduced in a
+ * fixed order independent of scheduling.
+ */
+FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
+                          const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                          int64_t N, int64_t D, int64_t V, int dtype,
+                          const float* m, const float* logs,
+                          float lambda, const float* lambda_dev,
+                          float* dH, float* dW, float* db,
+                          void* ws, size_t ws_bytes, flce_stream stream);
+
+/* Synchronises `stream`, then reads and returns the device error word of the
+ * workspace (FLCE_OK when no device error was recorded by the last call). */
+FLCE_API flce_status flce_device_status(const void* ws, flce_stream stream);
+
+/* Static, human-readable name of a status code. */
+FLCE_API const char* flce_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H_ */

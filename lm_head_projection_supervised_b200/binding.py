@@ -1,0 +1,267 @@
+"""ctypes binding of libflce.so.
+
+Argument marshalling only: every step of the loss runs in the library's CUDA
+kernels.  torch provides device memory (inputs, outputs, workspace) and the
+current stream.  There is no fallback: when the library is missing or the
+device is not sm_100, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libflce.so")
+
+FLCE_BF16, FLCE_FP16 = 0, 1
+STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DTYPE",
+          4: "FLCE_ERR_ALIGN", 5: "FLCE_ERR_WORKSPACE", 6: "FLCE_ERR_CUDA", 7: "FLCE_ERR_LABEL",
+          8: "FLCE_ERR_TIMEOUT", 9: "FLCE_ERR_NONFINITE", 10: "FLCE_ERR_DEVICE"}
+STATUS_CODE = {v: k for k, v in STATUS.items()}
+
+_lib = None
+
+
+class FlceError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}" if where else status_string(status))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libflce.so (built in-tree); raises if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built: run "
+                           "`python -m lm_head_projection_supervised_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, \
+        ctypes.c_float
+    L.flce_workspace_bytes.argtypes = [i64, i64, i64, i32]
+    L.flce_workspace_bytes.restype = sz
+    L.flce_status_string.argtypes = [i32]
+    L.flce_status_string.restype = ctypes.c_char_p
+    L.flce_compact.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, sz, vp]
+    L.flce_compact.restype = i32
+    L.flce_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, vp, sz,
+                               vp]
+    L.flce_forward.restype = i32
+    L.flce_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, f32, vp, vp,
+                                vp, vp, vp, sz, vp]
+    L.flce_backward.restype = i32
+    L.flce_device_status.argtypes = [vp, vp]
+    L.flce_device_status.restype = i32
+    L.flce_diag_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, f32, vp, sz, vp]
+    L.flce_diag_gemm.restype = i32
+    L.flce_diag_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
+    L.flce_diag_timeout.restype = i32
+    L.flce_diag_profile_begin.argtypes = []
+    L.flce_diag_profile_begin.restype = i32
+    L.flce_diag_profile_end.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                        ctypes.POINTER(ctypes.c_int64), i32]
+    L.flce_diag_profile_end.restype = i32
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().flce_status_string(int(status)).decode()
+    except RuntimeError:
+        return STATUS.get(int(status), f"status {status}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise FlceError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return FLCE_BF16
+    if dt == torch.float16:
+        return FLCE_FP16
+    raise TypeError(f"H and W must be bfloat16 or float16, got {dt}")
+
+
+def workspace_bytes(N: int, D: int, V: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib().flce_workspace_bytes(N, D, V, dtype_code(dtype)))
+
+
+class Workspace:
+    """Caller-owned device scratch of flce_workspace_bytes() bytes."""
+
+    def __init__(self, N: int, D: int, V: int, dtype: torch.dtype, device=None):
+        n = workspace_bytes(N, D, V, dtype)
+        if n == 0:
+            raise FlceError(STATUS_CODE["FLCE_ERR_SHAPE"], "workspace_bytes")
+        self.nbytes = n
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def _prep(H, W, b, labels, mask):
+    if not (H.is_cuda and W.is_cuda and labels.is_cuda):
+        raise ValueError("H, W and labels must be CUDA tensors")
+    if H.dtype != W.dtype or (b is not None and b.dtype != H.dtype):
+        raise TypeError("H, W and b must share one dtype")
+    D = H.shape[-1]
+    H2 = H.reshape(-1, D)
+    if not H2.is_contiguous():
+        H2 = H2.contiguous()
+    if W.dim() != 2 or W.shape[1] != D:
+        raise ValueError(f"W must be [V, {D}]")
+    W2 = W if W.is_contiguous() else W.contiguous()
+    y = labels.reshape(-1)
+    if y.dtype != torch.int64:
+        y = y.to(torch.int64)
+    if y.numel() != H2.shape[0]:
+        raise ValueError("labels must have one entry per row of H")
+    y = y.contiguous()
+    mk = None
+    if mask is not None:
+        mk = mask.reshape(-1)
+        if mk.dtype == torch.bool:
+            mk = mk.view(torch.uint8)
+        elif mk.dtype != torch.uint8:
+            mk = (mk != 0).view(torch.uint8)
+        mk = mk.contiguous()
+    b2 = None if b is None else b.contiguous()
+    return H2, W2, b2, y, mk
+
+
+def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[Workspace] = None,
+            stream=None):
+    """loss (0-d float32), m [N], logs [N] -- flce_forward()."""
+    H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
+    N, D = H2.shape
+    V = W2.shape[0]
+    if ws is None:
+        ws = Workspace(N, D, V, H2.dtype, H2.device)
+    loss = torch.empty((), dtype=torch.float32, device=H2.device)
+    m = torch.empty(N, dtype=torch.float32, device=H2.device)
+    logs = torch.empty(N, dtype=torch.float32, device=H2.device)
+    st = lib().flce_forward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D, V,
+                            dtype_code(H2.dtype), _ptr(loss), _ptr(m), _ptr(logs), ws.ptr(),
+                            ws.nbytes, _stream(stream))
+    _check(st, "flce_forward")
+    return loss, m, logs
+
+
+def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0, lam_dev=None,
+             ws: Optional[Workspace] = None, out=None, stream=None):
+    """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward()."""
+    H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
+    N, D = H2.shape
+    V = W2.shape[0]
+    if ws is None:
+        ws = Workspace(N, D, V, H2.dtype, H2.device)
+    if out is None:
+        dH = torch.empty((N, D), dtype=torch.float32, device=H2.device)
+        dW = torch.empty((V, D), dtype=torch.float32, device=H2.device)
+        db = None if b2 is None else torch.empty(V, dtype=torch.float32, device=H2.device)
+    else:
+        dH, dW, db = out
+    if lam_dev is not None:
+        lam_dev = lam_dev.reshape(()).to(torch.float32).contiguous()
+    st = lib().flce_backward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D,
+                             V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), float(lam),
+                             _ptr(lam_dev), _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
+                             _stream(stream))
+    _check(st, "flce_backward")
+    return dH, dW, db
+
+
+def device_status(ws: Workspace, stream=None) -> int:
+    return int(lib().flce_device_status(ws.ptr(), _stream(stream)))
+
+
+def compact(labels, mask, ignore_index: int, V: int, stream=None):
+    """idx (int32, first C valid) and C (int32 device scalar) -- flce_compact()."""
+    y = labels.reshape(-1).to(torch.int64).contiguous()
+    mk = None
+    if mask is not None:
+        mk = mask.reshape(-1).to(torch.uint8).contiguous()
+    N = y.numel()
+    idx = torch.empty(max(N, 1), dtype=torch.int32, device=y.device)
+    C = torch.empty((), dtype=torch.int32, device=y.device)
+    ws = torch.empty(256, dtype=torch.uint8, device=y.device)
+    st = lib().flce_compact(_ptr(y), _ptr(mk), ignore_index, N, V, _ptr(idx), _ptr(C),
+                            _ptr(ws), 256, _stream(stream))
+    _check(st, "flce_compact")
+    return idx, C, ws
+
+
+def diag_gemm(A, B, M: int, N: int, K: int, a_mn: bool, b_mn: bool, scale: float = 1.0,
+              stream=None):
+    out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=A.device)
+    st = lib().flce_diag_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, dtype_code(A.dtype),
+                              int(a_mn), int(b_mn), float(scale), _ptr(ws), 256, _stream(stream))
+    _check(st, "flce_diag_gemm")
+    s2 = lib().flce_device_status(_ptr(ws), _stream(stream))
+    _check(s2, "flce_diag_gemm (device)")
+    return out
+
+
+def diag_timeout(limit_ns: int, device="cuda", stream=None) -> int:
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    _check(lib().flce_diag_timeout(_ptr(ws), 256, int(limit_ns), _stream(stream)),
+           "flce_diag_timeout")
+    return int(lib().flce_device_status(_ptr(ws), _stream(stream)))
+
+
+PROFILE_KINDS = ("fwd_gemm", "grad_gemm", "wh_gemm", "aux")
+
+
+def profile_begin():
+    _check(lib().flce_diag_profile_begin(), "flce_diag_profile_begin")
+
+
+def profile_end():
+    """Per kernel kind: (total ms, launches) recorded since profile_begin()."""
+    ms = (ctypes.c_double * 4)()
+    n = (ctypes.c_int64 * 4)()
+    _check(lib().flce_diag_profile_end(ms, n, 4), "flce_diag_profile_end")
+    return {k: (ms[i], int(n[i])) for i, k in enumerate(PROFILE_KINDS)}
+
+
+class FusedLinearCrossEntropy(torch.autograd.Function):
+    """L = mean over supervised rows of CE(H W^T + b, y); gradients from the
+    library's backward, with the upstream gradient passed on the device."""
+
+    @staticmethod
+    def forward(ctx, H, W, b, labels, mask, ignore_index):
+        loss, m, logs = forward(H, W, b, labels, mask, ignore_index)
+        ctx.save_for_backward(H, W, b, labels, mask, m, logs)
+        ctx.ignore_index = ignore_index
+        return loss
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        H, W, b, labels, mask, m, logs = ctx.saved_tensors
+        dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs,
+                              lam_dev=grad_out.detach())
+        return (dH.reshape(H.shape).to(H.dtype), dW.to(W.dtype),
+                None if db is None else db.to(b.dtype), None, None, None)
+
+
+def fused_linear_cross_entropy(H, W, labels, b=None, mask=None, ignore_index: int = -100):
+    return FusedLinearCrossEntropy.apply(H, W, b, labels, mask, ignore_index)

@@ -1,0 +1,244 @@
+// Memory-bound helper kernels around the tensor-core GEMMs: supervised-row
+// compaction, row gather, merge of per-tile statistics, the deterministic
+// loss mean, bias-gradient column sums and zeroing of unsupervised dH rows.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace flce {
+
+constexpr int COMPACT_THREADS = 1024;
+
+__device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8_t* mask,
+                                              int64_t ignore, int64_t i) {
+  return labels[i] != ignore && (mask == nullptr || mask[i] != 0);
+}
+
+// a_i = 1[mask_i] 1[y_i != ignore]; idx = supervised rows ascending (stable),
+// y_c = their labels (optional), C = count ("分块交叉熵" page §01; the supervised-row
+// filter of "ChunkedLinearCrossEntropy").  One block: each thread scans a
+// contiguous slice, a block-wide exclusive scan of the slice counts gives
+// every thread its output offset.  Labels outside [0, V) on supervised rows
+// set the label error bit and are clamped to 0 so later indexing stays in
+// range.  Unsupervised rows get m = log s = -inf when m_out is given.
+__global__ void __launch_bounds__(COMPACT_THREADS)
+    compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
+                   int64_t ignore, int64_t N, int64_t V, int* __restrict__ idx,
+                   int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
+                   float* __restrict__ m_out, float* __restrict__ logs_out) {
+  __shared__ int warp_tot[COMPACT_THREADS / 32];
+  const int t = threadIdx.x;
+  const int64_t per = (N + COMPACT_THREADS - 1) / COMPACT_THREADS;
+  const int64_t beg = min(N, t * per);
+  const int64_t end = min(N, beg + per);
+  int cnt = 0;
+  for (int64_t i = beg; i < end; ++i) cnt += is_supervised(labels, mask, ignore, i) ? 1 : 0;
+  // block exclusive scan of cnt
+  const int lane = t & 31, warp = t >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += v;
+    }
+    warp_tot[lane] = wi - w;  // exclusive warp offsets
+    if (lane == 31) *C_out = wi;
+  }
+  __syncthreads();
+  int off = warp_tot[warp] + incl - cnt;
+  bool bad = false;
+  for (int64_t i = beg; i < end; ++i) {
+    if (is_supervised(labels, mask, ignore, i)) {
+      int64_t y = labels[i];
+      if (y < 0 || y >= V) {
+        bad = true;
+        y = 0;
+      }
+      idx[off] = static_cast<int>(i);
+      if (y_c != nullptr) y_c[off] = static_cast<int>(y);
+      ++off;
+    } else if (m_out != nullptr) {
+      m_out[i] = -INFINITY;
+      logs_out[i] = -INFINITY;
+    }
+  }
+  if (bad) atomicOr(err, kErrBitLabel);
+}
+
+// H_c[k] = H[idx[k]] for k < C, zero rows for C <= k < Np (16-byte vectors,
+// one warp per row).
+__global__ void gather_rows_kernel(const uint4* __restrict__ H, const int* __restrict__ idx,
+                                   const int* __restrict__ C_dev, int64_t Np, int64_t vec_per_row,
+                                   uint4* __restrict__ Hc) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= Np) return;
+  const int lane = threadIdx.x & 31;
+  const int C = *C_dev;
+  uint4* dst = Hc + row * vec_per_row;
+  if (row < C) {
+    const uint4* src = H + static_cast<int64_t>(idx[row]) * vec_per_row;
+    for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = __ldg(src + k);
+  } else {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
+  }
+}
+
+// Online-softmax merge of two partial states (m, s): the running update of
+// the "分块交叉熵" page §02, in the two-state form of the maths-basics page
+// (online softmax block merge).  -inf marks an empty state.
+__device__ __forceinline__ void merge_state(float& m, float& s, float om, float os) {
+  if (om == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = om;
+    s = os;
+    return;
+  }
+  const float mn = fmaxf(m, om);
+  s = s * expf(m - mn) + os * expf(om - mn);
+  m = mn;
+}
+
+// Per supervised row: merge the per-vocabulary-tile partials (lane-strided,
+// then a butterfly of warp shuffles, symmetric so that every lane ends with
+// the same state), then m_i, log s_i and l_i = (m_i - target_i) + log s_i.
+__global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld, int nvt,
+                                   const float* __restrict__ tgt, const int* __restrict__ C_dev,
+                                   const int* __restrict__ idx, float* __restrict__ m_out,
+                                   float* __restrict__ logs_out, float* __restrict__ loss_rows,
+                                   uint32_t* err) {
+  const int C = *C_dev;
+  const int lane = threadIdx.x & 31;
+  const int warps = (blockDim.x >> 5) * gridDim.x;
+  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < C; i += warps) {
+    const float2* pr = part + static_cast<size_t>(i) * part_ld;
+    float m = -INFINITY, s = 0.f;
+    for (int v = lane; v < nvt; v += 32) {
+      const float2 ps = pr[v];
+      merge_state(m, s, ps.x, ps.y);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, m, o);
+      const float os = __shfl_xor_sync(0xffffffffu, s, o);
+      merge_state(m, s, om, os);
+    }
+    if (lane == 0) {
+      const float logs = logf(s);
+      const float li = (m - tgt[i]) + logs;
+      const int o = idx[i];
+      m_out[o] = m;
+      logs_out[o] = logs;
+      loss_rows[i] = li;
+      if (!isfinite(li) || !isfinite(m) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
+    }
+  }
+}
+
+// L = (1/C) sum_i l_i in a fixed order (per-thread strided sums in double,
+// then a fixed tree); 0 when C = 0; NaN when the label or timeout bit is set.
+__global__ void __launch_bounds__(1024)
+    loss_mean_kernel(const float* __restrict__ loss_rows, const int* __restrict__ C_dev,
+                     const uint32_t* err, float* __restrict__ loss) {
+  __shared__ double red[1024];
+  const int C = *C_dev;
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < C; i += blockDim.x) acc += static_cast<double>(loss_rows[i]);
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float L = (C > 0) ? static_cast<float>(red[0] / C) : 0.f;
+    if (*err & (kErrBitLabel | kErrBitTimeout)) L = __int_as_float(0x7fc00000);
+    *loss = L;
+  }
+}
+
+// db[vp + j] = scale * sum_{i < C} Gp[i][j] for the panel's columns, in a
+// fixed order: 8 row groups per block, combined in group order.
+__global__ void __launch_bounds__(256)
+    bias_grad_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
+                     const int* __restrict__ C_dev, float lam, const float* lam_dev,
+                     float inv_sigma, int is_bf16, int vp, float* __restrict__ db) {
+  __shared__ float2 part[8][32];
+  const int C = *C_dev;
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int j = blockIdx.x * 64 + 2 * lane;  // two adjacent columns per thread
+  float2 acc = make_float2(0.f, 0.f);
+  if (j < w) {
+    for (int i = grp; i < C; i += 8) {
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(Gp + static_cast<int64_t>(i) * ldg + j);
+      if (is_bf16) {
+        acc.x += __uint_as_float((v & 0xFFFFu) << 16);
+        acc.y += __uint_as_float(v & 0xFFFF0000u);
+      } else {
+        const __half2 h = *reinterpret_cast<const __half2*>(&v);
+        const float2 f = __half22float2(h);
+        acc.x += f.x;
+        acc.y += f.y;
+      }
+    }
+  }
+  part[grp][lane] = acc;
+  __syncthreads();
+  if (grp == 0 && j < w) {
+    float2 t = part[0][lane];
+    for (int k = 1; k < 8; ++k) {
+      t.x += part[k][lane].x;
+      t.y += part[k][lane].y;
+    }
+    const float lam_v = (lam_dev != nullptr) ? *lam_dev : lam;
+    const float scale = (C > 0) ? lam_v / static_cast<float>(C) * inv_sigma : 0.f;
+    db[vp + j] = t.x * scale;
+    if (j + 1 < w) db[vp + j + 1] = t.y * scale;
+  }
+}
+
+// dH rows of unsupervised positions are zero (one warp per row).
+__global__ void zero_unsupervised_rows_kernel(const int64_t* __restrict__ labels,
+                                              const uint8_t* __restrict__ mask, int64_t ignore,
+                                              int64_t N, int64_t vec_per_row,
+                                              float4* __restrict__ dH) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= N) return;
+  if (is_supervised(labels, mask, ignore, row)) return;
+  const int lane = threadIdx.x & 31;
+  float4* dst = dH + row * vec_per_row;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
+}
+
+// Failure-path check: waits on a barrier nothing completes, with a short
+// limit; the bounded wait records the timeout bit and the kernel returns.
+__global__ void timeout_probe_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, err, limit_ns);
+    if (ok) atomicOr(err, 1u << 31);  // impossible: nothing arrives on `bar`
+  }
+}
+
+}  // namespace flce

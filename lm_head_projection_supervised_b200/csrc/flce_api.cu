@@ -1,0 +1,543 @@
+// C ABI of libflce.so: argument validation, workspace carving, TMA tensor
+// maps and the launch sequence of the forward and backward passes.
+//
+// Forward  (one stream, no host synchronisation):
+//   compact -> gather H_c -> gemm<fwd> (Z tiles + online (m, s) + target)
+//   -> merge partials per row -> fixed-order loss mean
+// Backward:
+//   compact -> gather H_c -> zero dH rows of unsupervised positions ->
+//   for each vocabulary panel of Vc columns:
+//       gemm<grad>  G panel = (p - onehot) * sigma, 16-bit, C x Vc
+//       gemm<wh>    dW[panel] = scale G^T H_c ;  dH[idx] (+)= scale G W[panel]
+//       bias_grad   db[panel] = scale * column sums of G   (bias only)
+//   with scale = lambda / (C sigma).
+#include <mutex>
+#include <vector>
+
+#include "../../include/flce.h"
+#include "../../include/flce_diag.h"
+#include "aux_kernels.cuh"
+#include "gemm.cuh"
+
+using namespace flce;
+
+namespace {
+
+constexpr int64_t kMaxN = int64_t(1) << 24;
+constexpr int64_t kMaxD = int64_t(1) << 16;
+constexpr int64_t kMaxV = int64_t(1) << 24;
+constexpr int64_t kPanelCols = 4096;  // vocabulary columns per gradient panel
+constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
+
+int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
+
+struct Layout {
+  size_t err, C, idx, yc, hc, part, tgt, loss_rows, gpanel, total;
+  int64_t Np, nvt, vc;
+};
+
+// Workspace carve-up.  The error word sits at offset 0 for every size.
+Layout make_layout(int64_t N, int64_t D, int64_t V) {
+  Layout L{};
+  L.Np = roundup64(N > 0 ? N : 1, BM);
+  L.nvt = cdiv64(V, BN);
+  L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += static_cast<size_t>(roundup64(static_cast<int64_t>(bytes), 1024));
+    return o;
+  };
+  L.err = take(256);
+  L.C = take(256);
+  L.idx = take(static_cast<size_t>(L.Np) * 4);
+  L.yc = take(static_cast<size_t>(L.Np) * 4);
+  L.hc = take(static_cast<size_t>(L.Np) * D * 2);
+  L.part = take(static_cast<size_t>(L.Np) * L.nvt * 8);
+  L.tgt = take(static_cast<size_t>(L.Np) * 4);
+  L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
+  L.gpanel = take(static_cast<size_t>(L.Np) * L.vc * 2);
+  L.total = off;
+  return L;
+}
+
+bool shape_ok(int64_t N, int64_t D, int64_t V) {
+  return N >= 0 && N <= kMaxN && D >= 8 && D <= kMaxD && V >= 1 && V <= kMaxV;
+}
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---- driver entry point for tensor-map encoding (no link against libcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D map over a row-major 16-bit matrix [outer x inner] with row pitch
+// `pitch` bytes, 128-byte swizzle, zero fill outside the extents.
+bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+              uint64_t pitch, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- per-device set-up
+struct DevInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+flce_status device_setup(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FLCE_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0) && encode_fn() != nullptr;
+    if (d.ok) {
+      const int bytes = static_cast<int>(GEMM_SMEM_BYTES);
+      if (cudaFuncSetAttribute(flce_gemm_kernel<kModeFwd>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+          cudaFuncSetAttribute(flce_gemm_kernel<kModeGrad>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+          cudaFuncSetAttribute(flce_gemm_kernel<kModeWH>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+          cudaFuncSetAttribute(flce_gemm_kernel<kModePlain>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+    }
+    d.sms = sms;
+    d.init = true;
+  }
+  *out = d;
+  return d.ok ? FLCE_OK : FLCE_ERR_DEVICE;
+}
+
+#define FLCE_CK(expr)                               \
+  do {                                              \
+    if ((expr) != cudaSuccess) return FLCE_ERR_CUDA; \
+  } while (0)
+
+// ---- optional per-launch timing (diagnostic; off unless profile_begin)
+struct ProfRec {
+  int kind;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+
+enum ProfKind : int { kProfFwd = 0, kProfGrad = 1, kProfWH = 2, kProfAux = 3 };
+
+// Runs `launch` (which enqueues one kernel on s); when profiling is on, the
+// launch is bracketed by two events on the same stream.
+template <class F>
+cudaError_t timed_launch(int kind, cudaStream_t s, F&& launch) {
+  bool on;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    on = g_prof_on;
+  }
+  if (!on) {
+    launch();
+    return cudaGetLastError();
+  }
+  ProfRec r{kind, nullptr, nullptr};
+  if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess)
+    return cudaErrorUnknown;
+  cudaEventRecord(r.start, s);
+  launch();
+  const cudaError_t e = cudaGetLastError();
+  cudaEventRecord(r.stop, s);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof.push_back(r);
+  return e;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int sms, cudaStream_t s) {
+  if (units_upper <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(units_upper < sms ? units_upper : sms);
+  const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeGrad ? kProfGrad
+                 : MODE == kModeWH ? kProfWH : kProfAux;
+  return timed_launch(kind, s, [&] {
+    flce_gemm_kernel<MODE><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, s>>>(a);
+  });
+}
+
+struct WsPtrs {
+  uint32_t* err;
+  int* C;
+  int* idx;
+  int* yc;
+  uint16_t* hc;
+  float2* part;
+  float* tgt;
+  float* loss_rows;
+  uint16_t* gpanel;
+};
+
+WsPtrs carve(void* ws, const Layout& L) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return WsPtrs{reinterpret_cast<uint32_t*>(w + L.err), reinterpret_cast<int*>(w + L.C),
+                reinterpret_cast<int*>(w + L.idx),       reinterpret_cast<int*>(w + L.yc),
+                reinterpret_cast<uint16_t*>(w + L.hc),   reinterpret_cast<float2*>(w + L.part),
+                reinterpret_cast<float*>(w + L.tgt),     reinterpret_cast<float*>(w + L.loss_rows),
+                reinterpret_cast<uint16_t*>(w + L.gpanel)};
+}
+
+// compaction + gather of the supervised rows into the workspace
+flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
+                     int64_t N, int64_t D, int64_t V, const Layout& L, const WsPtrs& p,
+                     float* m_out, float* logs_out, cudaStream_t s) {
+  FLCE_CK(cudaMemsetAsync(p.err, 0, 256, s));
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, p.idx, p.yc, p.C,
+                                               p.err, m_out, logs_out);
+  }));
+  const int64_t vec = D / 8;
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    gather_rows_kernel<<<static_cast<unsigned>(cdiv64(L.Np, 8)), 256, 0, s>>>(
+      static_cast<const uint4*>(H), p.idx, p.C, L.Np, vec, reinterpret_cast<uint4*>(p.hc));
+  }));
+  return FLCE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype) {
+  if (!shape_ok(N, D, V) || (dtype != FLCE_BF16 && dtype != FLCE_FP16)) return 0;
+  return make_layout(N, D, V).total;
+}
+
+const char* flce_status_string(int status) {
+  switch (status) {
+    case FLCE_OK: return "FLCE_OK";
+    case FLCE_ERR_NULL: return "FLCE_ERR_NULL: a required pointer is NULL";
+    case FLCE_ERR_SHAPE: return "FLCE_ERR_SHAPE: N, D or V out of range";
+    case FLCE_ERR_DTYPE: return "FLCE_ERR_DTYPE: dtype must be FLCE_BF16 or FLCE_FP16";
+    case FLCE_ERR_ALIGN: return "FLCE_ERR_ALIGN: misaligned pointer or D not a multiple of 8";
+    case FLCE_ERR_WORKSPACE: return "FLCE_ERR_WORKSPACE: workspace too small";
+    case FLCE_ERR_CUDA: return "FLCE_ERR_CUDA: a CUDA runtime call failed";
+    case FLCE_ERR_LABEL: return "FLCE_ERR_LABEL: supervised label outside [0, V)";
+    case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT: a device pipeline wait ran out";
+    case FLCE_ERR_NONFINITE: return "FLCE_ERR_NONFINITE: non-finite per-row statistic";
+    case FLCE_ERR_DEVICE: return "FLCE_ERR_DEVICE: current device is not sm_100";
+    default: return "FLCE_ERR_UNKNOWN";
+  }
+}
+
+flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                         int64_t N, int64_t V, int32_t* idx, int32_t* C_out, void* ws,
+                         size_t ws_bytes, flce_stream stream) {
+  if (labels == nullptr || idx == nullptr || C_out == nullptr || ws == nullptr)
+    return FLCE_ERR_NULL;
+  if (N < 0 || N > kMaxN || V < 1 || V > kMaxV) return FLCE_ERR_SHAPE;
+  if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
+  if (ws_bytes < 256) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
+  compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, idx, nullptr,
+                                               C_out, err, nullptr, nullptr);
+  FLCE_CK(cudaGetLastError());
+  return FLCE_OK;
+}
+
+flce_status flce_forward(const void* H, const void* W, const void* b, const int64_t* labels,
+                         const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                         int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
+                         size_t ws_bytes, flce_stream stream) {
+  if (H == nullptr || W == nullptr || labels == nullptr || loss == nullptr || m == nullptr ||
+      logs == nullptr || ws == nullptr)
+    return FLCE_ERR_NULL;
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
+  if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
+  if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
+      !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) || !aligned(loss, 4))
+    return FLCE_ERR_ALIGN;
+  const Layout L = make_layout(N, D, V);
+  if (ws_bytes < L.total) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsPtrs p = carve(ws, L);
+  const bool bf16 = dtype == FLCE_BF16;
+
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, s);
+  if (st != FLCE_OK) return st;
+
+  GemmArgs a{};
+  if (!make_map(&a.tmA[0], p.hc, bf16, D, L.Np, D * 2, BK, BM) ||
+      !make_map(&a.tmB[0], W, bf16, D, V, D * 2, BK, BN))
+    return FLCE_ERR_CUDA;
+  a.is_bf16 = bf16;
+  a.C_dev = p.C;
+  a.ncols = static_cast<int>(V);
+  a.K = static_cast<int>(D);
+  a.D = static_cast<int>(D);
+  a.V = static_cast<int>(V);
+  a.vp = 0;
+  a.y_c = p.yc;
+  a.idx = p.idx;
+  a.bias = static_cast<const uint16_t*>(b);
+  a.part = p.part;
+  a.part_ld = static_cast<int>(L.nvt);
+  a.tgt = p.tgt;
+  a.err = p.err;
+  FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, BM) * L.nvt, di.sms, s));
+
+  if (N > 0) {
+    const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+    merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
+        p.loss_rows, p.err);
+  }));
+  }
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    loss_mean_kernel<<<1, 1024, 0, s>>>(p.loss_rows, p.C, p.err, loss);
+  }));
+  return FLCE_OK;
+}
+
+flce_status flce_backward(const void* H, const void* W, const void* b, const int64_t* labels,
+                          const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                          int64_t V, int dtype, const float* m, const float* logs, float lambda,
+                          const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
+                          size_t ws_bytes, flce_stream stream) {
+  if (H == nullptr || W == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
+      dH == nullptr || dW == nullptr || ws == nullptr || (b != nullptr && db == nullptr))
+    return FLCE_ERR_NULL;
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
+  if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
+  if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
+      !aligned(ws, 256) || !aligned(dH, 16) || !aligned(dW, 16) ||
+      (db != nullptr && !aligned(db, 8)) || !aligned(m, 4) || !aligned(logs, 4))
+    return FLCE_ERR_ALIGN;
+  const Layout L = make_layout(N, D, V);
+  if (ws_bytes < L.total) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsPtrs p = carve(ws, L);
+  const bool bf16 = dtype == FLCE_BF16;
+  const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
+  const float sigma = exp2f(log2_sigma);
+
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, s);
+  if (st != FLCE_OK) return st;
+  if (N > 0) {
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+    zero_unsupervised_rows_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
+        labels, mask, ignore_index, N, D / 4, reinterpret_cast<float4*>(dH));
+  }));
+  }
+
+  // operand maps that do not depend on the panel
+  CUtensorMap hcK, wK, hcMN, wMN;
+  if (!make_map(&hcK, p.hc, bf16, D, L.Np, D * 2, BK, BM) ||
+      !make_map(&wK, W, bf16, D, V, D * 2, BK, BN) ||
+      !make_map(&hcMN, p.hc, bf16, D, L.Np, D * 2, 64, BK) ||
+      !make_map(&wMN, W, bf16, D, V, D * 2, 64, BK))
+    return FLCE_ERR_CUDA;
+
+  const int64_t nT_max = cdiv64(N, BM);
+  const int64_t nD = cdiv64(D, BN);
+  for (int64_t vp = 0; vp < V; vp += L.vc) {
+    const int64_t w = (V - vp) < L.vc ? (V - vp) : L.vc;
+    CUtensorMap gK, gMN;
+    if (!make_map(&gK, p.gpanel, bf16, w, L.Np, L.vc * 2, 64, BM) ||
+        !make_map(&gMN, p.gpanel, bf16, w, L.Np, L.vc * 2, 64, BK))
+      return FLCE_ERR_CUDA;
+
+    GemmArgs a{};
+    a.tmA[0] = hcK;
+    a.tmB[0] = wK;
+    a.tmOut = gK;
+    a.is_bf16 = bf16;
+    a.C_dev = p.C;
+    a.ncols = static_cast<int>(w);
+    a.K = static_cast<int>(D);
+    a.D = static_cast<int>(D);
+    a.V = static_cast<int>(V);
+    a.vp = static_cast<int>(vp);
+    a.y_c = p.yc;
+    a.idx = p.idx;
+    a.bias = static_cast<const uint16_t*>(b);
+    a.m_saved = m;
+    a.logs_saved = logs;
+    a.log2_sigma = log2_sigma;
+    a.sigma = sigma;
+    a.err = p.err;
+    FLCE_CK(launch_gemm<kModeGrad>(a, nT_max * cdiv64(w, BN), di.sms, s));
+
+    GemmArgs c{};
+    c.tmA[0] = gMN;   // dW: A = G panel, vocabulary-major
+    c.tmB[0] = hcMN;  //     B = H_c, hidden-major
+    c.tmA[1] = gK;    // dH: A = G panel, K = vocabulary
+    c.tmB[1] = wMN;   //     B = W[panel], hidden-major
+    c.is_bf16 = bf16;
+    c.C_dev = p.C;
+    c.K = static_cast<int>(w);
+    c.D = static_cast<int>(D);
+    c.V = static_cast<int>(V);
+    c.vp = static_cast<int>(vp);
+    c.nVb = static_cast<int>(cdiv64(w, BM));
+    c.nDW = static_cast<int>(cdiv64(w, BM) * nD);
+    c.idx = p.idx;
+    c.lam = lambda;
+    c.lam_dev = lambda_dev;
+    c.inv_sigma = 1.f / sigma;
+    c.dW = dW;
+    c.dH = dH;
+    c.err = p.err;
+    FLCE_CK(launch_gemm<kModeWH>(c, c.nDW + nT_max * nD, di.sms, s));
+
+    if (b != nullptr) {
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+    bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w, 64)), 256, 0, s>>>(
+          p.gpanel, L.vc, static_cast<int>(w), p.C, lambda, lambda_dev, 1.f / sigma, bf16 ? 1 : 0,
+          static_cast<int>(vp), db);
+  }));
+    }
+  }
+  return FLCE_OK;
+}
+
+flce_status flce_device_status(const void* ws, flce_stream stream) {
+  if (ws == nullptr) return FLCE_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FLCE_ERR_CUDA;
+  uint32_t e = 0;
+  if (cudaMemcpy(&e, ws, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (e & kErrBitLabel) return FLCE_ERR_LABEL;
+  if (e & kErrBitTimeout) return FLCE_ERR_TIMEOUT;
+  if (e & kErrBitNonfinite) return FLCE_ERR_NONFINITE;
+  if (e != 0) return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
+
+flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, int64_t N,
+                           int64_t K, int dtype, int a_mn, int b_mn, float scale, void* ws,
+                           size_t ws_bytes, flce_stream stream) {
+  if (A == nullptr || B == nullptr || out == nullptr || ws == nullptr) return FLCE_ERR_NULL;
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
+  if (M < 1 || N < 1 || K < 1 || M > kMaxN || N > kMaxV || K > kMaxN) return FLCE_ERR_SHAPE;
+  if ((a_mn ? M : K) % 8 != 0 || (b_mn ? N : K) % 8 != 0 || !aligned(A, 16) ||
+      !aligned(B, 16) || !aligned(ws, 256))
+    return FLCE_ERR_ALIGN;
+  if (ws_bytes < 256) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FLCE_BF16;
+  GemmArgs a{};
+  const bool okA = a_mn ? make_map(&a.tmA[0], A, bf16, M, K, M * 2, 64, BK)
+                        : make_map(&a.tmA[0], A, bf16, K, M, K * 2, BK, BM);
+  const bool okB = b_mn ? make_map(&a.tmB[0], B, bf16, N, K, N * 2, 64, BK)
+                        : make_map(&a.tmB[0], B, bf16, K, N, K * 2, BK, BN);
+  if (!okA || !okB) return FLCE_ERR_CUDA;
+  a.a_mn = a_mn ? 1 : 0;
+  a.b_mn = b_mn ? 1 : 0;
+  a.is_bf16 = bf16;
+  a.M = static_cast<int>(M);
+  a.ncols = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.out = out;
+  a.scale = scale;
+  a.err = static_cast<uint32_t*>(ws);
+  FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
+  FLCE_CK(launch_gemm<kModePlain>(a, cdiv64(M, BM) * cdiv64(N, BN), di.sms, s));
+  return FLCE_OK;
+}
+
+flce_status flce_diag_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, flce_stream stream) {
+  if (ws == nullptr) return FLCE_ERR_NULL;
+  if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
+  if (ws_bytes < 256) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
+  timeout_probe_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(ws), limit_ns);
+  FLCE_CK(cudaGetLastError());
+  return FLCE_OK;
+}
+
+flce_status flce_diag_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return FLCE_OK;
+}
+
+flce_status flce_diag_profile_end(double* ms, int64_t* launches, int nkinds) {
+  if (ms == nullptr || launches == nullptr) return FLCE_ERR_NULL;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  for (int k = 0; k < nkinds; ++k) {
+    ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  flce_status st = FLCE_OK;
+  for (auto& r : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+      st = FLCE_ERR_CUDA;
+    if (r.kind < nkinds) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  g_prof.clear();
+  return st;
+}
+
+}  // extern "C"
