@@ -82,19 +82,20 @@ def ncu_traffic(kernel_kind):
 # clocks sampled while the timed region runs
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
+    def __init__(self, uuid: str):
+        self.uuid = "".join(c for c in uuid.lower() if c in "0123456789abcdef")
         self.proc = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -108,12 +109,15 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        rows = [[x.strip() for x in line.split(",")] for line in out.strip().splitlines()]
+        rows = [r for r in rows if len(r) >= 9]
+        mine = [r for r in rows
+                if "".join(c for c in r[0].lower() if c in "0123456789abcdef").endswith(self.uuid)]
+        if mine:
+            rows = mine
         sm, smax, reasons, power = [], [], set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
+        for parts in rows:
             try:
                 sm.append(float(parts[1]))
                 smax.append(float(parts[2]))
@@ -126,7 +130,7 @@ class ClockSampler:
         load = [s for s, p in zip(sm, power) if p > 300.0] or sm
         return {"sm_mhz": statistics.median(load) if load else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
+                "reasons": sorted(reasons), "samples": len(sm), "matched_uuid": bool(mine),
                 "power_w_max": max(power) if power else None}
 
 
@@ -193,6 +197,22 @@ def workload_config(spec, inp, n):
                         f"{' +bias' if inp.b is not None else ''}, C={C}",
             "N": inp.N, "D": inp.D, "V": inp.V, "C": C, "dtype": spec.dtype,
             "labels": spec.label_dist, "parallelism": f"replicas{n}", "l2": l2}
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(flop_step: float, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of `flop_step` FLOP."""
+    return world * flop_step * steps / (ms_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------
@@ -272,8 +292,7 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error during warm-up: {binding.status_string(st)}")
 
-    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(dev)
@@ -296,12 +315,9 @@ def main():
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
     fwd_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
     bwd_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
-    t_max = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(t_max, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flop_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = weak_scaling_tflops(flop_step, args.steps, total_ms, world)
     peak_mib = torch.cuda.max_memory_allocated(dev) / 2**20
     launches = sum(n for _, n in prof.values())
 
@@ -330,11 +346,8 @@ def main():
             loss_host.copy_(loss, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = s0.elapsed_time(s1)
-        te = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        if world > 1:
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * flop_step * args.steps / (float(te.item()) * 1e-3) / 1e12,
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e = {"value": weak_scaling_tflops(flop_step, args.steps, e2e_ms, world),
                "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4,
                "loss": float(loss_host.item())}
 

@@ -26,7 +26,8 @@
  *    one call have the same type.  H and W must be 16-byte aligned and D a
  *    multiple of 8 (rows of 16-byte multiples, needed by the TMA engine).
  *  - labels are int64 [N]; mask is uint8 [N] (nonzero = position takes part)
- *    or NULL (all positions take part).
+ *    or NULL (all positions take part).  Arrays with N entries (H, labels,
+ *    m, logs, dH, idx) may be NULL when N == 0.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and runs asynchronously.  Argument errors are returned before
  *    anything is enqueued.  Errors found on the device (a supervised label

@@ -262,7 +262,7 @@ const char* flce_status_string(int status) {
 flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
                          int64_t N, int64_t V, int32_t* idx, int32_t* C_out, void* ws,
                          size_t ws_bytes, flce_stream stream) {
-  if (labels == nullptr || idx == nullptr || C_out == nullptr || ws == nullptr)
+  if ((N > 0 && (labels == nullptr || idx == nullptr)) || C_out == nullptr || ws == nullptr)
     return FLCE_ERR_NULL;
   if (N < 0 || N > kMaxN || V < 1 || V > kMaxV) return FLCE_ERR_SHAPE;
   if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
@@ -283,8 +283,8 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
                          const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
                          int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
                          size_t ws_bytes, flce_stream stream) {
-  if (H == nullptr || W == nullptr || labels == nullptr || loss == nullptr || m == nullptr ||
-      logs == nullptr || ws == nullptr)
+  if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr)) ||
+      W == nullptr || loss == nullptr || ws == nullptr)
     return FLCE_ERR_NULL;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
   if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
@@ -342,8 +342,9 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
                           int64_t V, int dtype, const float* m, const float* logs, float lambda,
                           const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
                           size_t ws_bytes, flce_stream stream) {
-  if (H == nullptr || W == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
-      dH == nullptr || dW == nullptr || ws == nullptr || (b != nullptr && db == nullptr))
+  if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
+                 dH == nullptr)) ||
+      W == nullptr || dW == nullptr || ws == nullptr || (b != nullptr && db == nullptr))
     return FLCE_ERR_NULL;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
   if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
