@@ -8,7 +8,7 @@ from lm_head_projection_supervised_b200 import binding
 from lm_head_projection_supervised_b200 import workloads as wl
 from oracle import flce_oracle as orc
 
-from _gpu_helpers import check_grad, check_loss, check_stats, to_device
+from _gpu_helpers import check_grad, check_loss, check_stats, logs_floor, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,7 @@ def full_check(inp, got):
     idx = ref["idx"]
     unsup = np.setdiff1d(np.arange(inp.N), idx)
     check_stats(got["m"], ref["m"], idx)
-    check_stats(got["logs"], ref["logs"], idx)
+    check_stats(got["logs"], ref["logs"], idx, floor=logs_floor(ref["m"][idx], inp.D))
     assert np.all(np.isneginf(got["m"][unsup])) and np.all(np.isneginf(got["logs"][unsup]))
     assert not got["dH"][unsup].any()
     check_grad("dH", got["dH"], ref["dH"])
@@ -192,12 +192,12 @@ def sampled_check(inp, got, n_rows=64, n_cols=192, full_stats=True):
     rows = np.sort(rng.choice(idx, size=min(n_rows, C), replace=False))
     r = orc.row_outputs(H64, W64, b64, inp.labels, inp.mask, -100, inp.lam, rows)
     check_stats(got["m"][rows], r["m"])
-    check_stats(got["logs"][rows], r["logs"])
+    check_stats(got["logs"][rows], r["logs"], floor=logs_floor(r["m"], inp.D))
     if full_stats:
         f = orc.forward(H64, W64, b64, inp.labels, inp.mask)
         check_loss(got["loss"], f["loss"])
         check_stats(got["m"], f["m"], idx)
-        check_stats(got["logs"], f["logs"], idx)
+        check_stats(got["logs"], f["logs"], idx, floor=logs_floor(f["m"][idx], inp.D))
         # vocabulary columns: the most frequent targets, the tail tile, random ids
         ys, counts = np.unique(inp.labels[idx], return_counts=True)
         hot = ys[np.argsort(-counts)[:32]]
