@@ -130,6 +130,42 @@ FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
                           float* dH, float* dW, float* db,
                           void* ws, size_t ws_bytes, flce_stream stream);
 
+/* Bytes of the fixed scratch buffer that flce_forward_noalloc() uses. */
+#define FLCE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * Forward that needs no workspace from the caller and allocates nothing.
+ * The pages have no counterpart of this entry point; it exists for callers.
+ *
+ * Some callers cannot provide device scratch memory: a plug-in running inside
+ * a host framework that owns every device allocation and allows no
+ * cudaMalloc outside its own pool, or code on a latency-critical path where
+ * cudaMalloc (which can synchronise the whole device) is not acceptable.
+ * This call computes the same loss, m and logs as flce_forward(), with its
+ * scratch in a FLCE_NOALLOC_SCRATCH_BYTES buffer compiled into the library
+ * (a static device array: every GPU that loads libflce.so holds it until the
+ * process exits).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.  The caller still passes all inputs and outputs.
+ *
+ *  - Size limit: flce_workspace_bytes(N, D, V, dtype) must not exceed
+ *    FLCE_NOALLOC_SCRATCH_BYTES (the small workload, N=2048 D=512 V=32000,
+ *    fits); larger problems get FLCE_ERR_WORKSPACE before anything is
+ *    enqueued.
+ *  - The first call on each device looks up the buffer's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls on a device share the one buffer, which keeps the previous
+ *    call's contents; the call clears what has to start at zero.  Calls that
+ *    overlap on the GPU (different streams or host threads) race on the
+ *    buffer and must be serialised by the caller.
+ *  - A device-side error (bad label, wait timeout) shows up as a NaN loss;
+ *    the error word lives in the shared buffer and is not returned.
+ */
+FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const void* b,
+                                          const int64_t* labels, const uint8_t* mask,
+                                          int64_t ignore_index, int64_t N, int64_t D, int64_t V,
+                                          int dtype, float* loss, float* m, float* logs,
+                                          flce_stream stream);
+
 /* Synchronises `stream`, then reads and returns the device error word of the
  * workspace (FLCE_OK when no device error was recorded by the last call). */
 FLCE_API flce_status flce_device_status(const void* ws, flce_stream stream);

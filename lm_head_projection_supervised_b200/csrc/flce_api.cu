@@ -542,3 +542,45 @@ flce_status flce_diag_profile_end(double* ms, int64_t* launches, int nkinds) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward with the library's own fixed scratch, for callers that cannot
+// allocate device memory (see flce_forward_noalloc in flce.h).
+// ---------------------------------------------------------------------------
+namespace {
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device pointer).
+flce_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FLCE_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FLCE_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FLCE_OK;
+}
+}  // namespace
+
+extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const void* b,
+                                            const int64_t* labels, const uint8_t* mask,
+                                            int64_t ignore_index, int64_t N, int64_t D,
+                                            int64_t V, int dtype, float* loss, float* m,
+                                            float* logs, flce_stream stream) {
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
+  if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
+  if (make_layout(N, D, V).total > FLCE_NOALLOC_SCRATCH_BYTES) return FLCE_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const flce_status st = noalloc_scratch(&scratch);
+  if (st != FLCE_OK) return st;
+  return flce_forward(H, W, b, labels, mask, ignore_index, N, D, V, dtype, loss, m, logs, scratch,
+                      FLCE_NOALLOC_SCRATCH_BYTES, stream);
+}
