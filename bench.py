@@ -353,23 +353,21 @@ def main():
 
     # roofline of the dominant kernel (largest share of device time)
     peaks, peak_src = load_peaks()
-    n_panels = -(-inp.V // 4096)
-    algo_flops = {  # algorithmic FLOP per launch
-        "fwd_gemm": 2.0 * C * inp.D * inp.V,
-        "grad_gemm": 2.0 * C * inp.D * inp.V / n_panels,
-        "wh_gemm": 4.0 * C * inp.D * inp.V / n_panels,
-    }
-    dom = max(algo_flops, key=lambda k: prof[k][0])
+    flop_per_step = {"fwd_gemm": 2.0 * C * inp.D * inp.V,   # algorithmic FLOP per step
+                     "bwd_gemm": 6.0 * C * inp.D * inp.V}
+    dom = max(flop_per_step, key=lambda k: prof[k][0])
     ms_tot, n_l = prof[dom]
     avg_ms = ms_tot / max(n_l, 1)
-    achieved = algo_flops[dom] / (avg_ms * 1e-3) / 1e12
+    flop_per_launch = flop_per_step[dom] * args.steps / max(n_l, 1)
+    achieved = flop_per_launch / (avg_ms * 1e-3) / 1e12
     # fp16 and bf16 share the dense tensor-core rate on this part
     peak = peaks.get("bf16_tflops_sustained")
     tb = ncu_traffic(dom)
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_note": f"sustained dense bf16, {peak_src} (kernel timed inside a long step)",
-                "traffic": tb, "avg_launch_ms": avg_ms, "launches": n_l,
+                "traffic": tb, "flop_per_launch": flop_per_launch, "avg_launch_ms": avg_ms,
+                "launches": n_l,
                 "kernel_share": {k: round(v[0] / max(1e-9, sum(x[0] for x in prof.values())), 4)
                                  for k, v in prof.items()}}
 

@@ -35,9 +35,11 @@
  *    non-finite statistic) are recorded in an error word inside the
  *    workspace, make the loss NaN, and are reported by flce_device_status().
  *  - The workspace is caller-allocated device memory of at least
- *    flce_workspace_bytes(N, D, V, dtype) bytes, 256-byte aligned.  Calls are
- *    stateless: the workspace carries nothing from one call to the next, but
- *    two calls in flight at the same time must not share one workspace.
+ *    flce_workspace_bytes(N, D, V, dtype) bytes, 256-byte aligned (the
+ *    forward alone uses only its leading part and accepts a shorter buffer;
+ *    the size returned is always enough).  Calls are stateless: the
+ *    workspace carries nothing from one call to the next, but two calls in
+ *    flight at the same time must not share one workspace.
  *  - Only the current CUDA device is used; it must be compute capability
  *    10.0 (sm_100a).
  */
@@ -147,10 +149,11 @@ FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
  * process exits).  It calls no cudaMalloc, cudaFree or other allocating
  * routine.  The caller still passes all inputs and outputs.
  *
- *  - Size limit: flce_workspace_bytes(N, D, V, dtype) must not exceed
- *    FLCE_NOALLOC_SCRATCH_BYTES (the small workload, N=2048 D=512 V=32000,
- *    fits); larger problems get FLCE_ERR_WORKSPACE before anything is
- *    enqueued.
+ *  - Size limit: the forward's scratch, about (N rounded up to 128) x
+ *    (2 D + 8 ceil(V / 256) + 16) bytes, must fit in FLCE_NOALLOC_SCRATCH_BYTES
+ *    (the small workload, N=2048 D=512 V=32000, needs about 4 MiB; the
+ *    16k-row, 248320-vocabulary case needs about 160 MiB and does not fit);
+ *    larger problems get FLCE_ERR_WORKSPACE before anything is enqueued.
  *  - The first call on each device looks up the buffer's device address with
  *    that device current; make that first call before any stream capture.
  *  - All calls on a device share the one buffer, which keeps the previous

@@ -228,7 +228,7 @@ def diag_timeout(limit_ns: int, device="cuda", stream=None) -> int:
     return int(lib().flce_device_status(_ptr(ws), _stream(stream)))
 
 
-PROFILE_KINDS = ("fwd_gemm", "grad_gemm", "wh_gemm", "aux")
+PROFILE_KINDS = ("fwd_gemm", "bwd_gemm", "plain_gemm", "aux")
 
 
 def profile_begin():

@@ -1,6 +1,6 @@
 // Memory-bound helper kernels around the tensor-core GEMMs: supervised-row
 // compaction, row gather, merge of per-tile statistics, the deterministic
-// loss mean, bias-gradient column sums and zeroing of unsupervised dH rows.
+// loss mean, bias-gradient column sums and the scatter of dH to all rows.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -24,11 +24,13 @@ __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8
 // every thread its output offset.  Labels outside [0, V) on supervised rows
 // set the label error bit and are clamped to 0 so later indexing stays in
 // range.  Unsupervised rows get m = log s = -inf when m_out is given.
+// pos (optional) is the inverse map: pos[i] = compact row of i, or -1.
 __global__ void __launch_bounds__(COMPACT_THREADS)
     compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
                    int64_t ignore, int64_t N, int64_t V, int* __restrict__ idx,
                    int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
-                   float* __restrict__ m_out, float* __restrict__ logs_out) {
+                   float* __restrict__ m_out, float* __restrict__ logs_out,
+                   int* __restrict__ pos) {
   __shared__ int warp_tot[COMPACT_THREADS / 32];
   const int t = threadIdx.x;
   const int64_t per = (N + COMPACT_THREADS - 1) / COMPACT_THREADS;
@@ -69,10 +71,14 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
       }
       idx[off] = static_cast<int>(i);
       if (y_c != nullptr) y_c[off] = static_cast<int>(y);
+      if (pos != nullptr) pos[i] = off;
       ++off;
-    } else if (m_out != nullptr) {
-      m_out[i] = -INFINITY;
-      logs_out[i] = -INFINITY;
+    } else {
+      if (m_out != nullptr) {
+        m_out[i] = -INFINITY;
+        logs_out[i] = -INFINITY;
+      }
+      if (pos != nullptr) pos[i] = -1;
     }
   }
   if (bad) atomicOr(err, kErrBitLabel);
@@ -210,18 +216,22 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// dH rows of unsupervised positions are zero (one warp per row).
-__global__ void zero_unsupervised_rows_kernel(const int64_t* __restrict__ labels,
-                                              const uint8_t* __restrict__ mask, int64_t ignore,
-                                              int64_t N, int64_t vec_per_row,
-                                              float4* __restrict__ dH) {
+// dH[i] = dH_c[pos[i]] for supervised rows, 0 for the others (one warp per
+// row, 16-byte vectors).
+__global__ void scatter_dh_kernel(const float4* __restrict__ dHc, const int* __restrict__ pos,
+                                  int64_t N, int64_t vec_per_row, float4* __restrict__ dH) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= N) return;
-  if (is_supervised(labels, mask, ignore, row)) return;
   const int lane = threadIdx.x & 31;
+  const int p = pos[row];
   float4* dst = dH + row * vec_per_row;
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
+  if (p >= 0) {
+    const float4* src = dHc + static_cast<int64_t>(p) * vec_per_row;
+    for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = src[k];
+  } else {
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
+  }
 }
 
 // Failure-path check: waits on a barrier nothing completes, with a short

@@ -4,13 +4,14 @@
 // Forward  (one stream, no host synchronisation):
 //   compact -> gather H_c -> gemm<fwd> (Z tiles + online (m, s) + target)
 //   -> merge partials per row -> fixed-order loss mean
-// Backward:
-//   compact -> gather H_c -> zero dH rows of unsupervised positions ->
-//   for each vocabulary panel of Vc columns:
-//       gemm<grad>  G panel = (p - onehot) * sigma, 16-bit, C x Vc
-//       gemm<wh>    dW[panel] = scale G^T H_c ;  dH[idx] (+)= scale G W[panel]
-//       bias_grad   db[panel] = scale * column sums of G   (bias only)
-//   with scale = lambda / (C sigma).
+// Backward, with P vocabulary panels of Vc columns and two panel buffers:
+//   compact -> gather H_c ->
+//   for L = 0 .. P:   gemm<bwd> with
+//                       grad units of panel L     (if L < P) -> buffer L % 2
+//                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 2
+//                     bias_grad of panel L (bias only, if L < P)
+//   -> scatter dH_c to dH (zero rows for unsupervised positions)
+//   with scale = lambda / (C sigma) applied in the dW / dH epilogues.
 #include <mutex>
 #include <vector>
 
@@ -26,30 +27,36 @@ namespace {
 constexpr int64_t kMaxN = int64_t(1) << 24;
 constexpr int64_t kMaxD = int64_t(1) << 16;
 constexpr int64_t kMaxV = int64_t(1) << 24;
-constexpr int64_t kPanelCols = 4096;  // vocabulary columns per gradient panel
+constexpr int64_t kPanelCols = 4096;   // vocabulary columns per gradient panel
 constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
+constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
 int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
 struct Layout {
-  size_t err, C, idx, yc, hc, part, tgt, loss_rows, gpanel, total;
-  int64_t Np, nvt, vc;
+  size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
+  size_t pos, dhc, gpanel[2], total;
+  int64_t Np, nvt, vc, panels;
 };
 
-// Workspace carve-up.  The error word sits at offset 0 for every size.
+// Workspace carve-up.  The control block (error word, then one work counter
+// per GEMM launch) sits at offset 0 for every size.  The regions the forward
+// pass uses come first (fwd_total bytes); the backward's follow.
 Layout make_layout(int64_t N, int64_t D, int64_t V) {
   Layout L{};
   L.Np = roundup64(N > 0 ? N : 1, BM);
   L.nvt = cdiv64(V, BN);
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
+  L.panels = cdiv64(V, L.vc);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += static_cast<size_t>(roundup64(static_cast<int64_t>(bytes), 1024));
     return o;
   };
-  L.err = take(256);
+  L.ctrl_bytes = kCounterOffset + 4 * static_cast<size_t>(L.panels + 2);
+  L.ctrl = take(L.ctrl_bytes);
   L.C = take(256);
   L.idx = take(static_cast<size_t>(L.Np) * 4);
   L.yc = take(static_cast<size_t>(L.Np) * 4);
@@ -57,7 +64,11 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.part = take(static_cast<size_t>(L.Np) * L.nvt * 8);
   L.tgt = take(static_cast<size_t>(L.Np) * 4);
   L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
-  L.gpanel = take(static_cast<size_t>(L.Np) * L.vc * 2);
+  L.fwd_total = off;
+  L.pos = take(static_cast<size_t>(L.Np) * 4);
+  L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
+  L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.vc * 2);
+  L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.vc * 2);
   L.total = off;
   return L;
 }
@@ -86,9 +97,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major 16-bit matrix [outer x inner] with row pitch
-// `pitch` bytes, 128-byte swizzle, zero fill outside the extents.
-bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+enum MapType { kMapBF16, kMapFP16, kMapF32 };
+
+// 2-D map over a row-major matrix [outer x inner] with row pitch `pitch`
+// bytes, 128-byte swizzle, zero fill outside the extents.
+bool make_map(CUtensorMap* m, const void* base, MapType t, uint64_t inner, uint64_t outer,
               uint64_t pitch, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
@@ -96,10 +109,12 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint6
   const cuuint64_t strides[1] = {pitch};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
-  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-            const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUtensorMapDataType dt = t == kMapBF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : t == kMapFP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---- per-device set-up
@@ -128,9 +143,7 @@ flce_status device_setup(DevInfo* out) {
       const int bytes = static_cast<int>(GEMM_SMEM_BYTES);
       if (cudaFuncSetAttribute(flce_gemm_kernel<kModeFwd>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-          cudaFuncSetAttribute(flce_gemm_kernel<kModeGrad>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
-          cudaFuncSetAttribute(flce_gemm_kernel<kModeWH>,
+          cudaFuncSetAttribute(flce_gemm_kernel<kModeBwd>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
           cudaFuncSetAttribute(flce_gemm_kernel<kModePlain>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
@@ -157,7 +170,7 @@ std::mutex g_prof_mu;
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof;
 
-enum ProfKind : int { kProfFwd = 0, kProfGrad = 1, kProfWH = 2, kProfAux = 3 };
+enum ProfKind : int { kProfFwd = 0, kProfBwd = 1, kProfPlain = 2, kProfAux = 3 };
 
 // Runs `launch` (which enqueues one kernel on s); when profiling is on, the
 // launch is bracketed by two events on the same stream.
@@ -188,8 +201,7 @@ template <int MODE>
 cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int sms, cudaStream_t s) {
   if (units_upper <= 0) return cudaSuccess;
   const int grid = static_cast<int>(units_upper < sms ? units_upper : sms);
-  const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeGrad ? kProfGrad
-                 : MODE == kModeWH ? kProfWH : kProfAux;
+  const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeBwd ? kProfBwd : kProfPlain;
   return timed_launch(kind, s, [&] {
     flce_gemm_kernel<MODE><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, s>>>(a);
   });
@@ -197,38 +209,51 @@ cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int sms, cudaStr
 
 struct WsPtrs {
   uint32_t* err;
+  int* counters;
   int* C;
   int* idx;
   int* yc;
+  int* pos;
   uint16_t* hc;
   float2* part;
   float* tgt;
   float* loss_rows;
-  uint16_t* gpanel;
+  float* dhc;
+  uint16_t* gpanel[2];
 };
 
 WsPtrs carve(void* ws, const Layout& L) {
   uint8_t* w = static_cast<uint8_t*>(ws);
-  return WsPtrs{reinterpret_cast<uint32_t*>(w + L.err), reinterpret_cast<int*>(w + L.C),
-                reinterpret_cast<int*>(w + L.idx),       reinterpret_cast<int*>(w + L.yc),
-                reinterpret_cast<uint16_t*>(w + L.hc),   reinterpret_cast<float2*>(w + L.part),
-                reinterpret_cast<float*>(w + L.tgt),     reinterpret_cast<float*>(w + L.loss_rows),
-                reinterpret_cast<uint16_t*>(w + L.gpanel)};
+  WsPtrs p;
+  p.err = reinterpret_cast<uint32_t*>(w + L.ctrl);
+  p.counters = reinterpret_cast<int*>(w + L.ctrl + kCounterOffset);
+  p.C = reinterpret_cast<int*>(w + L.C);
+  p.idx = reinterpret_cast<int*>(w + L.idx);
+  p.yc = reinterpret_cast<int*>(w + L.yc);
+  p.pos = reinterpret_cast<int*>(w + L.pos);
+  p.hc = reinterpret_cast<uint16_t*>(w + L.hc);
+  p.part = reinterpret_cast<float2*>(w + L.part);
+  p.tgt = reinterpret_cast<float*>(w + L.tgt);
+  p.loss_rows = reinterpret_cast<float*>(w + L.loss_rows);
+  p.dhc = reinterpret_cast<float*>(w + L.dhc);
+  p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
+  p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
+  return p;
 }
 
-// compaction + gather of the supervised rows into the workspace
+// control block reset + compaction + gather of the supervised rows
 flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
                      int64_t N, int64_t D, int64_t V, const Layout& L, const WsPtrs& p,
-                     float* m_out, float* logs_out, cudaStream_t s) {
-  FLCE_CK(cudaMemsetAsync(p.err, 0, 256, s));
+                     float* m_out, float* logs_out, int* pos, cudaStream_t s) {
+  FLCE_CK(cudaMemsetAsync(p.err, 0, L.ctrl_bytes, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, p.idx, p.yc, p.C,
-                                               p.err, m_out, logs_out);
+                                                 p.err, m_out, logs_out, pos);
   }));
   const int64_t vec = D / 8;
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     gather_rows_kernel<<<static_cast<unsigned>(cdiv64(L.Np, 8)), 256, 0, s>>>(
-      static_cast<const uint4*>(H), p.idx, p.C, L.Np, vec, reinterpret_cast<uint4*>(p.hc));
+        static_cast<const uint4*>(H), p.idx, p.C, L.Np, vec, reinterpret_cast<uint4*>(p.hc));
   }));
   return FLCE_OK;
 }
@@ -273,9 +298,10 @@ flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ign
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
-  compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, idx, nullptr,
-                                               C_out, err, nullptr, nullptr);
-  FLCE_CK(cudaGetLastError());
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, idx, nullptr,
+                                                 C_out, err, nullptr, nullptr, nullptr);
+  }));
   return FLCE_OK;
 }
 
@@ -292,28 +318,29 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
       !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) || !aligned(loss, 4))
     return FLCE_ERR_ALIGN;
   const Layout L = make_layout(N, D, V);
-  if (ws_bytes < L.total) return FLCE_ERR_WORKSPACE;
+  if (ws_bytes < L.fwd_total) return FLCE_ERR_WORKSPACE;
   DevInfo di;
   flce_status st = device_setup(&di);
   if (st != FLCE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsPtrs p = carve(ws, L);
   const bool bf16 = dtype == FLCE_BF16;
+  const MapType mt = bf16 ? kMapBF16 : kMapFP16;
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, s);
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, nullptr, s);
   if (st != FLCE_OK) return st;
 
   GemmArgs a{};
-  if (!make_map(&a.tmA[0], p.hc, bf16, D, L.Np, D * 2, BK, BM) ||
-      !make_map(&a.tmB[0], W, bf16, D, V, D * 2, BK, BN))
+  if (!make_map(&a.tmA[0], p.hc, mt, D, L.Np, D * 2, BK, BM) ||
+      !make_map(&a.tmB[0], W, mt, D, V, D * 2, BK, BN))
     return FLCE_ERR_CUDA;
   a.is_bf16 = bf16;
   a.C_dev = p.C;
+  a.counter = p.counters;
   a.ncols = static_cast<int>(V);
   a.K = static_cast<int>(D);
   a.D = static_cast<int>(D);
   a.V = static_cast<int>(V);
-  a.vp = 0;
   a.y_c = p.yc;
   a.idx = p.idx;
   a.bias = static_cast<const uint16_t*>(b);
@@ -326,10 +353,10 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
   if (N > 0) {
     const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
-    merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
-        p.loss_rows, p.err);
-  }));
+      merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+          p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
+          p.loss_rows, p.err);
+    }));
   }
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     loss_mean_kernel<<<1, 1024, 0, s>>>(p.loss_rows, p.C, p.err, loss);
@@ -360,46 +387,60 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsPtrs p = carve(ws, L);
   const bool bf16 = dtype == FLCE_BF16;
+  const MapType mt = bf16 ? kMapBF16 : kMapFP16;
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, s);
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, p.pos, s);
   if (st != FLCE_OK) return st;
-  if (N > 0) {
-    FLCE_CK(timed_launch(kProfAux, s, [&] {
-    zero_unsupervised_rows_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
-        labels, mask, ignore_index, N, D / 4, reinterpret_cast<float4*>(dH));
-  }));
-  }
 
-  // operand maps that do not depend on the panel
-  CUtensorMap hcK, wK, hcMN, wMN;
-  if (!make_map(&hcK, p.hc, bf16, D, L.Np, D * 2, BK, BM) ||
-      !make_map(&wK, W, bf16, D, V, D * 2, BK, BN) ||
-      !make_map(&hcMN, p.hc, bf16, D, L.Np, D * 2, 64, BK) ||
-      !make_map(&wMN, W, bf16, D, V, D * 2, 64, BK))
+  // maps that do not depend on the panel
+  CUtensorMap hcK, wK, hcMN, wMN, dwMap, dhMap;
+  if (!make_map(&hcK, p.hc, mt, D, L.Np, D * 2, BK, BM) ||
+      !make_map(&wK, W, mt, D, V, D * 2, BK, BN) ||
+      !make_map(&hcMN, p.hc, mt, D, L.Np, D * 2, 64, BK) ||
+      !make_map(&wMN, W, mt, D, V, D * 2, 64, BK) ||
+      !make_map(&dwMap, dW, kMapF32, D, V, D * 4, 32, BM) ||
+      !make_map(&dhMap, p.dhc, kMapF32, D, L.Np, D * 4, 32, BM))
     return FLCE_ERR_CUDA;
 
   const int64_t nT_max = cdiv64(N, BM);
   const int64_t nD = cdiv64(D, BN);
-  for (int64_t vp = 0; vp < V; vp += L.vc) {
-    const int64_t w = (V - vp) < L.vc ? (V - vp) : L.vc;
-    CUtensorMap gK, gMN;
-    if (!make_map(&gK, p.gpanel, bf16, w, L.Np, L.vc * 2, 64, BM) ||
-        !make_map(&gMN, p.gpanel, bf16, w, L.Np, L.vc * 2, 64, BK))
-      return FLCE_ERR_CUDA;
+  for (int64_t Lp = 0; Lp <= L.panels; ++Lp) {
+    const bool has_g = Lp < L.panels;
+    const bool has_wh = Lp > 0;
+    const int64_t vp_g = Lp * L.vc;
+    const int64_t w_g = has_g ? ((V - vp_g) < L.vc ? (V - vp_g) : L.vc) : 0;
+    const int64_t vp_wh = (Lp - 1) * L.vc;
+    const int64_t w_wh = has_wh ? ((V - vp_wh) < L.vc ? (V - vp_wh) : L.vc) : 0;
 
     GemmArgs a{};
-    a.tmA[0] = hcK;
-    a.tmB[0] = wK;
-    a.tmOut = gK;
+    a.tmA[kClsGrad] = hcK;
+    a.tmB[kClsGrad] = wK;
+    a.tmB[kClsDW] = hcMN;
+    a.tmB[kClsDH] = wMN;
+    a.tmDW = dwMap;
+    a.tmDH = dhMap;
+    if (has_g && !make_map(&a.tmG, p.gpanel[Lp & 1], mt, w_g, L.Np, L.vc * 2, 64, BM))
+      return FLCE_ERR_CUDA;
+    if (has_wh) {
+      const uint16_t* gp = p.gpanel[(Lp - 1) & 1];
+      if (!make_map(&a.tmA[kClsDW], gp, mt, w_wh, L.Np, L.vc * 2, 64, BK) ||
+          !make_map(&a.tmA[kClsDH], gp, mt, w_wh, L.Np, L.vc * 2, BK, BM))
+        return FLCE_ERR_CUDA;
+    }
     a.is_bf16 = bf16;
     a.C_dev = p.C;
-    a.ncols = static_cast<int>(w);
-    a.K = static_cast<int>(D);
+    a.counter = p.counters + 1 + Lp;
     a.D = static_cast<int>(D);
     a.V = static_cast<int>(V);
-    a.vp = static_cast<int>(vp);
+    a.has_wh = has_wh;
+    a.vp_wh = static_cast<int>(vp_wh);
+    a.w_wh = static_cast<int>(w_wh);
+    a.dh_accumulate = Lp > 1;
+    a.has_g = has_g;
+    a.vp_g = static_cast<int>(vp_g);
+    a.w_g = static_cast<int>(w_g);
     a.y_c = p.yc;
     a.idx = p.idx;
     a.bias = static_cast<const uint16_t*>(b);
@@ -407,38 +448,28 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
     a.logs_saved = logs;
     a.log2_sigma = log2_sigma;
     a.sigma = sigma;
+    a.lam = lambda;
+    a.lam_dev = lambda_dev;
+    a.inv_sigma = 1.f / sigma;
     a.err = p.err;
-    FLCE_CK(launch_gemm<kModeGrad>(a, nT_max * cdiv64(w, BN), di.sms, s));
+    const int64_t units = (has_wh ? cdiv64(w_wh, BM) * nD + nT_max * nD : 0) +
+                          (has_g ? nT_max * cdiv64(w_g, BN) : 0);
+    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.sms, s));
 
-    GemmArgs c{};
-    c.tmA[0] = gMN;   // dW: A = G panel, vocabulary-major
-    c.tmB[0] = hcMN;  //     B = H_c, hidden-major
-    c.tmA[1] = gK;    // dH: A = G panel, K = vocabulary
-    c.tmB[1] = wMN;   //     B = W[panel], hidden-major
-    c.is_bf16 = bf16;
-    c.C_dev = p.C;
-    c.K = static_cast<int>(w);
-    c.D = static_cast<int>(D);
-    c.V = static_cast<int>(V);
-    c.vp = static_cast<int>(vp);
-    c.nVb = static_cast<int>(cdiv64(w, BM));
-    c.nDW = static_cast<int>(cdiv64(w, BM) * nD);
-    c.idx = p.idx;
-    c.lam = lambda;
-    c.lam_dev = lambda_dev;
-    c.inv_sigma = 1.f / sigma;
-    c.dW = dW;
-    c.dH = dH;
-    c.err = p.err;
-    FLCE_CK(launch_gemm<kModeWH>(c, c.nDW + nT_max * nD, di.sms, s));
-
-    if (b != nullptr) {
+    if (b != nullptr && has_g) {
+      const uint16_t* gp = p.gpanel[Lp & 1];
       FLCE_CK(timed_launch(kProfAux, s, [&] {
-    bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w, 64)), 256, 0, s>>>(
-          p.gpanel, L.vc, static_cast<int>(w), p.C, lambda, lambda_dev, 1.f / sigma, bf16 ? 1 : 0,
-          static_cast<int>(vp), db);
-  }));
+        bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w_g, 64)), 256, 0, s>>>(
+            gp, L.vc, static_cast<int>(w_g), p.C, lambda, lambda_dev, 1.f / sigma, bf16 ? 1 : 0,
+            static_cast<int>(vp_g), db);
+      }));
     }
+  }
+  if (N > 0) {
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      scatter_dh_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(p.dhc), p.pos, N, D / 4, reinterpret_cast<float4*>(dH));
+    }));
   }
   return FLCE_OK;
 }
@@ -470,22 +501,23 @@ flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, 
   const flce_status st = device_setup(&di);
   if (st != FLCE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == FLCE_BF16;
+  const MapType mt = dtype == FLCE_BF16 ? kMapBF16 : kMapFP16;
   GemmArgs a{};
-  const bool okA = a_mn ? make_map(&a.tmA[0], A, bf16, M, K, M * 2, 64, BK)
-                        : make_map(&a.tmA[0], A, bf16, K, M, K * 2, BK, BM);
-  const bool okB = b_mn ? make_map(&a.tmB[0], B, bf16, N, K, N * 2, 64, BK)
-                        : make_map(&a.tmB[0], B, bf16, K, N, K * 2, BK, BN);
+  const bool okA = a_mn ? make_map(&a.tmA[0], A, mt, M, K, M * 2, 64, BK)
+                        : make_map(&a.tmA[0], A, mt, K, M, K * 2, BK, BM);
+  const bool okB = b_mn ? make_map(&a.tmB[0], B, mt, N, K, N * 2, 64, BK)
+                        : make_map(&a.tmB[0], B, mt, K, N, K * 2, BK, BN);
   if (!okA || !okB) return FLCE_ERR_CUDA;
   a.a_mn = a_mn ? 1 : 0;
   a.b_mn = b_mn ? 1 : 0;
-  a.is_bf16 = bf16;
+  a.is_bf16 = dtype == FLCE_BF16;
   a.M = static_cast<int>(M);
   a.ncols = static_cast<int>(N);
   a.K = static_cast<int>(K);
   a.out = out;
   a.scale = scale;
   a.err = static_cast<uint32_t*>(ws);
+  a.counter = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kCounterOffset);
   FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
   FLCE_CK(launch_gemm<kModePlain>(a, cdiv64(M, BM) * cdiv64(N, BN), di.sms, s));
   return FLCE_OK;
@@ -500,8 +532,9 @@ flce_status flce_diag_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, flce
   if (st != FLCE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
-  timeout_probe_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(ws), limit_ns);
-  FLCE_CK(cudaGetLastError());
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    timeout_probe_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(ws), limit_ns);
+  }));
   return FLCE_OK;
 }
 
@@ -577,7 +610,7 @@ extern "C" flce_status flce_forward_noalloc(const void* H, const void* W, const 
                                             float* logs, flce_stream stream) {
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
   if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
-  if (make_layout(N, D, V).total > FLCE_NOALLOC_SCRATCH_BYTES) return FLCE_ERR_WORKSPACE;
+  if (make_layout(N, D, V).fwd_total > FLCE_NOALLOC_SCRATCH_BYTES) return FLCE_ERR_WORKSPACE;
   void* scratch = nullptr;
   const flce_status st = noalloc_scratch(&scratch);
   if (st != FLCE_OK) return st;

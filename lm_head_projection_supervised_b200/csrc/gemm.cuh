@@ -1,12 +1,13 @@
 // Persistent, warp-specialised tcgen05 GEMM for sm_100a with the fused
 // epilogues of exact linear cross-entropy.
 //
-// One CTA per SM.  Warp 0 (one lane) streams operand tiles with TMA into a
-// STAGES-deep shared-memory ring; warp 1 (one lane) issues
-// tcgen05.mma.kind::f16 (M=128, N=256, K=16) into one of two 128x256 f32
-// accumulators in TMEM (512 columns); warps 4..7 read the finished
-// accumulator back with tcgen05.ld (thread = TMEM lane = tile row) and run
-// the epilogue while the next tile accumulates in the other buffer.
+// One CTA per SM.  Warp 0 (one lane) takes work units from a global counter
+// (longest units first), publishes each unit id through a small shared-memory
+// ring, and streams the unit's operand tiles with TMA into a STAGES-deep
+// ring; warp 1 (one lane) issues tcgen05.mma.kind::f16 (M=128, N=256, K=16)
+// into one of two 128x256 f32 accumulators in TMEM (512 columns); warps 4..7
+// read a finished accumulator with tcgen05.ld (thread = TMEM lane = tile
+// row) and run the epilogue while the next unit accumulates in the other.
 //
 // Modes (one launch = one mode):
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
@@ -14,16 +15,19 @@
 //              captures the target logit from the tile that holds it
 //              ("分块交叉熵" page, §02), writing one (m, s) partial per row
 //              and vocabulary tile.
-//   kModeGrad  the same tile recomputed for the backward; the epilogue
-//              rebuilds p = exp((Z - m) - log s) from the saved statistics,
-//              subtracts the one-hot target (§04), rounds to the 16-bit
-//              input type, stages the tile in shared memory and stores it
-//              with TMA into a C x Vc gradient panel.
-//   kModeWH    one launch with two unit classes fed by the same panel:
-//              class 0: dW[panel rows] = G_panel^T H_c   (K = C)
-//              class 1: dH[idx] (+)= G_panel W[panel]    (K = panel width)
-//              every output tile is owned by one unit, so both are
-//              deterministic; dH accumulates over panels in panel order.
+//   kModeBwd   three unit classes in one launch, with no dependency between
+//              them:
+//              class 2 (grad): the tile of vocabulary panel p recomputed; the
+//                 epilogue rebuilds p = exp((Z - m) - log s) from the saved
+//                 statistics, subtracts the one-hot target (§04), rounds to
+//                 the 16-bit input type, stages 128 x 64 boxes in shared
+//                 memory and stores them with TMA into gradient buffer p % 2;
+//              class 0 (dW): dW[panel p-1 rows] = G^T H_c  (K = C), stored by TMA;
+//              class 1 (dH): dH_c (+)= G W[panel p-1]      (K = panel width),
+//                 stored (first panel) or added with a TMA reduction (later
+//                 panels).
+//              Every output tile is owned by one unit and panels run in
+//              order, so dW, dH and the panel buffers are deterministic.
 //   kModePlain diagnostic: out = scale * A B^T with a plain store.
 #pragma once
 
@@ -38,54 +42,58 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
+constexpr int UQ = 4;                            // depth of the unit-id ring
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KiB
 constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;  // 32 KiB
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;   // 8 KiB: 64 MN-elements x 64 K rows
-constexpr uint32_t STG_BYTES = BM * 64 * 2;      // 16 KiB: 128 rows x 64 16-bit columns
+constexpr uint32_t STG_BYTES = BM * 128;         // 16 KiB: 128 rows x 128 bytes
 constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr size_t GEMM_SMEM_BYTES =
-    1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 2 * STG_BYTES + 256;
+    1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 2 * STG_BYTES + 512;
 
-enum GemmMode : int { kModeFwd = 0, kModeGrad = 1, kModeWH = 2, kModePlain = 3 };
+enum GemmMode : int { kModeFwd = 0, kModeBwd = 1, kModePlain = 2 };
+enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
 
 struct GemmArgs {
-  CUtensorMap tmA[2];  // A operand map of unit class 0 / 1
-  CUtensorMap tmB[2];  // B operand map of unit class 0 / 1
-  CUtensorMap tmOut;   // gradient panel store map (kModeGrad)
-  int a_mn;            // kModePlain: A is MN-major
-  int b_mn;            // kModePlain: B is MN-major
+  CUtensorMap tmA[3];  // A operand map per unit class (fwd / plain use [0])
+  CUtensorMap tmB[3];  // B operand map per unit class
+  CUtensorMap tmG;     // bwd: store map of the gradient panel being produced
+  CUtensorMap tmDW;    // bwd: fp32 dW [V x D], 128 x 32 boxes
+  CUtensorMap tmDH;    // bwd: fp32 compact dH [Np x D], 128 x 32 boxes
+  int a_mn;            // plain: A is MN-major
+  int b_mn;            // plain: B is MN-major
   int is_bf16;
-  const int* C_dev;    // supervised-row count (device); unused in kModePlain
-  int M;               // kModePlain: rows of out
-  int ncols;           // fwd: V; grad: panel width; plain: N
-  int K;               // fwd/grad: D; plain: K; wh: panel width
+  const int* C_dev;    // supervised-row count (device); unused in plain mode
+  int* counter;        // work-unit counter of this launch, zero at launch
+  int M;               // plain: rows of out
+  int ncols;           // fwd: V; plain: N
+  int K;               // fwd: D; plain: K
   int D;
   int V;
-  int vp;              // first vocabulary id of the panel (grad, wh); 0 for fwd
-  int nDW;             // wh: number of dW units
-  int nVb;             // wh: 128-row blocks in the panel
+  // bwd: the dW/dH part works on panel [vp_wh, vp_wh + w_wh), the gradient
+  // part produces panel [vp_g, vp_g + w_g)
+  int has_wh, vp_wh, w_wh, dh_accumulate;
+  int has_g, vp_g, w_g;
   // epilogue data
-  const int* y_c;              // compact labels
-  const int* idx;              // compact row -> original row
-  const uint16_t* bias;        // 16-bit bias [V] or null
-  float2* part;                // fwd: (m, s) partials [rows][part_ld]
+  const int* y_c;          // compact labels
+  const int* idx;          // compact row -> original row
+  const uint16_t* bias;    // 16-bit bias [V] or null
+  float2* part;            // fwd: (m, s) partials [rows][part_ld]
   int part_ld;
-  float* tgt;                  // fwd: target logits [rows]
-  const float* m_saved;        // grad: saved statistics [N]
+  float* tgt;              // fwd: target logits [rows]
+  const float* m_saved;    // bwd: saved statistics [N]
   const float* logs_saved;
-  float log2_sigma;            // grad: the panel holds (p - onehot) * sigma
+  float log2_sigma;        // bwd: the panel holds (p - onehot) * sigma
   float sigma;
-  float lam;                   // wh: upstream gradient
-  const float* lam_dev;        //     (device copy, overrides lam when set)
+  float lam;               // bwd: upstream gradient
+  const float* lam_dev;    //      (device copy, overrides lam when set)
   float inv_sigma;
-  float* dW;
-  float* dH;
-  float* out;                  // plain
-  float scale;                 // plain
+  float* out;              // plain
+  float scale;             // plain
   uint32_t* err;
 };
 
@@ -98,52 +106,94 @@ struct Unit {
 
 __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
 
-template <int MODE>
-__device__ __forceinline__ int num_units(const GemmArgs& g, int C) {
-  if (MODE == kModeWH) return g.nDW + cdiv_i(C, BM) * cdiv_i(g.D, BN);
-  const int rows = (MODE == kModePlain) ? g.M : C;
-  return cdiv_i(rows, BM) * cdiv_i(g.ncols, BN);
+// Work units of one launch, grouped by class and ordered longest-first.
+// Fields are scalars (no arrays) so that they stay in registers.
+struct UnitSpace {
+  int n0, n1, n2;     // units per class
+  int k0, k1, k2;     // K-blocks per unit of each class
+  int o0, o1, o2;     // classes, longest first
+  int total;
+};
+
+__device__ __forceinline__ int pick3(int c, int a, int b, int d) {
+  return c == 0 ? a : (c == 1 ? b : d);
 }
 
-// Unit u -> tile.  Token (row) tiles vary fastest so that CTAs running at the
-// same time share the W / G columns they read through L2.
 template <int MODE>
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& g, int C, int u) {
+__device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
+  UnitSpace s;
+  if (MODE == kModeBwd) {
+    const int nT = cdiv_i(C, BM), nD = cdiv_i(g.D, BN);
+    s.n0 = g.has_wh ? cdiv_i(g.w_wh, BM) * nD : 0;       // dW
+    s.n1 = g.has_wh ? nT * nD : 0;                       // dH
+    s.n2 = g.has_g ? nT * cdiv_i(g.w_g, BN) : 0;         // grad
+    s.k0 = cdiv_i(C, BK);
+    s.k1 = cdiv_i(g.w_wh, BK);
+    s.k2 = cdiv_i(g.D, BK);
+    // order the three classes by K-blocks per unit, longest first (stable)
+    int a = 0, b = 1, c = 2;
+    int ka = s.k0, kb = s.k1, kc = s.k2;
+    if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
+    if (kb < kc) { int t = b; b = c; c = t; t = kb; kb = kc; kc = t; }
+    if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
+    s.o0 = a;
+    s.o1 = b;
+    s.o2 = c;
+    s.total = s.n0 + s.n1 + s.n2;
+  } else {
+    const int rows = (MODE == kModePlain) ? g.M : C;
+    s.n0 = cdiv_i(rows, BM) * cdiv_i(g.ncols, BN);
+    s.n1 = s.n2 = 0;
+    s.k0 = cdiv_i(g.K, BK);
+    s.k1 = s.k2 = 0;
+    s.o0 = 0;
+    s.o1 = 1;
+    s.o2 = 2;
+    s.total = s.n0;
+  }
+  return s;
+}
+
+// Unit u -> tile.  Row (token) tiles vary fastest so that units running at
+// the same time share the W / G columns they read through L2.
+template <int MODE>
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& s, int C, int u) {
   Unit un;
-  if (MODE == kModeWH) {
-    if (u < g.nDW) {
-      un.cls = 0;
-      un.m0 = (u % g.nVb) * BM;
-      un.n0 = (u / g.nVb) * BN;
-      un.nk = cdiv_i(C, BK);
-    } else {
-      const int v = u - g.nDW;
-      const int nT = cdiv_i(C, BM);
-      un.cls = 1;
-      un.m0 = (v % nT) * BM;
-      un.n0 = (v / nT) * BN;
-      un.nk = cdiv_i(g.K, BK);
+  int cls = s.o0;
+  const int c0 = pick3(s.o0, s.n0, s.n1, s.n2);
+  if (u >= c0) {
+    u -= c0;
+    cls = s.o1;
+    const int c1 = pick3(s.o1, s.n0, s.n1, s.n2);
+    if (u >= c1) {
+      u -= c1;
+      cls = s.o2;
     }
+  }
+  un.cls = cls;
+  un.nk = pick3(cls, s.k0, s.k1, s.k2);
+  if (MODE == kModeBwd && cls == kClsDW) {
+    const int nVb = cdiv_i(g.w_wh, BM);
+    un.m0 = (u % nVb) * BM;
+    un.n0 = (u / nVb) * BN;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
     const int nT = cdiv_i(rows, BM);
-    un.cls = 0;
     un.m0 = (u % nT) * BM;
     un.n0 = (u / nT) * BN;
-    un.nk = cdiv_i(g.K, BK);
   }
   return un;
 }
 
 template <int MODE>
 __device__ __forceinline__ bool unit_a_mn(const GemmArgs& g, const Unit& un) {
-  if (MODE == kModeWH) return un.cls == 0;
+  if (MODE == kModeBwd) return un.cls == kClsDW;
   if (MODE == kModePlain) return g.a_mn != 0;
   return false;
 }
 template <int MODE>
 __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
-  if (MODE == kModeWH) return true;
+  if (MODE == kModeBwd) return un.cls != kClsGrad;
   if (MODE == kModePlain) return g.b_mn != 0;
   return false;
 }
@@ -152,26 +202,26 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
 template <int MODE>
 __device__ __forceinline__ void issue_stage_loads(const GemmArgs& g, const Unit& un, int kb,
                                                   uint32_t sa, uint32_t sb, uint64_t* bar) {
-  const CUtensorMap* tA = &g.tmA[un.cls];
-  const CUtensorMap* tB = &g.tmB[un.cls];
+  const int mapi = (MODE == kModeBwd) ? un.cls : 0;
+  const CUtensorMap* tA = &g.tmA[mapi];
+  const CUtensorMap* tB = &g.tmB[mapi];
   const int k0 = kb * BK;
-  const bool a_mn = unit_a_mn<MODE>(g, un);
-  const bool b_mn = unit_b_mn<MODE>(g, un);
   // A: 128 rows x 64 k
-  if (a_mn) {
+  if (unit_a_mn<MODE>(g, un)) {
     tma_load_2d(sa, tA, bar, un.m0, k0);
     tma_load_2d(sa + MN_BOX_BYTES, tA, bar, un.m0 + 64, k0);
   } else {
     tma_load_2d(sa, tA, bar, k0, un.m0);
   }
-  // B: 256 rows x 64 k.  In the wh mode's dH class the k index is a vocabulary
-  // id of the panel; in fwd/grad the row index is.
-  const int kB = (MODE == kModeWH && un.cls == 1) ? g.vp + k0 : k0;
-  if (b_mn) {
+  // B: 256 rows x 64 k
+  if (unit_b_mn<MODE>(g, un)) {
+    // dH: the k index is a vocabulary id of the panel
+    const int kB = (MODE == kModeBwd && un.cls == kClsDH) ? g.vp_wh + k0 : k0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) tma_load_2d(sb + j * MN_BOX_BYTES, tB, bar, un.n0 + 64 * j, kB);
   } else {
-    const int nrow = (MODE == kModeFwd || MODE == kModeGrad) ? g.vp + un.n0 : un.n0;
+    // fwd / grad: the row index is a vocabulary id
+    const int nrow = (MODE == kModeBwd) ? g.vp_g + un.n0 : un.n0;
     tma_load_2d(sb, tB, bar, k0, nrow);
   }
 }
@@ -312,6 +362,21 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   }
 }
 
+// Writes 128 bytes of this thread's row into a 128-row staging box laid out
+// as the 128-byte-swizzled TMA box (16-byte chunk j of row r sits at chunk
+// j ^ (r & 7)).
+template <int NW>
+__device__ __forceinline__ void stage_row128(uint8_t* stg, int r, int chunk0,
+                                             const uint32_t (&w)[NW]) {
+  uint8_t* rowp = stg + r * 128;
+#pragma unroll
+  for (int j = 0; j < NW / 4; ++j) {
+    const int c = (chunk0 + j) ^ (r & 7);
+    *reinterpret_cast<uint4*>(rowp + c * 16) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
@@ -327,10 +392,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* done_bar = tempty + 2;
+  uint64_t* uq_full = tempty + 2;
+  uint64_t* uq_empty = uq_full + UQ;
+  uint64_t* done_bar = uq_empty + UQ;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* decision = abort_flag + 1;  // [2]
+  volatile int* s_unit = decision + 2;      // [UQ]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -344,6 +412,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], NUM_EPI_THREADS);
     }
+    for (int q = 0; q < UQ; ++q) {
+      mbar_init(&uq_full[q], 1);
+      mbar_init(&uq_empty[q], 1 + NUM_EPI_THREADS / 32);  // MMA lane + one lane per epilogue warp
+    }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     decision[0] = 0;
@@ -351,13 +423,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&g.tmA[0]);
-    tma_prefetch_map(&g.tmB[0]);
-    if (MODE == kModeWH) {
-      tma_prefetch_map(&g.tmA[1]);
-      tma_prefetch_map(&g.tmB[1]);
+    const int nmaps = (MODE == kModeBwd) ? 3 : 1;
+    for (int i = 0; i < nmaps; ++i) {
+      tma_prefetch_map(&g.tmA[i]);
+      tma_prefetch_map(&g.tmB[i]);
     }
-    if (MODE == kModeGrad) tma_prefetch_map(&g.tmOut);
+    if (MODE == kModeBwd) {
+      tma_prefetch_map(&g.tmG);
+      tma_prefetch_map(&g.tmDW);
+      tma_prefetch_map(&g.tmDH);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -369,15 +444,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   const uint32_t tmem_base = *tmem_slot;
 
   const int C = (MODE == kModePlain) ? g.M : *g.C_dev;
-  const int nunits = num_units<MODE>(g, C);
+  const UnitSpace us = make_unit_space<MODE>(g, C);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ scheduler + producer
     if (lane == 0) {
       uint32_t n_issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const Unit un = decode_unit<MODE>(g, C, u);
+      for (int it = 0; ok; ++it) {
+        const int slot = it % UQ;
+        const uint32_t ph = (it / UQ) & 1;
+        if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
+        int u = atomicAdd(g.counter, 1);
+        if (u >= us.total) u = -1;
+        s_unit[slot] = u;
+        mbar_arrive(&uq_full[slot]);
+        if (u < 0) break;
+        const Unit un = decode_unit<MODE>(g, us, C, u);
         for (int kb = 0; kb < un.nk; ++kb) {
           const uint32_t stage = n_issued % STAGES;
           const uint32_t phase = (n_issued / STAGES) & 1u;
@@ -402,9 +485,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       uint32_t n_used = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const Unit un = decode_unit<MODE>(g, C, u);
+      for (int it = 0;; ++it) {
+        const int slot = it % UQ;
+        if (!mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err)) break;
+        const int u = s_unit[slot];
+        mbar_arrive(&uq_empty[slot]);
+        if (u < 0) break;
+        const Unit un = decode_unit<MODE>(g, us, C, u);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, g.err)) break;
         tc_fence_after();
         const bool a_mn = unit_a_mn<MODE>(g, un);
@@ -415,6 +502,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         const uint32_t b_lbo = b_mn ? MN_BOX_BYTES : 16u;
         const uint32_t a_step = a_mn ? 16u * 128u : 32u;  // bytes per K=16 slice
         const uint32_t b_step = b_mn ? 16u * 128u : 32u;
+        bool ok = true;
         for (int kb = 0; kb < un.nk; ++kb) {
           const uint32_t stage = n_used % STAGES;
           const uint32_t phase = (n_used / STAGES) & 1u;
@@ -453,50 +541,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t nstore = 0;  // grad: 64-column boxes stored so far by this CTA
+    uint32_t nstore = 0;  // TMA stores issued by this CTA (staging buffer parity)
     float wh_scale = 0.f;
-    if (MODE == kModeWH) {
+    if (MODE == kModeBwd) {
       const float lam = (g.lam_dev != nullptr) ? *g.lam_dev : g.lam;
       wh_scale = (C > 0) ? lam / static_cast<float>(C) * g.inv_sigma : 0.f;
     }
-    int it = 0;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
-      const Unit un = decode_unit<MODE>(g, C, u);
+    // Shared decision of the four epilogue warps (they pass named barriers
+    // together, so they leave the loop together).
+    int round = 0;
+    auto decide_abort = [&]() -> bool {
+      named_bar_sync(1, NUM_EPI_THREADS);
+      if (epi_tid == 0) decision[round & 1] = *abort_flag;
+      named_bar_sync(1, NUM_EPI_THREADS);
+      return decision[(round++) & 1] != 0;
+    };
+    // Stages one 128 x 128-byte box and hands it to the TMA engine.
+    auto emit_box = [&](const uint32_t (&w)[32], const CUtensorMap* map, int x, int y,
+                        bool reduce, bool issue) {
+      uint8_t* stg = sStg + (nstore & 1u) * STG_BYTES;
+      if (epi_tid == 0) bulk_wait_group_read<1>();  // the box stored two boxes ago left smem
+      named_bar_sync(1, NUM_EPI_THREADS);
+      stage_row128(stg, r, 0, w);
+      fence_proxy_async_smem();
+      named_bar_sync(1, NUM_EPI_THREADS);
+      if (epi_tid == 0) {
+        if (issue) {
+          if (reduce)
+            tma_reduce_add_2d(map, smem_addr(stg), x, y);
+          else
+            tma_store_2d(map, smem_addr(stg), x, y);
+        }
+        bulk_commit_group();
+      }
+      ++nstore;
+    };
+
+    for (int it = 0;; ++it) {
+      const int slot = it % UQ;
+      const bool got = mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err);
+      const int u = got ? s_unit[slot] : -1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&uq_empty[slot]);
+      if (decide_abort() || u < 0) break;
+      const Unit un = decode_unit<MODE>(g, us, C, u);
+
       // per-row data, fetched before waiting for the accumulator
       const int row = un.m0 + r;
       bool valid = false;
-      int yl = -1;
+      int yl = -1000000;
       float mrow = 0.f, krow = 0.f;
-      int orow = 0;
       int vglob0 = 0, vlim = 0;
-      if (MODE == kModeFwd || MODE == kModeGrad) {
+      if (MODE == kModeFwd || (MODE == kModeBwd && un.cls == kClsGrad)) {
         valid = row < C;
-        vglob0 = g.vp + un.n0;
+        vglob0 = (MODE == kModeBwd ? g.vp_g : 0) + un.n0;
         vlim = g.V - vglob0;
-        const int y = valid ? __ldg(g.y_c + row) : -1;
-        yl = valid ? y - vglob0 : -1000000;
-        if (MODE == kModeGrad && valid) {
+        if (valid) yl = __ldg(g.y_c + row) - vglob0;
+        if (MODE == kModeBwd && valid) {
           const int o = __ldg(g.idx + row);
           mrow = __ldg(g.m_saved + o);
           krow = g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e;
         }
-      } else if (MODE == kModeWH) {
-        if (un.cls == 0) {
-          valid = (un.m0 + r) < g.K;
-          orow = g.vp + un.m0 + r;  // dW row (vocabulary id)
-        } else {
-          valid = row < C;
-          orow = valid ? __ldg(g.idx + row) : 0;  // dH row (original position)
-        }
-      } else {
+      } else if (MODE == kModePlain) {
         valid = row < g.M;
       }
 
       mbar_wait(&tfull[acc], acc_phase, abort_flag, g.err);
-      named_bar_sync(1, NUM_EPI_THREADS);
-      if (epi_tid == 0) decision[it & 1] = *abort_flag;
-      named_bar_sync(1, NUM_EPI_THREADS);
-      if (decision[it & 1]) break;
+      if (decide_abort()) break;
       tc_fence_after();
       const uint32_t t_acc = lane_base + static_cast<uint32_t>(acc * BN);
 
@@ -520,85 +631,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           g.part[static_cast<size_t>(row) * g.part_ld + un.n0 / BN] = make_float2(st.m, st.s);
           if (st.have_tgt) g.tgt[row] = st.tgt;
         }
-      } else if (MODE == kModeGrad) {
+      } else if (MODE == kModeBwd && un.cls == kClsGrad) {
         uint32_t za[32], zb[32];
         tmem_ld32(t_acc, za);
         tmem_wait_ld(za);
 #pragma unroll 1
         for (int c = 0; c < BN / 32; c += 2) {
-          // chunks c, c+1 form one 64-column box staged in buffer (nstore & 1)
+          // chunks c, c+1 form one 64-column box of the 16-bit panel
           uint8_t* stg = sStg + (nstore & 1u) * STG_BYTES;
-          if (epi_tid == 0) bulk_wait_group_read<1>();  // the box stored 2 boxes ago left smem
+          if (epi_tid == 0) bulk_wait_group_read<1>();
           named_bar_sync(1, NUM_EPI_THREADS);
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
           grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, pk);
-          uint8_t* rowp = stg + r * 128;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int chunk16 = j ^ (r & 7);
-            *reinterpret_cast<uint4*>(rowp + chunk16 * 16) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          }
+          stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
           if (c + 2 < BN / 32) tmem_ld32(t_acc + (c + 2) * 32, za);
           grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, pk);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int chunk16 = (4 + j) ^ (r & 7);
-            *reinterpret_cast<uint4*>(rowp + chunk16 * 16) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          }
+          stage_row128(stg, r, 4, pk);
           if (c + 2 < BN / 32) tmem_wait_ld(za);
           fence_proxy_async_smem();
           named_bar_sync(1, NUM_EPI_THREADS);
           if (epi_tid == 0) {
             // a box that starts past the panel's last column holds only padding
-            if (un.n0 + c * 32 < g.ncols) tma_store_2d(&g.tmOut, smem_addr(stg), un.n0 + c * 32, un.m0);
+            if (un.n0 + c * 32 < g.w_g) tma_store_2d(&g.tmG, smem_addr(stg), un.n0 + c * 32, un.m0);
             bulk_commit_group();
           }
           ++nstore;
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
-      } else if (MODE == kModeWH) {
-        float* dst = (un.cls == 0 ? g.dW : g.dH) + static_cast<size_t>(orow) * g.D;
-        const bool accumulate = (un.cls == 1) && (g.vp > 0);
+      } else if (MODE == kModeBwd) {
+        // dW (class 0) or dH (class 1): fp32, scaled by lambda / (C sigma)
+        const bool is_dw = un.cls == kClsDW;
+        const CUtensorMap* map = is_dw ? &g.tmDW : &g.tmDH;
+        const int y = is_dw ? g.vp_wh + un.m0 : un.m0;
+        const bool reduce = !is_dw && g.dh_accumulate;
         const bool zero = (un.nk == 0);
+        const int nch = min(BN / 32, cdiv_i(g.D - un.n0, 32));
+        uint32_t za[32], zb[32], w[32];
+        if (!zero) {
+          tmem_ld32(t_acc, za);
+          tmem_wait_ld(za);
+        }
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int d0 = un.n0 + c * 32;
-          if (d0 >= g.D) break;
-          uint32_t z[32];
-          if (!zero) {
-            tmem_ld32(t_acc + c * 32, z);
-            tmem_wait_ld(z);
-          }
-          if (valid) {
-            const int nv = min(32, g.D - d0);  // multiple of 8
-            float4* p = reinterpret_cast<float4*>(dst + d0);
+        for (int c = 0; c < nch; c += 2) {
+          // za holds chunk c; chunk c+1 loads into zb meanwhile
+          if (!zero && c + 1 < nch) tmem_ld32(t_acc + (c + 1) * 32, zb);
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              if (q4 * 4 < nv) {
-                float4 v;
-                if (zero) {
-                  v = make_float4(0.f, 0.f, 0.f, 0.f);
-                } else {
-                  v = make_float4(__uint_as_float(z[4 * q4]) * wh_scale,
-                                  __uint_as_float(z[4 * q4 + 1]) * wh_scale,
-                                  __uint_as_float(z[4 * q4 + 2]) * wh_scale,
-                                  __uint_as_float(z[4 * q4 + 3]) * wh_scale);
-                }
-                if (accumulate) {
-                  const float4 o = p[q4];
-                  v.x += o.x;
-                  v.y += o.y;
-                  v.z += o.z;
-                  v.w += o.w;
-                }
-                p[q4] = v;
-              }
-            }
+          for (int j = 0; j < 32; ++j)
+            w[j] = zero ? 0u : __float_as_uint(__uint_as_float(za[j]) * wh_scale);
+          emit_box(w, map, un.n0 + c * 32, y, reduce, true);
+          if (c + 1 < nch) {
+            if (!zero) tmem_wait_ld(zb);
+            if (!zero && c + 2 < nch) tmem_ld32(t_acc + (c + 2) * 32, za);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              w[j] = zero ? 0u : __float_as_uint(__uint_as_float(zb[j]) * wh_scale);
+            emit_box(w, map, un.n0 + (c + 1) * 32, y, reduce, true);
+            if (!zero && c + 2 < nch) tmem_wait_ld(za);
           }
         }
         tc_fence_before();
@@ -626,7 +717,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         acc_phase ^= 1u;
       }
     }
-    if (MODE == kModeGrad && epi_tid == 0) bulk_wait_group<0>();
+    if (MODE == kModeBwd && epi_tid == 0) bulk_wait_group<0>();
   }
 
   __syncthreads();

@@ -102,6 +102,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, uint32_t src
                "r"(src), "r"(x), "r"(y)
                : "memory");
 }
+// Element-wise fp32 add of a shared-memory tile into global memory (in L2).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, uint32_t src, int32_t x,
+                                                  int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

