@@ -45,7 +45,7 @@ struct Layout {
 // pass uses come first (fwd_total bytes); the backward's follow.
 Layout make_layout(int64_t N, int64_t D, int64_t V) {
   Layout L{};
-  L.Np = roundup64(N > 0 ? N : 1, BM);
+  L.Np = roundup64(N > 0 ? N : 1, PAIR_M);  // every half-tile of a CTA pair starts inside
   L.nvt = cdiv64(V, BN);
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
   L.panels = cdiv64(V, L.vc);
@@ -122,6 +122,7 @@ struct DevInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
+  int pairs = 0;  // CTA pairs of the GEMM kernel that fit on the device at once
 };
 std::mutex g_mu;
 DevInfo g_dev[64];
@@ -148,6 +149,24 @@ flce_status device_setup(DevInfo* out) {
           cudaFuncSetAttribute(flce_gemm_kernel<kModePlain>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return FLCE_ERR_CUDA;
+      // how many CTA pairs can be resident together (one CTA per SM)
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1));
+      cfg.blockDim = dim3(NUM_THREADS);
+      cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, flce_gemm_kernel<kModeBwd>, &cfg) !=
+              cudaSuccess ||
+          clusters < 1)
+        return FLCE_ERR_CUDA;
+      d.pairs = clusters;
     }
     d.sms = sms;
     d.init = true;
@@ -197,13 +216,26 @@ cudaError_t timed_launch(int kind, cudaStream_t s, F&& launch) {
   return e;
 }
 
+// Persistent launch of CTA pairs: min(work units, resident pairs) clusters of 2.
 template <int MODE>
-cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int sms, cudaStream_t s) {
+cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaStream_t s) {
   if (units_upper <= 0) return cudaSuccess;
-  const int grid = static_cast<int>(units_upper < sms ? units_upper : sms);
+  const int npairs = static_cast<int>(units_upper < pairs ? units_upper : pairs);
   const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeBwd ? kProfBwd : kProfPlain;
   return timed_launch(kind, s, [&] {
-    flce_gemm_kernel<MODE><<<grid, NUM_THREADS, GEMM_SMEM_BYTES, s>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, flce_gemm_kernel<MODE>, a);
   });
 }
 
@@ -332,7 +364,7 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
 
   GemmArgs a{};
   if (!make_map(&a.tmA[0], p.hc, mt, D, L.Np, D * 2, BK, BM) ||
-      !make_map(&a.tmB[0], W, mt, D, V, D * 2, BK, BN))
+      !make_map(&a.tmB[0], W, mt, D, V, D * 2, BK, BN_HALF))
     return FLCE_ERR_CUDA;
   a.is_bf16 = bf16;
   a.C_dev = p.C;
@@ -348,7 +380,7 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
   a.part_ld = static_cast<int>(L.nvt);
   a.tgt = p.tgt;
   a.err = p.err;
-  FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, BM) * L.nvt, di.sms, s));
+  FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
   if (N > 0) {
     const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
@@ -397,14 +429,14 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
   // maps that do not depend on the panel
   CUtensorMap hcK, wK, hcMN, wMN, dwMap, dhMap;
   if (!make_map(&hcK, p.hc, mt, D, L.Np, D * 2, BK, BM) ||
-      !make_map(&wK, W, mt, D, V, D * 2, BK, BN) ||
+      !make_map(&wK, W, mt, D, V, D * 2, BK, BN_HALF) ||
       !make_map(&hcMN, p.hc, mt, D, L.Np, D * 2, 64, BK) ||
       !make_map(&wMN, W, mt, D, V, D * 2, 64, BK) ||
       !make_map(&dwMap, dW, kMapF32, D, V, D * 4, 32, BM) ||
       !make_map(&dhMap, p.dhc, kMapF32, D, L.Np, D * 4, 32, BM))
     return FLCE_ERR_CUDA;
 
-  const int64_t nT_max = cdiv64(N, BM);
+  const int64_t nT_max = cdiv64(N, PAIR_M);
   const int64_t nD = cdiv64(D, BN);
   for (int64_t Lp = 0; Lp <= L.panels; ++Lp) {
     const bool has_g = Lp < L.panels;
@@ -452,9 +484,9 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
     a.lam_dev = lambda_dev;
     a.inv_sigma = 1.f / sigma;
     a.err = p.err;
-    const int64_t units = (has_wh ? cdiv64(w_wh, BM) * nD + nT_max * nD : 0) +
+    const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +
                           (has_g ? nT_max * cdiv64(w_g, BN) : 0);
-    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.sms, s));
+    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.pairs, s));
 
     if (b != nullptr && has_g) {
       const uint16_t* gp = p.gpanel[Lp & 1];
@@ -506,7 +538,7 @@ flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, 
   const bool okA = a_mn ? make_map(&a.tmA[0], A, mt, M, K, M * 2, 64, BK)
                         : make_map(&a.tmA[0], A, mt, K, M, K * 2, BK, BM);
   const bool okB = b_mn ? make_map(&a.tmB[0], B, mt, N, K, N * 2, 64, BK)
-                        : make_map(&a.tmB[0], B, mt, K, N, K * 2, BK, BN);
+                        : make_map(&a.tmB[0], B, mt, K, N, K * 2, BK, BN_HALF);
   if (!okA || !okB) return FLCE_ERR_CUDA;
   a.a_mn = a_mn ? 1 : 0;
   a.b_mn = b_mn ? 1 : 0;
@@ -519,7 +551,7 @@ flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, 
   a.err = static_cast<uint32_t*>(ws);
   a.counter = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kCounterOffset);
   FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
-  FLCE_CK(launch_gemm<kModePlain>(a, cdiv64(M, BM) * cdiv64(N, BN), di.sms, s));
+  FLCE_CK(launch_gemm<kModePlain>(a, cdiv64(M, PAIR_M) * cdiv64(N, BN), di.pairs, s));
   return FLCE_OK;
 }
 

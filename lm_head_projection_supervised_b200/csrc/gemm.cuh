@@ -1,13 +1,18 @@
 // Persistent, warp-specialised tcgen05 GEMM for sm_100a with the fused
 // epilogues of exact linear cross-entropy.
 //
-// One CTA per SM.  Warp 0 (one lane) takes work units from a global counter
-// (longest units first), publishes each unit id through a small shared-memory
-// ring, and streams the unit's operand tiles with TMA into a STAGES-deep
-// ring; warp 1 (one lane) issues tcgen05.mma.kind::f16 (M=128, N=256, K=16)
-// into one of two 128x256 f32 accumulators in TMEM (512 columns); warps 4..7
-// read a finished accumulator with tcgen05.ld (thread = TMEM lane = tile
-// row) and run the epilogue while the next unit accumulates in the other.
+// CTAs run in pairs (clusters of 2), one CTA per SM; a work unit is a
+// 256 x 256 output tile.  Each CTA holds half of the unit's A rows (128) and
+// half of its B rows (128) in a STAGES-deep ring of 32 KiB stages loaded by
+// TMA, and half of the accumulator (128 rows x 256 f32 columns) in its TMEM.
+// The even CTA of the pair takes work units from a global counter (longest
+// units first) and broadcasts each unit id into both CTAs' unit rings; its
+// warp 1 issues tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256, K=16),
+// which reads both CTAs' stages and writes both CTAs' TMEM, into one of two
+// accumulators (512 columns).  In each CTA, warp 0 streams that CTA's halves
+// of the operands and warps 4..7 read a finished accumulator with
+// tcgen05.ld (thread = TMEM lane = tile row) and run the epilogue while the
+// next unit accumulates in the other.
 //
 // Modes (one launch = one mode):
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
@@ -38,13 +43,16 @@
 
 namespace flce {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                          // rows per CTA
+constexpr int PAIR_M = 2 * BM;                   // rows per work unit (CTA pair)
+constexpr int BN = 256;                          // columns per work unit
+constexpr int BN_HALF = BN / 2;                  // B rows held by each CTA
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int UQ = 4;                            // depth of the unit-id ring
-constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KiB
-constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;  // 32 KiB
+constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;       // 16 KiB
+constexpr uint32_t B_STAGE_BYTES = BN_HALF * BK * 2;  // 16 KiB
+constexpr uint32_t PAIR_TX_BYTES = 2 * (A_STAGE_BYTES + B_STAGE_BYTES);  // both CTAs' loads
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;   // 8 KiB: 64 MN-elements x 64 K rows
 constexpr uint32_t STG_BYTES = BM * 128;         // 16 KiB: 128 rows x 128 bytes
 constexpr int NUM_THREADS = 256;
@@ -123,8 +131,8 @@ template <int MODE>
 __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
   UnitSpace s;
   if (MODE == kModeBwd) {
-    const int nT = cdiv_i(C, BM), nD = cdiv_i(g.D, BN);
-    s.n0 = g.has_wh ? cdiv_i(g.w_wh, BM) * nD : 0;       // dW
+    const int nT = cdiv_i(C, PAIR_M), nD = cdiv_i(g.D, BN);
+    s.n0 = g.has_wh ? cdiv_i(g.w_wh, PAIR_M) * nD : 0;   // dW
     s.n1 = g.has_wh ? nT * nD : 0;                       // dH
     s.n2 = g.has_g ? nT * cdiv_i(g.w_g, BN) : 0;         // grad
     s.k0 = cdiv_i(C, BK);
@@ -142,7 +150,7 @@ __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
     s.total = s.n0 + s.n1 + s.n2;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
-    s.n0 = cdiv_i(rows, BM) * cdiv_i(g.ncols, BN);
+    s.n0 = cdiv_i(rows, PAIR_M) * cdiv_i(g.ncols, BN);
     s.n1 = s.n2 = 0;
     s.k0 = cdiv_i(g.K, BK);
     s.k1 = s.k2 = 0;
@@ -154,7 +162,7 @@ __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
   return s;
 }
 
-// Unit u -> tile.  Row (token) tiles vary fastest so that units running at
+// Unit u -> 256 x 256 tile (m0, n0) of the pair.  Row (token) tiles vary fastest so that units running at
 // the same time share the W / G columns they read through L2.
 template <int MODE>
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& s, int C, int u) {
@@ -173,13 +181,13 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& 
   un.cls = cls;
   un.nk = pick3(cls, s.k0, s.k1, s.k2);
   if (MODE == kModeBwd && cls == kClsDW) {
-    const int nVb = cdiv_i(g.w_wh, BM);
-    un.m0 = (u % nVb) * BM;
+    const int nVb = cdiv_i(g.w_wh, PAIR_M);
+    un.m0 = (u % nVb) * PAIR_M;
     un.n0 = (u / nVb) * BN;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
-    const int nT = cdiv_i(rows, BM);
-    un.m0 = (u % nT) * BM;
+    const int nT = cdiv_i(rows, PAIR_M);
+    un.m0 = (u % nT) * PAIR_M;
     un.n0 = (u / nT) * BN;
   }
   return un;
@@ -198,31 +206,34 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
   return false;
 }
 
-// TMA loads of k-block kb of unit `un` into one ring stage (48 KiB in total).
+// TMA loads of k-block kb of unit `un` into this CTA's ring stage: its 128
+// A rows (16 KiB) and its 128 of the 256 B rows (16 KiB).  Completion is
+// counted on the even CTA's barrier `bar_cluster`.
 template <int MODE>
 __device__ __forceinline__ void issue_stage_loads(const GemmArgs& g, const Unit& un, int kb,
-                                                  uint32_t sa, uint32_t sb, uint64_t* bar) {
+                                                  uint32_t rank, uint32_t sa, uint32_t sb,
+                                                  uint32_t bar_cluster) {
   const int mapi = (MODE == kModeBwd) ? un.cls : 0;
   const CUtensorMap* tA = &g.tmA[mapi];
   const CUtensorMap* tB = &g.tmB[mapi];
   const int k0 = kb * BK;
-  // A: 128 rows x 64 k
+  const int am0 = un.m0 + static_cast<int>(rank) * BM;       // this CTA's A rows
+  const int bn0 = un.n0 + static_cast<int>(rank) * BN_HALF;  // this CTA's B rows
   if (unit_a_mn<MODE>(g, un)) {
-    tma_load_2d(sa, tA, bar, un.m0, k0);
-    tma_load_2d(sa + MN_BOX_BYTES, tA, bar, un.m0 + 64, k0);
+    tma_load_2d_pair(sa, tA, bar_cluster, am0, k0);
+    tma_load_2d_pair(sa + MN_BOX_BYTES, tA, bar_cluster, am0 + 64, k0);
   } else {
-    tma_load_2d(sa, tA, bar, k0, un.m0);
+    tma_load_2d_pair(sa, tA, bar_cluster, k0, am0);
   }
-  // B: 256 rows x 64 k
   if (unit_b_mn<MODE>(g, un)) {
     // dH: the k index is a vocabulary id of the panel
     const int kB = (MODE == kModeBwd && un.cls == kClsDH) ? g.vp_wh + k0 : k0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tma_load_2d(sb + j * MN_BOX_BYTES, tB, bar, un.n0 + 64 * j, kB);
+    tma_load_2d_pair(sb, tB, bar_cluster, bn0, kB);
+    tma_load_2d_pair(sb + MN_BOX_BYTES, tB, bar_cluster, bn0 + 64, kB);
   } else {
     // fwd / grad: the row index is a vocabulary id
-    const int nrow = (MODE == kModeBwd) ? g.vp_g + un.n0 : un.n0;
-    tma_load_2d(sb, tB, bar, k0, nrow);
+    const int nrow = (MODE == kModeBwd) ? g.vp_g + bn0 : bn0;
+    tma_load_2d_pair(sb, tB, bar_cluster, k0, nrow);
   }
 }
 
@@ -378,7 +389,7 @@ __device__ __forceinline__ void stage_row128(uint8_t* stg, int r, int chunk0,
 }
 
 // ---------------------------------------------------------------------------
-// The kernel
+// The kernel (launched as clusters of 2 CTAs)
 // ---------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_constant__ GemmArgs g) {
@@ -402,19 +413,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the CTA that schedules and issues MMAs
+  const bool leader = rank == 0;
+  // Barriers that only the even CTA uses are counted there; the odd CTA
+  // reaches them through shared::cluster addresses.
+  auto leader_addr = [&](const void* p) -> uint32_t {
+    return leader ? smem_addr(p) : mapa_shared(smem_addr(p), 0);
+  };
+  auto arrive_on_leader = [&](uint64_t* bar) {
+    if (leader)
+      mbar_arrive(bar);
+    else
+      mbar_arrive_cluster(mapa_shared(smem_addr(bar), 0));
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1);   // even CTA: its expect_tx arrival + both CTAs' bytes
+      mbar_init(&empty[s], 1);  // one multicast MMA commit
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], NUM_EPI_THREADS);
+      mbar_init(&tfull[a], 1);                           // one multicast MMA commit
+      mbar_init(&tempty[a], 2 * NUM_EPI_THREADS / 32);   // one lane per epilogue warp, both CTAs
     }
     for (int q = 0; q < UQ; ++q) {
       mbar_init(&uq_full[q], 1);
-      mbar_init(&uq_empty[q], 1 + NUM_EPI_THREADS / 32);  // MMA lane + one lane per epilogue warp
+      // even CTA: its MMA lane and epilogue warps; odd CTA: its producer and epilogue warps
+      mbar_init(&uq_empty[q], 2 * (1 + NUM_EPI_THREADS / 32));
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -435,11 +460,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -451,14 +477,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     if (lane == 0) {
       uint32_t n_issued = 0;
       bool ok = true;
+      const uint32_t full_c0 = leader_addr(&full[0]);
       for (int it = 0; ok; ++it) {
         const int slot = it % UQ;
         const uint32_t ph = (it / UQ) & 1;
-        if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
-        int u = atomicAdd(g.counter, 1);
-        if (u >= us.total) u = -1;
-        s_unit[slot] = u;
-        mbar_arrive(&uq_full[slot]);
+        int u;
+        if (leader) {
+          if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
+          u = atomicAdd(g.counter, 1);
+          if (u >= us.total) u = -1;
+          s_unit[slot] = u;
+          st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<int*>(&s_unit[slot])), 1),
+                                static_cast<uint32_t>(u));
+          mbar_arrive(&uq_full[slot]);
+          mbar_arrive_cluster(mapa_shared(smem_addr(&uq_full[slot]), 1));
+        } else {
+          if (!mbar_wait_cluster(&uq_full[slot], ph, abort_flag, g.err)) break;
+          u = s_unit[slot];
+          arrive_on_leader(&uq_empty[slot]);
+        }
         if (u < 0) break;
         const Unit un = decode_unit<MODE>(g, us, C, u);
         for (int kb = 0; kb < un.nk; ++kb) {
@@ -468,20 +505,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], A_STAGE_BYTES + B_STAGE_BYTES);
-          issue_stage_loads<MODE>(g, un, kb, smem_addr(sA + stage * A_STAGE_BYTES),
-                                  smem_addr(sB + stage * B_STAGE_BYTES), &full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
+          issue_stage_loads<MODE>(g, un, kb, rank, smem_addr(sA + stage * A_STAGE_BYTES),
+                                  smem_addr(sB + stage * B_STAGE_BYTES),
+                                  full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)));
           ++n_issued;
         }
       }
-      // Let every copy still in flight land before the CTA can exit.
-      const uint32_t first = n_issued > STAGES ? n_issued - STAGES : 0u;
-      for (uint32_t i = first; i < n_issued; ++i)
-        mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, nullptr, nullptr, kDrainLimitNs);
+      // The even CTA lets every copy still in flight (its own and its peer's)
+      // land before the pair can exit.
+      if (leader) {
+        const uint32_t first = n_issued > STAGES ? n_issued - STAGES : 0u;
+        for (uint32_t i = first; i < n_issued; ++i)
+          mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, nullptr, nullptr, kDrainLimitNs);
+      }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
       uint32_t n_used = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
@@ -496,7 +537,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         tc_fence_after();
         const bool a_mn = unit_a_mn<MODE>(g, un);
         const bool b_mn = unit_b_mn<MODE>(g, un);
-        const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, BM, BN);
+        const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, PAIR_M, BN);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         const uint32_t a_lbo = a_mn ? MN_BOX_BYTES : 16u;
         const uint32_t b_lbo = b_mn ? MN_BOX_BYTES : 16u;
@@ -517,26 +558,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024u);
             const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024u);
-            umma_f16(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);  // frees the stage once these MMAs are done
+          umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
           ++n_used;
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);  // accumulator ready (immediately when nk == 0)
+        umma_commit_pair_mc(&tfull[acc], 0x3);  // accumulator ready in both CTAs
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      // All MMAs of this CTA complete before TMEM is released.
-      umma_commit(done_bar);
+      // All pair MMAs complete before either CTA releases its TMEM.
+      umma_commit_pair_mc(done_bar, 0x1);
       mbar_wait(done_bar, 0, nullptr, nullptr, kDrainLimitNs);
     }
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;              // TMEM lane quadrant of this warp
-    const int r = q * 32 + lane;         // row within the tile
+    const int r = q * 32 + lane;         // row within this CTA's half of the tile
+    const int rbase = static_cast<int>(rank) * BM;
     const int epi_tid = threadIdx.x - EPI_WARP0 * 32;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
@@ -579,15 +621,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 
     for (int it = 0;; ++it) {
       const int slot = it % UQ;
-      const bool got = mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err);
+      const bool got = leader ? mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err)
+                              : mbar_wait_cluster(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err);
       const int u = got ? s_unit[slot] : -1;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&uq_empty[slot]);
+      if (lane == 0) arrive_on_leader(&uq_empty[slot]);
       if (decide_abort() || u < 0) break;
       const Unit un = decode_unit<MODE>(g, us, C, u);
+      const int tm0 = un.m0 + rbase;  // first row of this CTA's half
 
       // per-row data, fetched before waiting for the accumulator
-      const int row = un.m0 + r;
+      const int row = tm0 + r;
       bool valid = false;
       int yl = -1000000;
       float mrow = 0.f, krow = 0.f;
@@ -626,7 +670,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           if (c + 2 < BN / 32) tmem_wait_ld(za);
         }
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
         if (valid) {
           g.part[static_cast<size_t>(row) * g.part_ld + un.n0 / BN] = make_float2(st.m, st.s);
           if (st.have_tgt) g.tgt[row] = st.tgt;
@@ -654,20 +699,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           named_bar_sync(1, NUM_EPI_THREADS);
           if (epi_tid == 0) {
             // a box that starts past the panel's last column holds only padding
-            if (un.n0 + c * 32 < g.w_g) tma_store_2d(&g.tmG, smem_addr(stg), un.n0 + c * 32, un.m0);
+            if (un.n0 + c * 32 < g.w_g) tma_store_2d(&g.tmG, smem_addr(stg), un.n0 + c * 32, tm0);
             bulk_commit_group();
           }
           ++nstore;
         }
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else if (MODE == kModeBwd) {
         // dW (class 0) or dH (class 1): fp32, scaled by lambda / (C sigma)
         const bool is_dw = un.cls == kClsDW;
         const CUtensorMap* map = is_dw ? &g.tmDW : &g.tmDH;
-        const int y = is_dw ? g.vp_wh + un.m0 : un.m0;
+        const int y = is_dw ? g.vp_wh + tm0 : tm0;
         const bool reduce = !is_dw && g.dh_accumulate;
         const bool zero = (un.nk == 0);
+        // a dW half that starts past the panel's last row has nothing to store
+        const bool issue = !is_dw || tm0 < g.w_wh;
         const int nch = min(BN / 32, cdiv_i(g.D - un.n0, 32));
         uint32_t za[32], zb[32], w[32];
         if (!zero) {
@@ -681,19 +729,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             w[j] = zero ? 0u : __float_as_uint(__uint_as_float(za[j]) * wh_scale);
-          emit_box(w, map, un.n0 + c * 32, y, reduce, true);
+          emit_box(w, map, un.n0 + c * 32, y, reduce, issue);
           if (c + 1 < nch) {
             if (!zero) tmem_wait_ld(zb);
             if (!zero && c + 2 < nch) tmem_ld32(t_acc + (c + 2) * 32, za);
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               w[j] = zero ? 0u : __float_as_uint(__uint_as_float(zb[j]) * wh_scale);
-            emit_box(w, map, un.n0 + (c + 1) * 32, y, reduce, true);
+            emit_box(w, map, un.n0 + (c + 1) * 32, y, reduce, issue);
             if (!zero && c + 2 < nch) tmem_wait_ld(za);
           }
         }
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else {  // kModePlain
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
@@ -710,7 +759,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           }
         }
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
       }
       if (++acc == 2) {
         acc = 0;
@@ -720,10 +770,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     if (MODE == kModeBwd && epi_tid == 0) bulk_wait_group<0>();
   }
 
+  // Neither CTA frees its TMEM (or exits) while the pair still uses it.
+  tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
