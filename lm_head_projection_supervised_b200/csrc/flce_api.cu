@@ -27,7 +27,10 @@ namespace {
 constexpr int64_t kMaxN = int64_t(1) << 24;
 constexpr int64_t kMaxD = int64_t(1) << 16;
 constexpr int64_t kMaxV = int64_t(1) << 24;
-constexpr int64_t kPanelCols = 4096;   // vocabulary columns per gradient panel
+#ifndef FLCE_PANEL_COLS
+#define FLCE_PANEL_COLS 8192
+#endif
+constexpr int64_t kPanelCols = FLCE_PANEL_COLS;  // vocabulary columns per gradient panel
 constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
 constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
@@ -141,13 +144,15 @@ flce_status device_setup(DevInfo* out) {
       return FLCE_ERR_CUDA;
     d.ok = (major == 10 && minor == 0) && encode_fn() != nullptr;
     if (d.ok) {
-      const int bytes = static_cast<int>(GEMM_SMEM_BYTES);
       if (cudaFuncSetAttribute(flce_gemm_kernel<kModeFwd>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(ModeCfg<kModeFwd>::SMEM_BYTES)) != cudaSuccess ||
           cudaFuncSetAttribute(flce_gemm_kernel<kModeBwd>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess ||
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(ModeCfg<kModeBwd>::SMEM_BYTES)) != cudaSuccess ||
           cudaFuncSetAttribute(flce_gemm_kernel<kModePlain>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(ModeCfg<kModePlain>::SMEM_BYTES)) != cudaSuccess)
         return FLCE_ERR_CUDA;
       // how many CTA pairs can be resident together (one CTA per SM)
       cudaLaunchConfig_t cfg = {};
@@ -231,7 +236,7 @@ cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaS
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
     cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+    cfg.dynamicSmemBytes = ModeCfg<MODE>::SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;

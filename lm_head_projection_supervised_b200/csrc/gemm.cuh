@@ -48,7 +48,6 @@ constexpr int PAIR_M = 2 * BM;                   // rows per work unit (CTA pair
 constexpr int BN = 256;                          // columns per work unit
 constexpr int BN_HALF = BN / 2;                  // B rows held by each CTA
 constexpr int BK = 64;
-constexpr int STAGES = 6;
 constexpr int UQ = 4;                            // depth of the unit-id ring
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;       // 16 KiB
 constexpr uint32_t B_STAGE_BYTES = BN_HALF * BK * 2;  // 16 KiB
@@ -60,10 +59,18 @@ constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr size_t GEMM_SMEM_BYTES =
-    1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 2 * STG_BYTES + 512;
-
 enum GemmMode : int { kModeFwd = 0, kModeBwd = 1, kModePlain = 2 };
+
+// Ring depth per mode: the backward epilogue stages TMA stores through two
+// 16 KiB boxes, the other modes use that shared memory for a 7th stage.
+template <int MODE>
+struct ModeCfg {
+  static constexpr int STAGES = (MODE == kModeBwd) ? 6 : 7;
+  static constexpr uint32_t STAGING = (MODE == kModeBwd) ? 2 * STG_BYTES : 0;
+  static constexpr size_t SMEM_BYTES =
+      1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + STAGING + 512;
+};
+constexpr size_t GEMM_SMEM_BYTES = ModeCfg<kModeBwd>::SMEM_BYTES;  // the largest
 enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
 
 struct GemmArgs {
@@ -393,13 +400,14 @@ __device__ __forceinline__ void stage_row128(uint8_t* stg, int r, int chunk0,
 // ---------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_constant__ GemmArgs g) {
+  constexpr int STAGES = ModeCfg<MODE>::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_STAGE_BYTES;
   uint8_t* sStg = sB + STAGES * B_STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 2 * STG_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + ModeCfg<MODE>::STAGING);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
