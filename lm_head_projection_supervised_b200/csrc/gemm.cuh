@@ -169,7 +169,8 @@ __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
   return s;
 }
 
-// Unit u -> 256 x 256 tile (m0, n0) of the pair.  Row (token) tiles vary fastest so that units running at
+// Unit u -> 256 x 256 tile (m0, n0) of the pair.  For the forward, gradient and
+// plain tiles, row (token) tiles vary fastest so that units running at
 // the same time share the W / G columns they read through L2.
 template <int MODE>
 __device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& s, int C, int u) {
@@ -187,10 +188,13 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& 
   }
   un.cls = cls;
   un.nk = pick3(cls, s.k0, s.k1, s.k2);
-  if (MODE == kModeBwd && cls == kClsDW) {
-    const int nVb = cdiv_i(g.w_wh, PAIR_M);
-    un.m0 = (u % nVb) * PAIR_M;
-    un.n0 = (u / nVb) * BN;
+  if (MODE == kModeBwd && cls != kClsGrad) {
+    // dW / dH: the hidden-dimension block varies fastest, so the units that
+    // read the same block of the gradient panel (a column strip for dW, a
+    // row block for dH) run side by side and share it through L2
+    const int nD = cdiv_i(g.D, BN);
+    un.m0 = (u / nD) * PAIR_M;
+    un.n0 = (u % nD) * BN;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
     const int nT = cdiv_i(rows, PAIR_M);
