@@ -4,7 +4,8 @@ Test infrastructure: imported only by the tests, the smoke check and the
 benchmark's CPU-baseline leg.  It shares no code with the CUDA path.
 """
 from .flce_oracle import (IGNORE_INDEX, backward, chunked, forward, forward_backward,
-                          objective, row_outputs, supervised_rows, vocab_outputs)
+                          objective, row_outputs, row_scales, supervised_rows,
+                          vocab_outputs)
 
 __all__ = ["IGNORE_INDEX", "backward", "chunked", "forward", "forward_backward",
-           "objective", "row_outputs", "supervised_rows", "vocab_outputs"]
+           "objective", "row_outputs", "row_scales", "supervised_rows", "vocab_outputs"]

@@ -90,12 +90,40 @@ def _rows_stats(Hs, W, b, y):
     return Z, m, logs, tgt, loss_rows
 
 
+REDUCTIONS = ("mean", "sum", "none")
+
+
+def _row_weights(weight, idx):
+    """w_i of the supervised rows (1 when no weights are given)."""
+    if weight is None:
+        return torch.ones(len(idx), dtype=torch.float64)
+    return _f64(weight)[torch.as_tensor(idx)]
+
+
+def _denominator(reduction, C, denom):
+    """mean: C (p2 §01); sum: the caller's global count (NeMo num_label_tokens) or 1."""
+    if reduction == "mean":
+        return float(C)
+    if reduction == "sum":
+        return float(denom) if denom is not None and denom > 0 else 1.0
+    return 1.0
+
+
 def forward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
-            row_block: int = 512):
+            row_block: int = 512, weight=None, reduction: str = "mean", denom=None):
     """Loss and saved statistics (§01, §02), dense in the vocabulary.
 
-    Returns dict(loss, m[N], logs[N], idx, C, loss_rows[C]).  For C = 0 the
-    loss is the zero sentinel of §01 and m = log s = -inf for every row."""
+    reduction "mean" is the objective of p2 §01, (1/C) sum_i w_i l_i; "sum"
+    is sum_i w_i l_i / denom and "none" the per-row w_i l_i (the NeMo
+    ChunkedCrossEntropy reductions, num_label_tokens and loss_weights).  w_i = 1
+    without weights.
+
+    Returns dict(loss, loss_vec[N], m[N], logs[N], idx, C, loss_rows[C]);
+    loss_vec holds w_i l_i on supervised rows and 0 elsewhere, loss is None for
+    "none".  For C = 0 the loss is the zero sentinel of §01 and m = log s = -inf
+    for every row."""
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"reduction must be one of {REDUCTIONS}")
     H, W, b = _f64(H), _f64(W), _f64(b)
     N, V = H.shape[0], W.shape[0]
     idx, C = supervised_rows(labels, mask, ignore_index)
@@ -108,17 +136,42 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
         rows = torch.as_tensor(idx[r0:r1])
         _, mb, lb, _, lr = _rows_stats(H[rows], W, b, y[r0:r1])
         m[rows], logs[rows], loss_rows[r0:r1] = mb, lb, lr
-    loss = float(loss_rows.sum() / C) if C > 0 else 0.0
-    return dict(loss=loss, m=m.numpy(), logs=logs.numpy(), idx=idx, C=C,
-                loss_rows=loss_rows.numpy())
+    w = _row_weights(weight, idx)
+    loss_vec = torch.zeros(N, dtype=torch.float64)
+    loss_vec[torch.as_tensor(idx)] = w * loss_rows
+    if reduction == "none":
+        loss = None
+    elif C == 0:
+        loss = 0.0
+    else:
+        loss = float((w * loss_rows).sum() / _denominator(reduction, C, denom))
+    return dict(loss=loss, loss_vec=loss_vec.numpy(), m=m.numpy(), logs=logs.numpy(), idx=idx,
+                C=C, loss_rows=loss_rows.numpy())
+
+
+def row_scales(labels, mask, ignore_index, lam, weight=None, reduction="mean", denom=None,
+               grad_rows=None):
+    """s_i of G_ij = s_i (p_ij - 1[j = y_i]) for the supervised rows (§04 with
+    lambda a_i / C generalised to the reductions): mean lambda w_i / C, sum
+    lambda w_i / denom, none g_i w_i with g the per-row upstream gradient."""
+    idx, C = supervised_rows(labels, mask, ignore_index)
+    w = _row_weights(weight, idx)
+    if reduction == "none":
+        if grad_rows is None:
+            raise ValueError("reduction 'none' needs grad_rows")
+        return _f64(grad_rows)[torch.as_tensor(idx)] * w
+    if C == 0:
+        return torch.zeros(0, dtype=torch.float64)
+    return (lam / _denominator(reduction, C, denom)) * w
 
 
 def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
-             lam: float = 1.0, m=None, logs=None, row_block: int = 512):
+             lam: float = 1.0, m=None, logs=None, row_block: int = 512, weight=None,
+             reduction: str = "mean", denom=None, grad_rows=None):
     """dH, dW, db from the reconstruction of §04, dense in the vocabulary.
 
     m and logs are the saved statistics (recomputed here when not given).
-    db is None when b is None."""
+    db is None when b is None.  See row_scales for the reductions."""
     H, W, bt = _f64(H), _f64(W), _f64(b)
     N, D, V = H.shape[0], H.shape[1], W.shape[0]
     idx, C = supervised_rows(labels, mask, ignore_index)
@@ -133,7 +186,7 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
                      ignore_index, row_block)
         m, logs = st["m"], st["logs"]
     m, logs = _f64(m), _f64(logs)
-    scale = lam / C
+    scale = row_scales(labels, mask, ignore_index, lam, weight, reduction, denom, grad_rows)
     for r0 in range(0, C, row_block):
         r1 = min(C, r0 + row_block)
         rows = torch.as_tensor(idx[r0:r1])
@@ -143,7 +196,7 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
             Z = Z + bt
         P = torch.exp((Z - m[rows][:, None]) - logs[rows][:, None])
         P[torch.arange(r1 - r0), torch.as_tensor(y[r0:r1])] -= 1.0
-        G = scale * P
+        G = scale[r0:r1, None] * P
         dH[rows] = G @ W
         dW += G.T @ Hs
         if db is not None:
@@ -152,10 +205,11 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
 
 
 def forward_backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
-                     lam: float = 1.0, row_block: int = 512):
-    f = forward(H, W, b, labels, mask, ignore_index, row_block)
+                     lam: float = 1.0, row_block: int = 512, weight=None,
+                     reduction: str = "mean", denom=None, grad_rows=None):
+    f = forward(H, W, b, labels, mask, ignore_index, row_block, weight, reduction, denom)
     dH, dW, db = backward(H, W, b, labels, mask, ignore_index, lam, f["m"], f["logs"],
-                          row_block)
+                          row_block, weight, reduction, denom, grad_rows)
     f.update(dH=dH, dW=dW, db=db)
     return f
 

@@ -321,3 +321,84 @@ def test_packed_layout_counts():
     inp = wl.make_inputs(dataclasses.replace(spec, V=1024, D=8))
     assert orc.supervised_rows(inp.labels, inp.mask)[1] == 11472
     assert np.all(inp.labels[:614] == -100) and inp.labels[614] >= 0
+
+
+# --- reductions, per-row weights and per-row upstream gradients ---------------
+# (NeMo ChunkedCrossEntropy: reduction 'sum'/'none', num_label_tokens,
+#  loss_weights; the page's objective is the 'mean' case)
+
+def _torch_rows(H, W, b, y, mask):
+    """Per-row CE of the dense logits from torch (0 for unsupervised rows)."""
+    Ht = torch.tensor(H, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    yy = torch.tensor(np.where(mask.astype(bool), y, -100))
+    rows = torch.nn.functional.cross_entropy(Ht @ Wt.T + bt, yy, ignore_index=-100,
+                                             reduction="none")
+    return Ht, Wt, bt, rows
+
+
+def test_reduction_none_matches_torch_per_row():
+    H, W, b, y, mask = _case(18, N=33, D=7, V=90)
+    w = np.random.default_rng(1).uniform(0.2, 2.0, 33)
+    f = orc.forward(H, W, b, y, mask, weight=w, reduction="none")
+    _, _, _, rows = _torch_rows(H, W, b, y, mask)
+    assert f["loss"] is None
+    assert _close(f["loss_vec"], w * rows.detach().numpy(), 1e-12)
+
+
+@pytest.mark.parametrize("denom", [None, 37.0])
+def test_weighted_sum_matches_torch_autograd(denom):
+    H, W, b, y, mask = _case(19, N=30, D=6, V=70)
+    w = np.random.default_rng(2).uniform(0.0, 3.0, 30)
+    lam = 0.8
+    f = orc.forward_backward(H, W, b, y, mask, lam=lam, weight=w, reduction="sum", denom=denom)
+    Ht, Wt, bt, rows = _torch_rows(H, W, b, y, mask)
+    L = (torch.tensor(w) * rows).sum() / (denom if denom else 1.0)
+    (lam * L).backward()
+    assert abs(f["loss"] - L.item()) < 1e-12 * max(1.0, abs(L.item()))
+    assert _close(f["dH"], Ht.grad.numpy()) and _close(f["dW"], Wt.grad.numpy())
+    assert _close(f["db"], bt.grad.numpy())
+
+
+def test_none_backward_matches_torch_autograd():
+    H, W, b, y, mask = _case(20, N=25, D=5, V=60)
+    rng = np.random.default_rng(3)
+    w = rng.uniform(0.5, 1.5, 25)
+    g = rng.standard_normal(25)
+    f = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="none", grad_rows=g)
+    Ht, Wt, bt, rows = _torch_rows(H, W, b, y, mask)
+    (torch.tensor(w) * rows).backward(torch.tensor(g))
+    assert _close(f["dH"], Ht.grad.numpy()) and _close(f["dW"], Wt.grad.numpy())
+    assert _close(f["db"], bt.grad.numpy())
+
+
+def test_sum_over_c_equals_mean():
+    H, W, b, y, mask = _case(21)
+    idx, C = orc.supervised_rows(y, mask)
+    a = orc.forward_backward(H, W, b, y, mask, lam=1.3)
+    s = orc.forward_backward(H, W, b, y, mask, lam=1.3, reduction="sum", denom=float(C))
+    assert abs(a["loss"] - s["loss"]) < 1e-13
+    for k in ("dH", "dW", "db"):
+        assert _close(a[k], s[k], 1e-13)
+
+
+def test_weighted_sum_finite_differences():
+    H, W, b, y, mask = _case(22, N=6, D=3, V=9, ignore=1, mask_false=1)
+    w = np.array([0.5, 2.0, 1.0, 0.0, 3.0, 1.5])
+    f = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="sum", denom=4.0)
+    eps = 1e-6
+    for ix in [(0, 0), (2, 1), (5, 2)]:
+        Hp, Hm = H.copy(), H.copy()
+        Hp[ix] += eps
+        Hm[ix] -= eps
+        fd = (orc.forward(Hp, W, b, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]
+              - orc.forward(Hm, W, b, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]) / (2 * eps)
+        assert abs(fd - f["dH"][ix]) < 1e-8
+    for j in [0, 4, 8]:
+        bp, bm = b.copy(), b.copy()
+        bp[j] += eps
+        bm[j] -= eps
+        fd = (orc.forward(H, W, bp, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]
+              - orc.forward(H, W, bm, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]) / (2 * eps)
+        assert abs(fd - f["db"][j]) < 1e-8
