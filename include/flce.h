@@ -70,7 +70,8 @@ typedef enum {
   FLCE_ERR_LABEL = 7,       /* device: a supervised label is outside [0, V)      */
   FLCE_ERR_TIMEOUT = 8,     /* device: a pipeline wait ran past its time limit   */
   FLCE_ERR_NONFINITE = 9,   /* device: a non-finite per-row statistic            */
-  FLCE_ERR_DEVICE = 10      /* current device is not sm_100 / cannot run kernels */
+  FLCE_ERR_DEVICE = 10,     /* current device is not sm_100 / cannot run kernels */
+  FLCE_ERR_ARG = 11         /* an argument value is invalid (e.g. the reduction) */
 } flce_status;
 
 typedef enum { FLCE_BF16 = 0, FLCE_FP16 = 1 } flce_dtype;
@@ -168,6 +169,47 @@ FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const vo
                                           int64_t ignore_index, int64_t N, int64_t D, int64_t V,
                                           int dtype, float* loss, float* m, float* logs,
                                           flce_stream stream);
+
+/*
+ * Reductions of the per-row losses l_i = (m_i - Z_{i,y_i}) + log s_i, with
+ * optional per-row weights w_i (1 when `weight` is NULL).  MEAN is the
+ * objective of the page's §01; SUM and NONE are the reductions of NeMo's
+ * ChunkedCrossEntropy ("reduction", "num_label_tokens", "loss_weights"):
+ *   FLCE_REDUCE_MEAN  L = (1/C) sum_i w_i l_i
+ *   FLCE_REDUCE_SUM   L = (1/denom) sum_i w_i l_i   (denom <= 0 means 1)
+ *   FLCE_REDUCE_NONE  loss_rows[i] = w_i l_i, 0 for unsupervised rows
+ */
+typedef enum { FLCE_REDUCE_MEAN = 0, FLCE_REDUCE_SUM = 1, FLCE_REDUCE_NONE = 2 } flce_reduction;
+
+/*
+ * Forward with a reduction.  weight: device float [N] or NULL.  loss: device
+ * scalar, required for MEAN and SUM (ignored for NONE); loss_rows: device
+ * float [N], required for NONE (ignored otherwise).  m and logs as in
+ * flce_forward().  flce_forward() is this call with weight NULL and MEAN.
+ */
+FLCE_API flce_status flce_forward_ex(const void* H, const void* W, const void* b,
+                                     const int64_t* labels, const uint8_t* mask,
+                                     int64_t ignore_index, int64_t N, int64_t D, int64_t V,
+                                     int dtype, const float* weight, int reduction, float denom,
+                                     float* loss, float* loss_rows, float* m, float* logs,
+                                     void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * Backward of flce_forward_ex() (§04 with G_ij = s_i (p_ij - 1[j = y_i])):
+ *   MEAN  s_i = lambda w_i / C        SUM  s_i = lambda w_i / denom
+ *   NONE  s_i = grad_rows[i] w_i      (grad_rows: device float [N], the
+ *                                      upstream gradient of each row's loss)
+ * lambda / lambda_dev as in flce_backward() (unused for NONE).
+ * flce_backward() is this call with weight NULL and MEAN.
+ */
+FLCE_API flce_status flce_backward_ex(const void* H, const void* W, const void* b,
+                                      const int64_t* labels, const uint8_t* mask,
+                                      int64_t ignore_index, int64_t N, int64_t D, int64_t V,
+                                      int dtype, const float* m, const float* logs,
+                                      const float* weight, int reduction, float denom,
+                                      float lambda, const float* lambda_dev,
+                                      const float* grad_rows, float* dH, float* dW, float* db,
+                                      void* ws, size_t ws_bytes, flce_stream stream);
 
 /* Synchronises `stream`, then reads and returns the device error word of the
  * workspace (FLCE_OK when no device error was recorded by the last call). */

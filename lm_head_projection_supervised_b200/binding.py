@@ -19,7 +19,9 @@ LIB_PATH = os.path.join(HERE, "libflce.so")
 FLCE_BF16, FLCE_FP16 = 0, 1
 STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DTYPE",
           4: "FLCE_ERR_ALIGN", 5: "FLCE_ERR_WORKSPACE", 6: "FLCE_ERR_CUDA", 7: "FLCE_ERR_LABEL",
-          8: "FLCE_ERR_TIMEOUT", 9: "FLCE_ERR_NONFINITE", 10: "FLCE_ERR_DEVICE"}
+          8: "FLCE_ERR_TIMEOUT", 9: "FLCE_ERR_NONFINITE", 10: "FLCE_ERR_DEVICE",
+          11: "FLCE_ERR_ARG"}
+REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 _lib = None
@@ -54,6 +56,12 @@ def lib() -> ctypes.CDLL:
     L.flce_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, f32, vp, vp,
                                 vp, vp, vp, sz, vp]
     L.flce_backward.restype = i32
+    L.flce_forward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, i32, f32, vp,
+                                  vp, vp, vp, vp, sz, vp]
+    L.flce_forward_ex.restype = i32
+    L.flce_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, i32,
+                                   f32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.flce_backward_ex.restype = i32
     L.flce_device_status.argtypes = [vp, vp]
     L.flce_device_status.restype = i32
     L.flce_diag_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, f32, vp, sz, vp]
@@ -147,30 +155,53 @@ def _prep(H, W, b, labels, mask):
     return H2, W2, b2, y, mk
 
 
+def _vec(t, N, device):
+    """float32 contiguous [N] device vector (or None)."""
+    if t is None:
+        return None
+    t = t.reshape(-1).to(device=device, dtype=torch.float32).contiguous()
+    if t.numel() != N:
+        raise ValueError("per-row vectors must have one entry per row of H")
+    return t
+
+
 def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[Workspace] = None,
-            stream=None):
-    """loss (0-d float32), m [N], logs [N] -- flce_forward()."""
+            stream=None, weight=None, reduction: str = "mean", denom: Optional[float] = None):
+    """(loss, m [N], logs [N]) -- flce_forward_ex().
+
+    loss is a 0-d float32 for "mean" and "sum", and the per-row losses [N] for
+    "none"; weight ([N], optional) multiplies each row's loss; denom divides
+    the "sum" (e.g. a global label count)."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
+    red = REDUCTIONS[reduction]
     if ws is None:
         ws = Workspace(N, D, V, H2.dtype, H2.device)
+    wt = _vec(weight, N, H2.device)
     loss = torch.empty((), dtype=torch.float32, device=H2.device)
+    rows = torch.empty(N, dtype=torch.float32, device=H2.device) if reduction == "none" else None
     m = torch.empty(N, dtype=torch.float32, device=H2.device)
     logs = torch.empty(N, dtype=torch.float32, device=H2.device)
-    st = lib().flce_forward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D, V,
-                            dtype_code(H2.dtype), _ptr(loss), _ptr(m), _ptr(logs), ws.ptr(),
-                            ws.nbytes, _stream(stream))
-    _check(st, "flce_forward")
-    return loss, m, logs
+    st = lib().flce_forward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
+                               D, V, dtype_code(H2.dtype), _ptr(wt), red,
+                               float(denom or 0.0), _ptr(loss), _ptr(rows), _ptr(m), _ptr(logs),
+                               ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "flce_forward_ex")
+    return (rows if reduction == "none" else loss), m, logs
 
 
 def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0, lam_dev=None,
-             ws: Optional[Workspace] = None, out=None, stream=None):
-    """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward()."""
+             ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
+             reduction: str = "mean", denom: Optional[float] = None, grad_rows=None):
+    """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex().
+
+    For reduction "none", grad_rows [N] is the upstream gradient of each row's
+    loss; otherwise lam (or the device scalar lam_dev) is dJ/dL."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
+    red = REDUCTIONS[reduction]
     if ws is None:
         ws = Workspace(N, D, V, H2.dtype, H2.device)
     if out is None:
@@ -181,11 +212,14 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
         dH, dW, db = out
     if lam_dev is not None:
         lam_dev = lam_dev.reshape(()).to(torch.float32).contiguous()
-    st = lib().flce_backward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D,
-                             V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), float(lam),
-                             _ptr(lam_dev), _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
-                             _stream(stream))
-    _check(st, "flce_backward")
+    wt = _vec(weight, N, H2.device)
+    gr = _vec(grad_rows, N, H2.device)
+    st = lib().flce_backward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
+                                D, V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red,
+                                float(denom or 0.0), float(lam), _ptr(lam_dev), _ptr(gr),
+                                _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
+                                _stream(stream))
+    _check(st, "flce_backward_ex")
     return dH, dW, db
 
 
@@ -244,24 +278,56 @@ def profile_end():
 
 
 class FusedLinearCrossEntropy(torch.autograd.Function):
-    """L = mean over supervised rows of CE(H W^T + b, y); gradients from the
-    library's backward, with the upstream gradient passed on the device."""
+    """L = reduce_i w_i CE(H W^T + b, y)_i over the supervised rows; gradients
+    from the library's backward, with the upstream gradient kept on the
+    device (no host round trip)."""
 
     @staticmethod
-    def forward(ctx, H, W, b, labels, mask, ignore_index):
-        loss, m, logs = forward(H, W, b, labels, mask, ignore_index)
-        ctx.save_for_backward(H, W, b, labels, mask, m, logs)
-        ctx.ignore_index = ignore_index
+    def forward(ctx, H, W, b, labels, mask, ignore_index, weight=None, reduction="mean",
+                denom=None):
+        loss, m, logs = forward(H, W, b, labels, mask, ignore_index, weight=weight,
+                                reduction=reduction, denom=denom)
+        ctx.save_for_backward(H, W, b, labels, mask, m, logs, weight)
+        ctx.ignore_index, ctx.reduction, ctx.denom = ignore_index, reduction, denom
         return loss
 
     @staticmethod
     def backward(ctx, grad_out):
-        H, W, b, labels, mask, m, logs = ctx.saved_tensors
-        dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs,
-                              lam_dev=grad_out.detach())
+        H, W, b, labels, mask, m, logs, weight = ctx.saved_tensors
+        g = grad_out.detach()
+        if ctx.reduction == "none":
+            dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs,
+                                  weight=weight, reduction="none", grad_rows=g)
+        else:
+            dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs, lam_dev=g,
+                                  weight=weight, reduction=ctx.reduction, denom=ctx.denom)
         return (dH.reshape(H.shape).to(H.dtype), dW.to(W.dtype),
-                None if db is None else db.to(b.dtype), None, None, None)
+                None if db is None else db.to(b.dtype), None, None, None, None, None, None)
 
 
-def fused_linear_cross_entropy(H, W, labels, b=None, mask=None, ignore_index: int = -100):
-    return FusedLinearCrossEntropy.apply(H, W, b, labels, mask, ignore_index)
+def fused_linear_cross_entropy(H, W, labels, b=None, mask=None, ignore_index: int = -100,
+                               weight=None, reduction: str = "mean", denom=None):
+    return FusedLinearCrossEntropy.apply(H, W, b, labels, mask, ignore_index, weight, reduction,
+                                         denom)
+
+
+class LinearCrossEntropyLoss(torch.nn.Module):
+    """Loss module over final hidden states and the projection weight, with
+    the reductions of a chunked linear cross-entropy loss ("mean", "sum",
+    "none"), an optional global label count for "sum" and optional per-token
+    loss weights.  Hidden states may have any leading token dimensions."""
+
+    def __init__(self, ignore_index: int = -100, reduction: str = "mean"):
+        super().__init__()
+        if reduction not in REDUCTIONS:
+            raise ValueError(f"reduction must be one of {tuple(REDUCTIONS)}")
+        self.ignore_index = ignore_index
+        self.reduction = reduction
+
+    def forward(self, hidden_states, labels, lm_weight, bias=None, num_label_tokens=None,
+                loss_weights=None, mask=None):
+        lead = hidden_states.shape[:-1]
+        out = fused_linear_cross_entropy(hidden_states, lm_weight, labels, b=bias, mask=mask,
+                                         ignore_index=self.ignore_index, weight=loss_weights,
+                                         reduction=self.reduction, denom=num_label_tokens)
+        return out.reshape(lead) if self.reduction == "none" else out

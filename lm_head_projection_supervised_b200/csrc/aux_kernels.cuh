@@ -25,12 +25,13 @@ __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8
 // set the label error bit and are clamped to 0 so later indexing stays in
 // range.  Unsupervised rows get m = log s = -inf when m_out is given.
 // pos (optional) is the inverse map: pos[i] = compact row of i, or -1.
+// lossvec (optional) gets 0 on unsupervised rows (per-row loss output).
 __global__ void __launch_bounds__(COMPACT_THREADS)
     compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
                    int64_t ignore, int64_t N, int64_t V, int* __restrict__ idx,
                    int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
                    float* __restrict__ m_out, float* __restrict__ logs_out,
-                   int* __restrict__ pos) {
+                   int* __restrict__ pos, float* __restrict__ lossvec) {
   __shared__ int warp_tot[COMPACT_THREADS / 32];
   const int t = threadIdx.x;
   const int64_t per = (N + COMPACT_THREADS - 1) / COMPACT_THREADS;
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
         logs_out[i] = -INFINITY;
       }
       if (pos != nullptr) pos[i] = -1;
+      if (lossvec != nullptr) lossvec[i] = 0.f;
     }
   }
   if (bad) atomicOr(err, kErrBitLabel);
@@ -121,11 +123,13 @@ __device__ __forceinline__ void merge_state(float& m, float& s, float om, float 
 // Per supervised row: merge the per-vocabulary-tile partials (lane-strided,
 // then a butterfly of warp shuffles, symmetric so that every lane ends with
 // the same state), then m_i, log s_i and l_i = (m_i - target_i) + log s_i.
+// loss_rows[i] = w_i l_i (compact order); lossvec[orig] = w_i l_i if given.
 __global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld, int nvt,
                                    const float* __restrict__ tgt, const int* __restrict__ C_dev,
                                    const int* __restrict__ idx, float* __restrict__ m_out,
                                    float* __restrict__ logs_out, float* __restrict__ loss_rows,
-                                   uint32_t* err) {
+                                   const float* __restrict__ weight,
+                                   float* __restrict__ lossvec, uint32_t* err) {
   const int C = *C_dev;
   const int lane = threadIdx.x & 31;
   const int warps = (blockDim.x >> 5) * gridDim.x;
@@ -148,17 +152,20 @@ __global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld,
       const int o = idx[i];
       m_out[o] = m;
       logs_out[o] = logs;
-      loss_rows[i] = li;
+      const float wl = (weight != nullptr) ? weight[o] * li : li;
+      loss_rows[i] = wl;
+      if (lossvec != nullptr) lossvec[o] = wl;
       if (!isfinite(li) || !isfinite(m) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
     }
   }
 }
 
-// L = (1/C) sum_i l_i in a fixed order (per-thread strided sums in double,
-// then a fixed tree); 0 when C = 0; NaN when the label or timeout bit is set.
+// L = sum_i loss_rows[i] / den in a fixed order (per-thread strided sums in
+// double, then a fixed tree), den = C for the mean and `denom` (or 1) for the
+// sum; 0 when C = 0; NaN when the label or timeout bit is set.
 __global__ void __launch_bounds__(1024)
-    loss_mean_kernel(const float* __restrict__ loss_rows, const int* __restrict__ C_dev,
-                     const uint32_t* err, float* __restrict__ loss) {
+    loss_reduce_kernel(const float* __restrict__ loss_rows, const int* __restrict__ C_dev,
+                       int is_mean, float denom, const uint32_t* err, float* __restrict__ loss) {
   __shared__ double red[1024];
   const int C = *C_dev;
   double acc = 0.0;
@@ -170,17 +177,55 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    float L = (C > 0) ? static_cast<float>(red[0] / C) : 0.f;
+    const double den = is_mean ? static_cast<double>(C) : (denom > 0.f ? denom : 1.0);
+    float L = (C > 0) ? static_cast<float>(red[0] / den) : 0.f;
     if (*err & (kErrBitLabel | kErrBitTimeout)) L = __int_as_float(0x7fc00000);
     *loss = L;
   }
 }
 
-// db[vp + j] = scale * sum_{i < C} Gp[i][j] for the panel's columns, in a
+// Backward row scales: s_k = lambda w_o / den (mean, sum) or g_o w_o (per-row
+// upstream gradients), o = idx[k].  Stores r_k = s_k / S and *scal = S with
+// S = max_k |s_k| (r = 0 when S = 0), so that the 16-bit gradient panel holds
+// r_k (p - onehot) sigma in range and the contractions multiply by S / sigma.
+// One block, fixed-order reduction.
+__global__ void __launch_bounds__(1024)
+    row_scale_kernel(const int* __restrict__ C_dev, const int* __restrict__ idx,
+                     const float* __restrict__ weight, const float* __restrict__ grad_rows,
+                     int reduction, float denom, float lam, const float* __restrict__ lam_dev,
+                     float* __restrict__ r, float* __restrict__ scal) {
+  __shared__ float red[1024];
+  const int C = *C_dev;
+  float base = 0.f;
+  if (grad_rows == nullptr) {
+    const float l = (lam_dev != nullptr) ? *lam_dev : lam;
+    const float den = (reduction == 0) ? static_cast<float>(C) : (denom > 0.f ? denom : 1.f);
+    base = (C > 0) ? l / den : 0.f;
+  }
+  float mx = 0.f;
+  for (int k = threadIdx.x; k < C; k += blockDim.x) {
+    const int o = idx[k];
+    float sk = (grad_rows != nullptr) ? grad_rows[o] : base;
+    if (weight != nullptr) sk *= weight[o];
+    r[k] = sk;
+    mx = fmaxf(mx, fabsf(sk));
+  }
+  red[threadIdx.x] = mx;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
+    __syncthreads();
+  }
+  const float S = red[0];
+  for (int k = threadIdx.x; k < C; k += blockDim.x) r[k] = (S > 0.f) ? r[k] / S : 0.f;
+  if (threadIdx.x == 0) *scal = S;
+}
+
+// db[vp + j] = (S / sigma) * sum_{i < C} Gp[i][j] for the panel's columns, in a
 // fixed order: 8 row groups per block, combined in group order.
 __global__ void __launch_bounds__(256)
     bias_grad_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
-                     const int* __restrict__ C_dev, float lam, const float* lam_dev,
+                     const int* __restrict__ C_dev, const float* __restrict__ scal,
                      float inv_sigma, int is_bf16, int vp, float* __restrict__ db) {
   __shared__ float2 part[8][32];
   const int C = *C_dev;
@@ -209,8 +254,7 @@ __global__ void __launch_bounds__(256)
       t.x += part[k][lane].x;
       t.y += part[k][lane].y;
     }
-    const float lam_v = (lam_dev != nullptr) ? *lam_dev : lam;
-    const float scale = (C > 0) ? lam_v / static_cast<float>(C) * inv_sigma : 0.f;
+    const float scale = (C > 0) ? *scal * inv_sigma : 0.f;
     db[vp + j] = t.x * scale;
     if (j + 1 < w) db[vp + j + 1] = t.y * scale;
   }

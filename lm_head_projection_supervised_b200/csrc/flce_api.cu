@@ -11,7 +11,8 @@
 //                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 2
 //                     bias_grad of panel L (bias only, if L < P)
 //   -> scatter dH_c to dH (zero rows for unsupervised positions)
-//   with scale = lambda / (C sigma) applied in the dW / dH epilogues.
+//   with row scales s_k = S r_k computed first (row_scale_kernel); the panels
+//   hold r_k (p - onehot) sigma and the dW / dH epilogues multiply by S / sigma.
 #include <mutex>
 #include <vector>
 
@@ -39,7 +40,7 @@ int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, dhc, gpanel[2], total;
+  size_t pos, rs, dhc, gpanel[2], total;
   int64_t Np, nvt, vc, panels;
 };
 
@@ -69,6 +70,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
   L.fwd_total = off;
   L.pos = take(static_cast<size_t>(L.Np) * 4);
+  L.rs = take(static_cast<size_t>(L.Np) * 4);
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
   L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.vc * 2);
   L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.vc * 2);
@@ -248,6 +250,7 @@ struct WsPtrs {
   uint32_t* err;
   int* counters;
   int* C;
+  float* scal;  // backward: S = max_k |s_k|
   int* idx;
   int* yc;
   int* pos;
@@ -255,6 +258,7 @@ struct WsPtrs {
   float2* part;
   float* tgt;
   float* loss_rows;
+  float* rs;
   float* dhc;
   uint16_t* gpanel[2];
 };
@@ -265,6 +269,7 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.err = reinterpret_cast<uint32_t*>(w + L.ctrl);
   p.counters = reinterpret_cast<int*>(w + L.ctrl + kCounterOffset);
   p.C = reinterpret_cast<int*>(w + L.C);
+  p.scal = reinterpret_cast<float*>(w + L.C + 64);
   p.idx = reinterpret_cast<int*>(w + L.idx);
   p.yc = reinterpret_cast<int*>(w + L.yc);
   p.pos = reinterpret_cast<int*>(w + L.pos);
@@ -272,6 +277,7 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.part = reinterpret_cast<float2*>(w + L.part);
   p.tgt = reinterpret_cast<float*>(w + L.tgt);
   p.loss_rows = reinterpret_cast<float*>(w + L.loss_rows);
+  p.rs = reinterpret_cast<float*>(w + L.rs);
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
   p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
   p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
@@ -281,11 +287,12 @@ WsPtrs carve(void* ws, const Layout& L) {
 // control block reset + compaction + gather of the supervised rows
 flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
                      int64_t N, int64_t D, int64_t V, const Layout& L, const WsPtrs& p,
-                     float* m_out, float* logs_out, int* pos, cudaStream_t s) {
+                     float* m_out, float* logs_out, int* pos, float* lossvec,
+                     cudaStream_t s) {
   FLCE_CK(cudaMemsetAsync(p.err, 0, L.ctrl_bytes, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, p.idx, p.yc, p.C,
-                                                 p.err, m_out, logs_out, pos);
+                                                 p.err, m_out, logs_out, pos, lossvec);
   }));
   const int64_t vec = D / 8;
   FLCE_CK(timed_launch(kProfAux, s, [&] {
@@ -317,6 +324,7 @@ const char* flce_status_string(int status) {
     case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT: a device pipeline wait ran out";
     case FLCE_ERR_NONFINITE: return "FLCE_ERR_NONFINITE: non-finite per-row statistic";
     case FLCE_ERR_DEVICE: return "FLCE_ERR_DEVICE: current device is not sm_100";
+    case FLCE_ERR_ARG: return "FLCE_ERR_ARG: invalid argument value";
     default: return "FLCE_ERR_UNKNOWN";
   }
 }
@@ -337,7 +345,7 @@ flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ign
   FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, idx, nullptr,
-                                                 C_out, err, nullptr, nullptr, nullptr);
+                                                 C_out, err, nullptr, nullptr, nullptr, nullptr);
   }));
   return FLCE_OK;
 }
@@ -346,13 +354,28 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
                          const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
                          int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
                          size_t ws_bytes, flce_stream stream) {
-  if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr)) ||
-      W == nullptr || loss == nullptr || ws == nullptr)
+  return flce_forward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, nullptr,
+                         FLCE_REDUCE_MEAN, 0.f, loss, nullptr, m, logs, ws, ws_bytes, stream);
+}
+
+flce_status flce_forward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
+                            const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                            int64_t V, int dtype, const float* weight, int reduction, float denom,
+                            float* loss, float* loss_rows, float* m, float* logs, void* ws,
+                            size_t ws_bytes, flce_stream stream) {
+  if (reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
+      reduction != FLCE_REDUCE_NONE)
+    return FLCE_ERR_ARG;
+  const bool none = reduction == FLCE_REDUCE_NONE;
+  if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
+                 (none && loss_rows == nullptr))) ||
+      W == nullptr || (!none && loss == nullptr) || ws == nullptr)
     return FLCE_ERR_NULL;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
   if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
   if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
-      !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) || !aligned(loss, 4))
+      !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) || !aligned(loss, 4) ||
+      !aligned(weight, 4) || !aligned(loss_rows, 4))
     return FLCE_ERR_ALIGN;
   const Layout L = make_layout(N, D, V);
   if (ws_bytes < L.fwd_total) return FLCE_ERR_WORKSPACE;
@@ -364,7 +387,8 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
   const bool bf16 = dtype == FLCE_BF16;
   const MapType mt = bf16 ? kMapBF16 : kMapFP16;
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, nullptr, s);
+  float* lossvec = none ? loss_rows : nullptr;
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, nullptr, lossvec, s);
   if (st != FLCE_OK) return st;
 
   GemmArgs a{};
@@ -392,12 +416,16 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
           p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
-          p.loss_rows, p.err);
+          p.loss_rows, weight, lossvec, p.err);
     }));
   }
-  FLCE_CK(timed_launch(kProfAux, s, [&] {
-    loss_mean_kernel<<<1, 1024, 0, s>>>(p.loss_rows, p.C, p.err, loss);
-  }));
+  if (!none) {
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      loss_reduce_kernel<<<1, 1024, 0, s>>>(p.loss_rows, p.C,
+                                            reduction == FLCE_REDUCE_MEAN ? 1 : 0, denom, p.err,
+                                            loss);
+    }));
+  }
   return FLCE_OK;
 }
 
@@ -406,15 +434,32 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
                           int64_t V, int dtype, const float* m, const float* logs, float lambda,
                           const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
                           size_t ws_bytes, flce_stream stream) {
+  return flce_backward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, m, logs, nullptr,
+                          FLCE_REDUCE_MEAN, 0.f, lambda, lambda_dev, nullptr, dH, dW, db, ws,
+                          ws_bytes, stream);
+}
+
+flce_status flce_backward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
+                             const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                             int64_t V, int dtype, const float* m, const float* logs,
+                             const float* weight, int reduction, float denom, float lambda,
+                             const float* lambda_dev, const float* grad_rows, float* dH,
+                             float* dW, float* db, void* ws, size_t ws_bytes,
+                             flce_stream stream) {
+  if (reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
+      reduction != FLCE_REDUCE_NONE)
+    return FLCE_ERR_ARG;
+  const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
-                 dH == nullptr)) ||
+                 dH == nullptr || (none && grad_rows == nullptr))) ||
       W == nullptr || dW == nullptr || ws == nullptr || (b != nullptr && db == nullptr))
     return FLCE_ERR_NULL;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
   if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
   if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
       !aligned(ws, 256) || !aligned(dH, 16) || !aligned(dW, 16) ||
-      (db != nullptr && !aligned(db, 8)) || !aligned(m, 4) || !aligned(logs, 4))
+      (db != nullptr && !aligned(db, 8)) || !aligned(m, 4) || !aligned(logs, 4) ||
+      !aligned(weight, 4) || !aligned(grad_rows, 4))
     return FLCE_ERR_ALIGN;
   const Layout L = make_layout(N, D, V);
   if (ws_bytes < L.total) return FLCE_ERR_WORKSPACE;
@@ -428,8 +473,13 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, p.pos, s);
+  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, p.pos, nullptr,
+                s);
   if (st != FLCE_OK) return st;
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    row_scale_kernel<<<1, 1024, 0, s>>>(p.C, p.idx, weight, none ? grad_rows : nullptr,
+                                        reduction, denom, lambda, lambda_dev, p.rs, p.scal);
+  }));
 
   // maps that do not depend on the panel
   CUtensorMap hcK, wK, hcMN, wMN, dwMap, dhMap;
@@ -485,8 +535,8 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
     a.logs_saved = logs;
     a.log2_sigma = log2_sigma;
     a.sigma = sigma;
-    a.lam = lambda;
-    a.lam_dev = lambda_dev;
+    a.row_scale = p.rs;
+    a.scal = p.scal;
     a.inv_sigma = 1.f / sigma;
     a.err = p.err;
     const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +
@@ -497,7 +547,7 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
       const uint16_t* gp = p.gpanel[Lp & 1];
       FLCE_CK(timed_launch(kProfAux, s, [&] {
         bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w_g, 64)), 256, 0, s>>>(
-            gp, L.vc, static_cast<int>(w_g), p.C, lambda, lambda_dev, 1.f / sigma, bf16 ? 1 : 0,
+            gp, L.vc, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma, bf16 ? 1 : 0,
             static_cast<int>(vp_g), db);
       }));
     }

@@ -27,6 +27,8 @@
 //                 statistics, subtracts the one-hot target (§04), rounds to
 //                 the 16-bit input type, stages 128 x 64 boxes in shared
 //                 memory and stores them with TMA into gradient buffer p % 2;
+//              The panel holds r_k (p - onehot) sigma with the row scale
+//              s_k = S r_k (S = max |s_k|), the contractions multiply by S / sigma.
 //              class 0 (dW): dW[panel p-1 rows] = G^T H_c  (K = C), stored by TMA;
 //              class 1 (dH): dH_c (+)= G W[panel p-1]      (K = panel width),
 //                 stored (first panel) or added with a TMA reduction (later
@@ -104,8 +106,8 @@ struct GemmArgs {
   const float* logs_saved;
   float log2_sigma;        // bwd: the panel holds (p - onehot) * sigma
   float sigma;
-  float lam;               // bwd: upstream gradient
-  const float* lam_dev;    //      (device copy, overrides lam when set)
+  const float* row_scale;  // bwd: r_k, relative row scale of compact row k, in [-1, 1]
+  const float* scal;       // bwd: S (device scalar); G = S r_k (p - onehot)
   float inv_sigma;
   float* out;              // plain
   float scale;             // plain
@@ -340,7 +342,7 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
                                            int vglob0, int vlim, int yl, bool valid, float mrow,
-                                           float krow, uint32_t (&packed)[16]) {
+                                           float krow, float rrow, uint32_t (&packed)[16]) {
   float x[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(z[j]);
@@ -369,6 +371,8 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
     for (int j = 0; j < 32; ++j)
       if (j == jt) gv[j] -= g.sigma;
   }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) gv[j] *= rrow;  // the row's scale relative to S
   if (g.is_bf16) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -597,10 +601,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     uint32_t acc_phase = 0;
     uint32_t nstore = 0;  // TMA stores issued by this CTA (staging buffer parity)
     float wh_scale = 0.f;
-    if (MODE == kModeBwd) {
-      const float lam = (g.lam_dev != nullptr) ? *g.lam_dev : g.lam;
-      wh_scale = (C > 0) ? lam / static_cast<float>(C) * g.inv_sigma : 0.f;
-    }
+    if (MODE == kModeBwd) wh_scale = (C > 0) ? *g.scal * g.inv_sigma : 0.f;
     // Shared decision of the four epilogue warps (they pass named barriers
     // together, so they leave the loop together).
     int round = 0;
@@ -646,7 +647,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       const int row = tm0 + r;
       bool valid = false;
       int yl = -1000000;
-      float mrow = 0.f, krow = 0.f;
+      float mrow = 0.f, krow = 0.f, rrow = 0.f;
       int vglob0 = 0, vlim = 0;
       if (MODE == kModeFwd || (MODE == kModeBwd && un.cls == kClsGrad)) {
         valid = row < C;
@@ -657,6 +658,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           const int o = __ldg(g.idx + row);
           mrow = __ldg(g.m_saved + o);
           krow = g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e;
+          rrow = __ldg(g.row_scale + row);
         }
       } else if (MODE == kModePlain) {
         valid = row < g.M;
@@ -700,11 +702,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           named_bar_sync(1, NUM_EPI_THREADS);
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
-          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, pk);
+          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, pk);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
           if (c + 2 < BN / 32) tmem_ld32(t_acc + (c + 2) * 32, za);
-          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, pk);
+          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, pk);
           stage_row128(stg, r, 4, pk);
           if (c + 2 < BN / 32) tmem_wait_ld(za);
           fence_proxy_async_smem();
