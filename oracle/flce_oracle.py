@@ -74,14 +74,28 @@ def _check_labels(labels, idx, V):
     return y
 
 
-def _rows_stats(Hs, W, b, y):
+LOGIT_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+def _logits(Hs, W, b, logits_dtype=None):
+    """Z = H W^T + b; with logits_dtype the logits are first rounded to
+    float32 and then to the 16-bit model dtype (round to nearest even, torch's
+    CPU casts), as a projection that outputs the model dtype does (NeMo
+    ``logits_dtype``; the bf16 logits of "ChunkedLinearCrossEntropy")."""
+    Z = Hs @ W.T
+    if b is not None:
+        Z = Z + b
+    if logits_dtype is not None:
+        Z = Z.to(torch.float32).to(LOGIT_DTYPES[logits_dtype]).to(torch.float64)
+    return Z
+
+
+def _rows_stats(Hs, W, b, y, logits_dtype=None):
     """Dense full-vocabulary statistics of a block of rows.
 
     Returns Z (rows x V), m, log s, the target logits and the per-row loss
     (m - Z_y) + log s (§02)."""
-    Z = Hs @ W.T
-    if b is not None:
-        Z = Z + b
+    Z = _logits(Hs, W, b, logits_dtype)
     m = Z.max(dim=1).values
     s = torch.exp(Z - m[:, None]).sum(dim=1)
     logs = torch.log(s)
@@ -110,7 +124,8 @@ def _denominator(reduction, C, denom):
 
 
 def forward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
-            row_block: int = 512, weight=None, reduction: str = "mean", denom=None):
+            row_block: int = 512, weight=None, reduction: str = "mean", denom=None,
+            logits_dtype=None):
     """Loss and saved statistics (§01, §02), dense in the vocabulary.
 
     reduction "mean" is the objective of p2 §01, (1/C) sum_i w_i l_i; "sum"
@@ -134,7 +149,7 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
     for r0 in range(0, C, row_block):
         r1 = min(C, r0 + row_block)
         rows = torch.as_tensor(idx[r0:r1])
-        _, mb, lb, _, lr = _rows_stats(H[rows], W, b, y[r0:r1])
+        _, mb, lb, _, lr = _rows_stats(H[rows], W, b, y[r0:r1], logits_dtype)
         m[rows], logs[rows], loss_rows[r0:r1] = mb, lb, lr
     w = _row_weights(weight, idx)
     loss_vec = torch.zeros(N, dtype=torch.float64)
@@ -167,7 +182,7 @@ def row_scales(labels, mask, ignore_index, lam, weight=None, reduction="mean", d
 
 def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
              lam: float = 1.0, m=None, logs=None, row_block: int = 512, weight=None,
-             reduction: str = "mean", denom=None, grad_rows=None):
+             reduction: str = "mean", denom=None, grad_rows=None, logits_dtype=None):
     """dH, dW, db from the reconstruction of §04, dense in the vocabulary.
 
     m and logs are the saved statistics (recomputed here when not given).
@@ -183,7 +198,7 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
         return dH.numpy(), dW.numpy(), (None if db is None else db.numpy())
     if m is None or logs is None:
         st = forward(H.numpy(), W.numpy(), None if bt is None else bt.numpy(), labels, mask,
-                     ignore_index, row_block)
+                     ignore_index, row_block, logits_dtype=logits_dtype)
         m, logs = st["m"], st["logs"]
     m, logs = _f64(m), _f64(logs)
     scale = row_scales(labels, mask, ignore_index, lam, weight, reduction, denom, grad_rows)
@@ -191,9 +206,7 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
         r1 = min(C, r0 + row_block)
         rows = torch.as_tensor(idx[r0:r1])
         Hs = H[rows]
-        Z = Hs @ W.T
-        if bt is not None:
-            Z = Z + bt
+        Z = _logits(Hs, W, bt, logits_dtype)  # the rounding passes the gradient through
         P = torch.exp((Z - m[rows][:, None]) - logs[rows][:, None])
         P[torch.arange(r1 - r0), torch.as_tensor(y[r0:r1])] -= 1.0
         G = scale[r0:r1, None] * P
@@ -206,10 +219,11 @@ def backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
 
 def forward_backward(H, W, b, labels, mask=None, ignore_index: int = IGNORE_INDEX,
                      lam: float = 1.0, row_block: int = 512, weight=None,
-                     reduction: str = "mean", denom=None, grad_rows=None):
-    f = forward(H, W, b, labels, mask, ignore_index, row_block, weight, reduction, denom)
+                     reduction: str = "mean", denom=None, grad_rows=None, logits_dtype=None):
+    f = forward(H, W, b, labels, mask, ignore_index, row_block, weight, reduction, denom,
+                logits_dtype)
     dH, dW, db = backward(H, W, b, labels, mask, ignore_index, lam, f["m"], f["logs"],
-                          row_block, weight, reduction, denom, grad_rows)
+                          row_block, weight, reduction, denom, grad_rows, logits_dtype)
     f.update(dH=dH, dW=dW, db=db)
     return f
 

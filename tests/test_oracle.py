@@ -402,3 +402,33 @@ def test_weighted_sum_finite_differences():
         fd = (orc.forward(H, W, bp, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]
               - orc.forward(H, W, bm, y, mask, weight=w, reduction="sum", denom=4.0)["loss"]) / (2 * eps)
         assert abs(fd - f["db"][j]) < 1e-8
+
+
+# --- logits rounded to the model dtype (opt-in variant) -----------------------
+
+@pytest.mark.parametrize("dt,tdt", [("bf16", torch.bfloat16), ("fp16", torch.float16)])
+def test_rounded_logits_match_torch_autograd(dt, tdt):
+    """Logits cast to the 16-bit dtype before the loss, gradient passed through
+    the cast: torch float64 autograd over an explicit round-trip cast."""
+    H, W, b, y, mask = _case(23, N=30, D=8, V=80)
+    f = orc.forward_backward(H, W, b, y, mask, lam=1.1, logits_dtype=dt)
+    Ht = torch.tensor(H, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    Z = Ht @ Wt.T + bt
+    Zr = Z + (Z.detach().to(torch.float32).to(tdt).to(torch.float64) - Z.detach())
+    yy = torch.tensor(np.where(mask.astype(bool), y, -100))
+    L = torch.nn.functional.cross_entropy(Zr, yy, ignore_index=-100)
+    (1.1 * L).backward()
+    assert abs(f["loss"] - L.item()) < 1e-12
+    assert _close(f["dH"], Ht.grad.numpy()) and _close(f["dW"], Wt.grad.numpy())
+    assert _close(f["db"], bt.grad.numpy())
+    # the rounding changes the result (the variant is not a no-op)
+    assert abs(orc.forward(H, W, b, y, mask)["loss"] - f["loss"]) > 1e-9
+
+
+def test_rounded_logits_are_exact_16bit_values():
+    H, W, b, y, mask = _case(24, N=5, D=4, V=11)
+    Z = orc._logits(torch.tensor(H), torch.tensor(W), torch.tensor(b), "bf16")
+    Zb = Z.to(torch.bfloat16).to(torch.float64)
+    assert torch.equal(Z, Zb)
