@@ -181,17 +181,27 @@ FLCE_API flce_status flce_forward_noalloc(const void* H, const void* W, const vo
  */
 typedef enum { FLCE_REDUCE_MEAN = 0, FLCE_REDUCE_SUM = 1, FLCE_REDUCE_NONE = 2 } flce_reduction;
 
+/* Option bits of the _ex calls.
+ * FLCE_FLAG_ROUND_LOGITS: each logit (after the bias) is rounded from fp32 to
+ *   the input dtype before the loss, as a projection that outputs the model
+ *   dtype does (NeMo "logits_dtype"; the bf16 logits of the
+ *   ChunkedLinearCrossEntropy article).  The backward treats the rounding as
+ *   the identity.  Pass the same flags to the forward and the backward. */
+#define FLCE_FLAG_ROUND_LOGITS 1u
+
 /*
  * Forward with a reduction.  weight: device float [N] or NULL.  loss: device
  * scalar, required for MEAN and SUM (ignored for NONE); loss_rows: device
  * float [N], required for NONE (ignored otherwise).  m and logs as in
- * flce_forward().  flce_forward() is this call with weight NULL and MEAN.
+ * flce_forward().  flags: FLCE_FLAG_* bits (0 for none).  flce_forward() is
+ * this call with weight NULL, MEAN and no flags.
  */
 FLCE_API flce_status flce_forward_ex(const void* H, const void* W, const void* b,
                                      const int64_t* labels, const uint8_t* mask,
                                      int64_t ignore_index, int64_t N, int64_t D, int64_t V,
                                      int dtype, const float* weight, int reduction, float denom,
-                                     float* loss, float* loss_rows, float* m, float* logs,
+                                     unsigned flags, float* loss, float* loss_rows, float* m,
+                                     float* logs,
                                      void* ws, size_t ws_bytes, flce_stream stream);
 
 /*
@@ -200,14 +210,15 @@ FLCE_API flce_status flce_forward_ex(const void* H, const void* W, const void* b
  *   NONE  s_i = grad_rows[i] w_i      (grad_rows: device float [N], the
  *                                      upstream gradient of each row's loss)
  * lambda / lambda_dev as in flce_backward() (unused for NONE).
- * flce_backward() is this call with weight NULL and MEAN.
+ * flags as given to the forward.  flce_backward() is this call with weight
+ * NULL, MEAN and no flags.
  */
 FLCE_API flce_status flce_backward_ex(const void* H, const void* W, const void* b,
                                       const int64_t* labels, const uint8_t* mask,
                                       int64_t ignore_index, int64_t N, int64_t D, int64_t V,
                                       int dtype, const float* m, const float* logs,
                                       const float* weight, int reduction, float denom,
-                                      float lambda, const float* lambda_dev,
+                                      unsigned flags, float lambda, const float* lambda_dev,
                                       const float* grad_rows, float* dH, float* dW, float* db,
                                       void* ws, size_t ws_bytes, flce_stream stream);
 

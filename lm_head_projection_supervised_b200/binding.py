@@ -22,6 +22,7 @@ STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DT
           8: "FLCE_ERR_TIMEOUT", 9: "FLCE_ERR_NONFINITE", 10: "FLCE_ERR_DEVICE",
           11: "FLCE_ERR_ARG"}
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
+FLAG_ROUND_LOGITS = 1
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 _lib = None
@@ -56,11 +57,12 @@ def lib() -> ctypes.CDLL:
     L.flce_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, f32, vp, vp,
                                 vp, vp, vp, sz, vp]
     L.flce_backward.restype = i32
-    L.flce_forward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, i32, f32, vp,
-                                  vp, vp, vp, vp, sz, vp]
+    u32 = ctypes.c_uint
+    L.flce_forward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, i32, f32, u32,
+                                  vp, vp, vp, vp, vp, sz, vp]
     L.flce_forward_ex.restype = i32
     L.flce_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, i32,
-                                   f32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+                                   f32, u32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.flce_backward_ex.restype = i32
     L.flce_device_status.argtypes = [vp, vp]
     L.flce_device_status.restype = i32
@@ -166,12 +168,14 @@ def _vec(t, N, device):
 
 
 def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[Workspace] = None,
-            stream=None, weight=None, reduction: str = "mean", denom: Optional[float] = None):
+            stream=None, weight=None, reduction: str = "mean", denom: Optional[float] = None,
+            round_logits: bool = False):
     """(loss, m [N], logs [N]) -- flce_forward_ex().
 
     loss is a 0-d float32 for "mean" and "sum", and the per-row losses [N] for
     "none"; weight ([N], optional) multiplies each row's loss; denom divides
-    the "sum" (e.g. a global label count)."""
+    the "sum" (e.g. a global label count); round_logits rounds each logit to
+    the input dtype before the loss."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
@@ -185,7 +189,8 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[W
     logs = torch.empty(N, dtype=torch.float32, device=H2.device)
     st = lib().flce_forward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
                                D, V, dtype_code(H2.dtype), _ptr(wt), red,
-                               float(denom or 0.0), _ptr(loss), _ptr(rows), _ptr(m), _ptr(logs),
+                               float(denom or 0.0), FLAG_ROUND_LOGITS if round_logits else 0,
+                               _ptr(loss), _ptr(rows), _ptr(m), _ptr(logs),
                                ws.ptr(), ws.nbytes, _stream(stream))
     _check(st, "flce_forward_ex")
     return (rows if reduction == "none" else loss), m, logs
@@ -193,7 +198,8 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[W
 
 def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0, lam_dev=None,
              ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
-             reduction: str = "mean", denom: Optional[float] = None, grad_rows=None):
+             reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
+             round_logits: bool = False):
     """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex().
 
     For reduction "none", grad_rows [N] is the upstream gradient of each row's
@@ -216,7 +222,8 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
     gr = _vec(grad_rows, N, H2.device)
     st = lib().flce_backward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
                                 D, V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red,
-                                float(denom or 0.0), float(lam), _ptr(lam_dev), _ptr(gr),
+                                float(denom or 0.0), FLAG_ROUND_LOGITS if round_logits else 0,
+                                float(lam), _ptr(lam_dev), _ptr(gr),
                                 _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
                                 _stream(stream))
     _check(st, "flce_backward_ex")
@@ -284,11 +291,12 @@ class FusedLinearCrossEntropy(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, H, W, b, labels, mask, ignore_index, weight=None, reduction="mean",
-                denom=None):
+                denom=None, round_logits=False):
         loss, m, logs = forward(H, W, b, labels, mask, ignore_index, weight=weight,
-                                reduction=reduction, denom=denom)
+                                reduction=reduction, denom=denom, round_logits=round_logits)
         ctx.save_for_backward(H, W, b, labels, mask, m, logs, weight)
         ctx.ignore_index, ctx.reduction, ctx.denom = ignore_index, reduction, denom
+        ctx.round_logits = round_logits
         return loss
 
     @staticmethod
@@ -297,37 +305,45 @@ class FusedLinearCrossEntropy(torch.autograd.Function):
         g = grad_out.detach()
         if ctx.reduction == "none":
             dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs,
-                                  weight=weight, reduction="none", grad_rows=g)
+                                  weight=weight, reduction="none", grad_rows=g,
+                                  round_logits=ctx.round_logits)
         else:
             dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs, lam_dev=g,
-                                  weight=weight, reduction=ctx.reduction, denom=ctx.denom)
+                                  weight=weight, reduction=ctx.reduction, denom=ctx.denom,
+                                  round_logits=ctx.round_logits)
         return (dH.reshape(H.shape).to(H.dtype), dW.to(W.dtype),
-                None if db is None else db.to(b.dtype), None, None, None, None, None, None)
+                None if db is None else db.to(b.dtype), None, None, None, None, None, None, None)
 
 
 def fused_linear_cross_entropy(H, W, labels, b=None, mask=None, ignore_index: int = -100,
-                               weight=None, reduction: str = "mean", denom=None):
+                               weight=None, reduction: str = "mean", denom=None,
+                               round_logits: bool = False):
     return FusedLinearCrossEntropy.apply(H, W, b, labels, mask, ignore_index, weight, reduction,
-                                         denom)
+                                         denom, round_logits)
 
 
 class LinearCrossEntropyLoss(torch.nn.Module):
     """Loss module over final hidden states and the projection weight, with
     the reductions of a chunked linear cross-entropy loss ("mean", "sum",
     "none"), an optional global label count for "sum" and optional per-token
-    loss weights.  Hidden states may have any leading token dimensions."""
+    loss weights.  Hidden states may have any leading token dimensions.
+    round_logits rounds the logits to the input dtype before the loss (a
+    projection that outputs the model dtype)."""
 
-    def __init__(self, ignore_index: int = -100, reduction: str = "mean"):
+    def __init__(self, ignore_index: int = -100, reduction: str = "mean",
+                 round_logits: bool = False):
         super().__init__()
         if reduction not in REDUCTIONS:
             raise ValueError(f"reduction must be one of {tuple(REDUCTIONS)}")
         self.ignore_index = ignore_index
         self.reduction = reduction
+        self.round_logits = round_logits
 
     def forward(self, hidden_states, labels, lm_weight, bias=None, num_label_tokens=None,
                 loss_weights=None, mask=None):
         lead = hidden_states.shape[:-1]
         out = fused_linear_cross_entropy(hidden_states, lm_weight, labels, b=bias, mask=mask,
                                          ignore_index=self.ignore_index, weight=loss_weights,
-                                         reduction=self.reduction, denom=num_label_tokens)
+                                         reduction=self.reduction, denom=num_label_tokens,
+                                         round_logits=self.round_logits)
         return out.reshape(lead) if self.reduction == "none" else out

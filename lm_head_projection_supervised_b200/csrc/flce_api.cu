@@ -355,16 +355,19 @@ flce_status flce_forward(const void* H, const void* W, const void* b, const int6
                          int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
                          size_t ws_bytes, flce_stream stream) {
   return flce_forward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, nullptr,
-                         FLCE_REDUCE_MEAN, 0.f, loss, nullptr, m, logs, ws, ws_bytes, stream);
+                         FLCE_REDUCE_MEAN, 0.f, 0u, loss, nullptr, m, logs, ws, ws_bytes,
+                         stream);
 }
 
 flce_status flce_forward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
                             const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
                             int64_t V, int dtype, const float* weight, int reduction, float denom,
-                            float* loss, float* loss_rows, float* m, float* logs, void* ws,
+                            unsigned flags, float* loss, float* loss_rows, float* m, float* logs,
+                            void* ws,
                             size_t ws_bytes, flce_stream stream) {
-  if (reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
-      reduction != FLCE_REDUCE_NONE)
+  if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
+       reduction != FLCE_REDUCE_NONE) ||
+      (flags & ~FLCE_FLAG_ROUND_LOGITS) != 0)
     return FLCE_ERR_ARG;
   const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
@@ -408,6 +411,7 @@ flce_status flce_forward_ex(const void* H, const void* W, const void* b, const i
   a.part = p.part;
   a.part_ld = static_cast<int>(L.nvt);
   a.tgt = p.tgt;
+  a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
   a.err = p.err;
   FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
@@ -435,19 +439,21 @@ flce_status flce_backward(const void* H, const void* W, const void* b, const int
                           const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
                           size_t ws_bytes, flce_stream stream) {
   return flce_backward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, m, logs, nullptr,
-                          FLCE_REDUCE_MEAN, 0.f, lambda, lambda_dev, nullptr, dH, dW, db, ws,
+                          FLCE_REDUCE_MEAN, 0.f, 0u, lambda, lambda_dev, nullptr, dH, dW, db, ws,
                           ws_bytes, stream);
 }
 
 flce_status flce_backward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
                              const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
                              int64_t V, int dtype, const float* m, const float* logs,
-                             const float* weight, int reduction, float denom, float lambda,
+                             const float* weight, int reduction, float denom, unsigned flags,
+                             float lambda,
                              const float* lambda_dev, const float* grad_rows, float* dH,
                              float* dW, float* db, void* ws, size_t ws_bytes,
                              flce_stream stream) {
-  if (reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
-      reduction != FLCE_REDUCE_NONE)
+  if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
+       reduction != FLCE_REDUCE_NONE) ||
+      (flags & ~FLCE_FLAG_ROUND_LOGITS) != 0)
     return FLCE_ERR_ARG;
   const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
@@ -537,6 +543,7 @@ flce_status flce_backward_ex(const void* H, const void* W, const void* b, const 
     a.sigma = sigma;
     a.row_scale = p.rs;
     a.scal = p.scal;
+    a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
     a.inv_sigma = 1.f / sigma;
     a.err = p.err;
     const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +

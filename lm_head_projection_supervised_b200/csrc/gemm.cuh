@@ -99,6 +99,7 @@ struct GemmArgs {
   const int* y_c;          // compact labels
   const int* idx;          // compact row -> original row
   const uint16_t* bias;    // 16-bit bias [V] or null
+  int round_logits;        // round each logit to the 16-bit input type first
   float2* part;            // fwd: (m, s) partials [rows][part_ld]
   int part_ld;
   float* tgt;              // fwd: target logits [rows]
@@ -286,6 +287,17 @@ __device__ __forceinline__ void load_bias32(const uint16_t* b, int col0, int V, 
   }
 }
 
+// Logits rounded to the 16-bit input type (round to nearest even).
+__device__ __forceinline__ void round_to_input_type(const GemmArgs& g, float (&x)[32]) {
+  if (g.is_bf16) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = __bfloat162float(__float2bfloat16_rn(x[j]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = __half2float(__float2half_rn(x[j]));
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Epilogue: forward statistics of one 32-column chunk.
 // ---------------------------------------------------------------------------
@@ -307,6 +319,7 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
 #pragma unroll
     for (int j = 0; j < 32; ++j) x[j] += bv[j];
   }
+  if (g.round_logits) round_to_input_type(g, x);
   if (cb + 32 > vlim) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -352,6 +365,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
 #pragma unroll
     for (int j = 0; j < 32; ++j) x[j] += bv[j];
   }
+  if (g.round_logits) round_to_input_type(g, x);
   float gv[32];
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
 #pragma unroll

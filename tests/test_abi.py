@@ -136,29 +136,32 @@ def test_product_path_does_not_import_the_oracle():
 
 def fwd_ex(L, **kw):
     a = dict(H=FAKE, W=FAKE, b=None, labels=FAKE, mask=None, ig=-100, N=64, D=32, V=1000, dt=0,
-             w=None, red=0, den=0.0, loss=FAKE, rows=None, m=FAKE, logs=FAKE, ws=FAKE,
+             w=None, red=0, den=0.0, fl=0, loss=FAKE, rows=None, m=FAKE, logs=FAKE, ws=FAKE,
              wsb=1 << 40, s=None)
     a.update(kw)
     return L.flce_forward_ex(P(a["H"]), P(a["W"]), P(a["b"]), P(a["labels"]), P(a["mask"]),
                              a["ig"], a["N"], a["D"], a["V"], a["dt"], P(a["w"]), a["red"],
-                             a["den"], P(a["loss"]), P(a["rows"]), P(a["m"]), P(a["logs"]),
+                             a["den"], a["fl"], P(a["loss"]), P(a["rows"]), P(a["m"]),
+                             P(a["logs"]),
                              P(a["ws"]), a["wsb"], P(a["s"]))
 
 
 def bwd_ex(L, **kw):
     a = dict(H=FAKE, W=FAKE, b=None, labels=FAKE, mask=None, ig=-100, N=64, D=32, V=1000, dt=0,
-             m=FAKE, logs=FAKE, w=None, red=0, den=0.0, lam=1.0, lamd=None, g=None, dH=FAKE,
+             m=FAKE, logs=FAKE, w=None, red=0, den=0.0, fl=0, lam=1.0, lamd=None, g=None, dH=FAKE,
              dW=FAKE, db=None, ws=FAKE, wsb=1 << 40, s=None)
     a.update(kw)
     return L.flce_backward_ex(P(a["H"]), P(a["W"]), P(a["b"]), P(a["labels"]), P(a["mask"]),
                               a["ig"], a["N"], a["D"], a["V"], a["dt"], P(a["m"]), P(a["logs"]),
-                              P(a["w"]), a["red"], a["den"], a["lam"], P(a["lamd"]), P(a["g"]),
+                              P(a["w"]), a["red"], a["den"], a["fl"], a["lam"], P(a["lamd"]),
+                              P(a["g"]),
                               P(a["dH"]), P(a["dW"]), P(a["db"]), P(a["ws"]), a["wsb"], P(a["s"]))
 
 
 @pytest.mark.parametrize("kw,want", [
     (dict(red=3), "FLCE_ERR_ARG"),
     (dict(red=-1), "FLCE_ERR_ARG"),
+    (dict(fl=2), "FLCE_ERR_ARG"),                    # unknown option bit
     (dict(red=2, rows=None), "FLCE_ERR_NULL"),       # 'none' needs the per-row output
     (dict(red=1, loss=None), "FLCE_ERR_NULL"),       # 'sum' needs the scalar
     (dict(red=0, w=FAKE + 2), "FLCE_ERR_ALIGN"),
@@ -170,6 +173,7 @@ def test_forward_ex_argument_errors(L, kw, want):
 
 @pytest.mark.parametrize("kw,want", [
     (dict(red=7), "FLCE_ERR_ARG"),
+    (dict(fl=0x80), "FLCE_ERR_ARG"),
     (dict(red=2, g=None), "FLCE_ERR_NULL"),          # 'none' needs per-row upstream gradients
     (dict(red=1, g=FAKE + 1), "FLCE_ERR_ALIGN"),
     (dict(red=2, g=FAKE, wsb=4096), "FLCE_ERR_WORKSPACE"),

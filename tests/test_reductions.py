@@ -109,3 +109,39 @@ def test_loss_module_none_with_leading_dims():
     dW = Wp.grad.float().cpu().numpy()
     assert np.max(np.abs(dH - ref["dH"])) <= 1e-2 * np.max(np.abs(ref["dH"]))
     assert np.max(np.abs(dW - ref["dW"])) <= 1e-2 * np.max(np.abs(ref["dW"]))
+
+
+def ulp16(x, dtype):
+    """Spacing of the 16-bit type at |x| (7 fraction bits for bf16, 10 for fp16)."""
+    frac = 7 if dtype == "bf16" else 10
+    e = np.floor(np.log2(np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -14)))
+    return 2.0 ** (e - frac)
+
+
+@pytest.mark.parametrize("kw", [dict(seed=41, N=300, D=64, V=9000),
+                                dict(seed=42, N=200, D=48, V=3000, dtype="fp16")],
+                         ids=["bf16", "fp16_bias"])
+def test_rounded_logits_parity(kw):
+    """Logits rounded to the input dtype (NeMo logits_dtype).  The GPU rounds
+    its fp32 logit, the oracle its exact one; a logit within fp32 error of a
+    16-bit rounding boundary can round the other way, so m and log s may
+    differ by one 16-bit spacing of the row's largest logit."""
+    inp = wl.random_case(**kw)
+    H, W, b, y, mk = to_device(inp)
+    loss, m, logs = binding.forward(H, W, b, y, mk, round_logits=True)
+    dH, dW, db = binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, round_logits=True)
+    ref = orc.forward_backward(inp.H64(), inp.W64(), inp.b64(), inp.labels, inp.mask,
+                               lam=inp.lam, logits_dtype=inp.dtype)
+    plain = orc.forward(inp.H64(), inp.W64(), inp.b64(), inp.labels, inp.mask)
+    idx = ref["idx"]
+    check_loss(loss.item(), ref["loss"])
+    # the variant is visible: the rounded-logit loss is not the exact one
+    assert abs(ref["loss"] - plain["loss"]) > 10 * abs(loss.item() - ref["loss"])
+    ulp = ulp16(ref["m"][idx], inp.dtype)
+    check_stats(m.cpu().numpy(), ref["m"], idx, floor=ulp)
+    check_stats(logs.cpu().numpy(), ref["logs"], idx,
+                floor=np.maximum(ulp, logs_floor(ref["m"][idx], inp.D)))
+    check_grad("dH", dH.cpu().numpy(), ref["dH"])
+    check_grad("dW", dW.cpu().numpy(), ref["dW"])
+    if inp.b is not None:
+        check_grad("db", db.cpu().numpy(), ref["db"])
