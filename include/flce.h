@@ -71,7 +71,9 @@ typedef enum {
   FLCE_ERR_TIMEOUT = 8,     /* device: a pipeline wait ran past its time limit   */
   FLCE_ERR_NONFINITE = 9,   /* device: a non-finite per-row statistic            */
   FLCE_ERR_DEVICE = 10,     /* current device is not sm_100 / cannot run kernels */
-  FLCE_ERR_ARG = 11         /* an argument value is invalid (e.g. the reduction) */
+  FLCE_ERR_ARG = 11,        /* an argument value is invalid (e.g. the reduction) */
+  FLCE_ERR_SHARD = 12       /* device: a supervised label is held by no
+                               vocabulary slice, or by several (shard combine) */
 } flce_status;
 
 typedef enum { FLCE_BF16 = 0, FLCE_FP16 = 1 } flce_dtype;
@@ -221,6 +223,87 @@ FLCE_API flce_status flce_backward_ex(const void* H, const void* W, const void* 
                                       unsigned flags, float lambda, const float* lambda_dev,
                                       const float* grad_rows, float* dH, float* dW, float* db,
                                       void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * Vocabulary-sharded (tensor-parallel over V) form.
+ *
+ * The vocabulary [0, V_total) is cut into disjoint slices; the caller that
+ * holds the slice [v0, v0 + V_slice) passes W_slice = rows v0 .. v0+V_slice-1
+ * of W ([V_slice x D]) and the same slice of b.  Labels stay global ids in
+ * [0, V_total).  One step is:
+ *
+ *   1. flce_shard_forward on every slice   -> stats_r [N] (float4 per row)
+ *   2. exchange: every caller obtains all slices' stats, stacked [P x N]
+ *      (an all-gather of P x N x 16 bytes)
+ *   3. flce_shard_combine                  -> loss, m, logs (full vocabulary)
+ *   4. flce_shard_backward on every slice  -> dW_slice, db_slice, dH_r
+ *   5. exchange: dH = sum_r dH_r (an all-reduce of N x D floats)
+ *
+ * The merge in step 3 is the two-state online-softmax merge ("数学基础"
+ * maths-basics page, worked example 9.4, and "分块交叉熵" §02), exact in the
+ * reals for any partition of the vocabulary; the need for a cross-device
+ * aggregation when the vocabulary is tensor-parallel is the maths-basics
+ * page's §5.9 remark.  With the merged statistics each slice forms its own
+ * columns of G (§04), so step 4 needs nothing from the other slices.  The
+ * library does no communication: steps 2 and 5 are the caller's (e.g. NCCL).
+ */
+
+/*
+ * Per-row partial statistics of one slice.
+ *   stats : device float4 [N] (16-byte aligned), per row
+ *           (m_r, log s_r, t_r, o_r) = the slice's max logit, the log of its
+ *           sum of exp(Z - m_r), the target logit when the slice holds the
+ *           label (else 0) and the ownership flag 1[v0 <= y < v0 + V_slice].
+ *           Unsupervised rows get (-inf, -inf, 0, 0).
+ *   0 <= v0, v0 + V_slice <= V_total <= the V limit; labels are checked
+ *   against V_total (FLCE_ERR_LABEL).  Workspace: flce_workspace_bytes(N, D,
+ *   V_slice, dtype).  flags: FLCE_FLAG_* as in flce_forward_ex().
+ */
+FLCE_API flce_status flce_shard_forward(const void* H, const void* W_slice, const void* b_slice,
+                                        const int64_t* labels, const uint8_t* mask,
+                                        int64_t ignore_index, int64_t N, int64_t D,
+                                        int64_t V_slice, int64_t v0, int64_t V_total, int dtype,
+                                        unsigned flags, float* stats, void* ws, size_t ws_bytes,
+                                        flce_stream stream);
+
+/* Bytes of device workspace flce_shard_combine() needs for N rows. */
+FLCE_API size_t flce_shard_combine_workspace_bytes(int64_t N);
+
+/*
+ * Merge of P slices' statistics into the full-vocabulary result.
+ *   stats_all : device float4 [P x N] (16-byte aligned), slice r's stats at
+ *               rows r*N .. r*N+N-1, slices in any order
+ *   labels, mask, ignore_index : as given to flce_shard_forward (same on
+ *               every slice); weight, reduction, denom, loss, loss_rows as in
+ *               flce_forward_ex(); m, logs : device float [N], the merged
+ *               statistics that flce_shard_backward() consumes.
+ * A supervised row held by no slice or by several records FLCE_ERR_SHARD
+ * (loss NaN).  Workspace: flce_shard_combine_workspace_bytes(N).
+ */
+FLCE_API flce_status flce_shard_combine(const float* stats_all, int P, const int64_t* labels,
+                                        const uint8_t* mask, int64_t ignore_index, int64_t N,
+                                        const float* weight, int reduction, float denom,
+                                        float* loss, float* loss_rows, float* m, float* logs,
+                                        void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * This slice's share of the backward: with the merged m and logs from
+ * flce_shard_combine(), dW_slice [V_slice x D] and db_slice [V_slice] (iff
+ * b_slice) are the slice's rows of dW and db, and dH [N x D] is this slice's
+ * term G_r W_slice of dH = sum_r G_r W_r (float32, fully overwritten; the
+ * caller sums the slices' dH).  Other arguments as in flce_backward_ex() and
+ * flce_shard_forward().  Workspace: flce_workspace_bytes(N, D, V_slice, dtype).
+ */
+FLCE_API flce_status flce_shard_backward(const void* H, const void* W_slice,
+                                         const void* b_slice, const int64_t* labels,
+                                         const uint8_t* mask, int64_t ignore_index, int64_t N,
+                                         int64_t D, int64_t V_slice, int64_t v0, int64_t V_total,
+                                         int dtype, const float* m, const float* logs,
+                                         const float* weight, int reduction, float denom,
+                                         unsigned flags, float lambda, const float* lambda_dev,
+                                         const float* grad_rows, float* dH, float* dW_slice,
+                                         float* db_slice, void* ws, size_t ws_bytes,
+                                         flce_stream stream);
 
 /* Synchronises `stream`, then reads and returns the device error word of the
  * workspace (FLCE_OK when no device error was recorded by the last call). */

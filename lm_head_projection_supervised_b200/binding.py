@@ -20,7 +20,7 @@ FLCE_BF16, FLCE_FP16 = 0, 1
 STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DTYPE",
           4: "FLCE_ERR_ALIGN", 5: "FLCE_ERR_WORKSPACE", 6: "FLCE_ERR_CUDA", 7: "FLCE_ERR_LABEL",
           8: "FLCE_ERR_TIMEOUT", 9: "FLCE_ERR_NONFINITE", 10: "FLCE_ERR_DEVICE",
-          11: "FLCE_ERR_ARG"}
+          11: "FLCE_ERR_ARG", 12: "FLCE_ERR_SHARD"}
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 FLAG_ROUND_LOGITS = 1
 STATUS_CODE = {v: k for k, v in STATUS.items()}
@@ -64,6 +64,17 @@ def lib() -> ctypes.CDLL:
     L.flce_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, i32,
                                    f32, u32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.flce_backward_ex.restype = i32
+    L.flce_shard_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, u32,
+                                     vp, vp, sz, vp]
+    L.flce_shard_forward.restype = i32
+    L.flce_shard_combine_workspace_bytes.argtypes = [i64]
+    L.flce_shard_combine_workspace_bytes.restype = sz
+    L.flce_shard_combine.argtypes = [vp, i32, vp, vp, i64, i64, vp, i32, f32, vp, vp, vp, vp, vp,
+                                     sz, vp]
+    L.flce_shard_combine.restype = i32
+    L.flce_shard_backward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, vp,
+                                      vp, vp, i32, f32, u32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.flce_shard_backward.restype = i32
     L.flce_device_status.argtypes = [vp, vp]
     L.flce_device_status.restype = i32
     L.flce_diag_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, f32, vp, sz, vp]
@@ -145,16 +156,20 @@ def _prep(H, W, b, labels, mask):
     if y.numel() != H2.shape[0]:
         raise ValueError("labels must have one entry per row of H")
     y = y.contiguous()
-    mk = None
-    if mask is not None:
-        mk = mask.reshape(-1)
-        if mk.dtype == torch.bool:
-            mk = mk.view(torch.uint8)
-        elif mk.dtype != torch.uint8:
-            mk = (mk != 0).view(torch.uint8)
-        mk = mk.contiguous()
     b2 = None if b is None else b.contiguous()
-    return H2, W2, b2, y, mk
+    return H2, W2, b2, y, _mask_u8(mask)
+
+
+def _mask_u8(mask):
+    """uint8 contiguous [N] view of a mask (nonzero = takes part), or None."""
+    if mask is None:
+        return None
+    mk = mask.reshape(-1)
+    if mk.dtype == torch.bool:
+        mk = mk.view(torch.uint8)
+    elif mk.dtype != torch.uint8:
+        mk = (mk != 0).view(torch.uint8)
+    return mk.contiguous()
 
 
 def _vec(t, N, device):
@@ -227,6 +242,104 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
                                 _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
                                 _stream(stream))
     _check(st, "flce_backward_ex")
+    return dH, dW, db
+
+
+class CombineWorkspace:
+    """Device scratch of flce_shard_combine_workspace_bytes(N) bytes."""
+
+    def __init__(self, N: int, device=None):
+        n = int(lib().flce_shard_combine_workspace_bytes(N))
+        if n == 0:
+            raise FlceError(STATUS_CODE["FLCE_ERR_SHAPE"], "shard_combine_workspace_bytes")
+        self.nbytes = n
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def shard_forward(H, W_slice, b_slice, labels, mask=None, ignore_index: int = -100, v0: int = 0,
+                  V_total: Optional[int] = None, ws: Optional[Workspace] = None, stream=None,
+                  round_logits: bool = False):
+    """Per-row partial statistics [N, 4] float32 (m_r, log s_r, t_r, o_r) of
+    the vocabulary slice [v0, v0 + V_slice) -- flce_shard_forward()."""
+    H2, W2, b2, y, mk = _prep(H, W_slice, b_slice, labels, mask)
+    N, D = H2.shape
+    Vs = W2.shape[0]
+    V_total = v0 + Vs if V_total is None else int(V_total)
+    if ws is None:
+        ws = Workspace(N, D, Vs, H2.dtype, H2.device)
+    stats = torch.empty((N, 4), dtype=torch.float32, device=H2.device)
+    st = lib().flce_shard_forward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index,
+                                  N, D, Vs, int(v0), V_total, dtype_code(H2.dtype),
+                                  FLAG_ROUND_LOGITS if round_logits else 0, _ptr(stats),
+                                  ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "flce_shard_forward")
+    return stats
+
+
+def shard_combine(stats_all, labels, mask=None, ignore_index: int = -100, weight=None,
+                  reduction: str = "mean", denom: Optional[float] = None,
+                  ws: Optional[CombineWorkspace] = None, stream=None):
+    """(loss, m [N], logs [N]) of the full vocabulary from the slices' stats
+    stacked as [P, N, 4] -- flce_shard_combine().  loss as in forward()."""
+    if not (stats_all.is_cuda and labels.is_cuda):
+        raise ValueError("stats and labels must be CUDA tensors")
+    if stats_all.dim() != 3 or stats_all.shape[2] != 4 or stats_all.dtype != torch.float32:
+        raise ValueError("stats_all must be float32 [P, N, 4]")
+    P, N = int(stats_all.shape[0]), int(stats_all.shape[1])
+    st_all = stats_all.contiguous()
+    y = labels.reshape(-1).to(torch.int64).contiguous()
+    if y.numel() != N:
+        raise ValueError("labels must have one entry per row")
+    mk = _mask_u8(mask)
+    dev = st_all.device
+    if ws is None:
+        ws = CombineWorkspace(N, dev)
+    wt = _vec(weight, N, dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    rows = torch.empty(N, dtype=torch.float32, device=dev) if reduction == "none" else None
+    m = torch.empty(N, dtype=torch.float32, device=dev)
+    logs = torch.empty(N, dtype=torch.float32, device=dev)
+    st = lib().flce_shard_combine(_ptr(st_all), P, _ptr(y), _ptr(mk), ignore_index, N, _ptr(wt),
+                                  REDUCTIONS[reduction], float(denom or 0.0), _ptr(loss),
+                                  _ptr(rows), _ptr(m), _ptr(logs), ws.ptr(), ws.nbytes,
+                                  _stream(stream))
+    _check(st, "flce_shard_combine")
+    return (rows if reduction == "none" else loss), m, logs
+
+
+def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index: int, m, logs, v0: int = 0,
+                   V_total: Optional[int] = None, lam: float = 1.0, lam_dev=None,
+                   ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
+                   reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
+                   round_logits: bool = False):
+    """(dH_r [N, D], dW_slice [V_slice, D], db_slice [V_slice] or None),
+    float32 -- flce_shard_backward().  dH_r is this slice's term of dH."""
+    H2, W2, b2, y, mk = _prep(H, W_slice, b_slice, labels, mask)
+    N, D = H2.shape
+    Vs = W2.shape[0]
+    V_total = v0 + Vs if V_total is None else int(V_total)
+    if ws is None:
+        ws = Workspace(N, D, Vs, H2.dtype, H2.device)
+    if out is None:
+        dH = torch.empty((N, D), dtype=torch.float32, device=H2.device)
+        dW = torch.empty((Vs, D), dtype=torch.float32, device=H2.device)
+        db = None if b2 is None else torch.empty(Vs, dtype=torch.float32, device=H2.device)
+    else:
+        dH, dW, db = out
+    if lam_dev is not None:
+        lam_dev = lam_dev.reshape(()).to(torch.float32).contiguous()
+    wt = _vec(weight, N, H2.device)
+    gr = _vec(grad_rows, N, H2.device)
+    st = lib().flce_shard_backward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index,
+                                   N, D, Vs, int(v0), V_total, dtype_code(H2.dtype), _ptr(m),
+                                   _ptr(logs), _ptr(wt), REDUCTIONS[reduction],
+                                   float(denom or 0.0), FLAG_ROUND_LOGITS if round_logits else 0,
+                                   float(lam), _ptr(lam_dev), _ptr(gr), _ptr(dH), _ptr(dW),
+                                   _ptr(db), ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "flce_shard_backward")
     return dH, dW, db
 
 

@@ -23,12 +23,14 @@ __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8
 // contiguous slice, a block-wide exclusive scan of the slice counts gives
 // every thread its output offset.  Labels outside [0, V) on supervised rows
 // set the label error bit and are clamped to 0 so later indexing stays in
-// range.  Unsupervised rows get m = log s = -inf when m_out is given.
+// range.  y_c holds y - v0: the label's column in a vocabulary slice that
+// starts at v0 (v0 = 0 unsharded), outside [0, V_slice) when another slice
+// holds it.  Unsupervised rows get m = log s = -inf when m_out is given.
 // pos (optional) is the inverse map: pos[i] = compact row of i, or -1.
 // lossvec (optional) gets 0 on unsupervised rows (per-row loss output).
 __global__ void __launch_bounds__(COMPACT_THREADS)
     compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
-                   int64_t ignore, int64_t N, int64_t V, int* __restrict__ idx,
+                   int64_t ignore, int64_t N, int64_t V, int64_t v0, int* __restrict__ idx,
                    int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
                    float* __restrict__ m_out, float* __restrict__ logs_out,
                    int* __restrict__ pos, float* __restrict__ lossvec) {
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
         y = 0;
       }
       idx[off] = static_cast<int>(i);
-      if (y_c != nullptr) y_c[off] = static_cast<int>(y);
+      if (y_c != nullptr) y_c[off] = static_cast<int>(y - v0);
       if (pos != nullptr) pos[i] = off;
       ++off;
     } else {
@@ -160,9 +162,88 @@ __global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld,
   }
 }
 
+// Vocabulary slice [v0, v0 + V_slice): per ORIGINAL row i the partial
+// statistics (m_r, log s_r, t_r, o_r) of the slice's columns: the merged
+// tile partials, the target logit when the slice holds the label (y_c in
+// [0, V_slice)) else 0, and the ownership flag.  Unsupervised rows (pos < 0)
+// get the recurrence's initial state (-inf, -inf, 0, 0).  One warp per row.
+__global__ void shard_stats_kernel(const float2* __restrict__ part, int part_ld, int nvt,
+                                   const float* __restrict__ tgt, const int* __restrict__ y_c,
+                                   const int* __restrict__ pos, int64_t N, int V_slice,
+                                   float4* __restrict__ stats, uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       i < N; i += warps) {
+    const int k = pos[i];
+    if (k < 0) {
+      if (lane == 0) stats[i] = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+      continue;
+    }
+    const float2* pr = part + static_cast<size_t>(k) * part_ld;
+    float m = -INFINITY, s = 0.f;
+    for (int v = lane; v < nvt; v += 32) {
+      const float2 ps = pr[v];
+      merge_state(m, s, ps.x, ps.y);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, m, o);
+      const float os = __shfl_xor_sync(0xffffffffu, s, o);
+      merge_state(m, s, om, os);
+    }
+    if (lane == 0) {
+      const float logs = logf(s);
+      const bool own = static_cast<unsigned>(y_c[k]) < static_cast<unsigned>(V_slice);
+      stats[i] = make_float4(m, logs, own ? tgt[k] : 0.f, own ? 1.f : 0.f);
+      if (!isfinite(m) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
+    }
+  }
+}
+
+// Merge of the slices' partial statistics stats[r * N + i], r < P (the
+// two-state online-softmax merge, maths-basics page worked example 9.4, in
+// log form): M = max_r m_r, log S = log sum_r exp((m_r - M) + log s_r),
+// target = the owning slice's t_r, l = (M - target) + log S ("分块交叉熵"
+// §02).  Per supervised row k (original row o = idx[k]): m_out[o], logs_out[o],
+// loss_rows[k] = w_o l and lossvec[o] = w_o l when given.  A row owned by no
+// slice or by several sets the shard error bit.  One thread per row.
+__global__ void shard_combine_kernel(const float4* __restrict__ stats, int P, int64_t N,
+                                     const int* __restrict__ C_dev, const int* __restrict__ idx,
+                                     float* __restrict__ m_out, float* __restrict__ logs_out,
+                                     float* __restrict__ loss_rows,
+                                     const float* __restrict__ weight,
+                                     float* __restrict__ lossvec, uint32_t* err) {
+  const int C = *C_dev;
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < C; k += blockDim.x * gridDim.x) {
+    const int o = idx[k];
+    float M = -INFINITY;
+    for (int r = 0; r < P; ++r) M = fmaxf(M, stats[static_cast<int64_t>(r) * N + o].x);
+    float S = 0.f, t = 0.f;
+    int owners = 0;
+    for (int r = 0; r < P; ++r) {
+      const float4 q = stats[static_cast<int64_t>(r) * N + o];
+      if (q.x != -INFINITY) S += expf((q.x - M) + q.y);
+      if (q.w != 0.f) {
+        t = q.z;
+        ++owners;
+      }
+    }
+    const float logs = logf(S);
+    const float li = (M - t) + logs;
+    m_out[o] = M;
+    logs_out[o] = logs;
+    const float wl = (weight != nullptr) ? weight[o] * li : li;
+    loss_rows[k] = wl;
+    if (lossvec != nullptr) lossvec[o] = wl;
+    if (owners != 1) atomicOr(err, kErrBitShard);
+    if (!isfinite(li) || !isfinite(M) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
+  }
+}
+
 // L = sum_i loss_rows[i] / den in a fixed order (per-thread strided sums in
 // double, then a fixed tree), den = C for the mean and `denom` (or 1) for the
-// sum; 0 when C = 0; NaN when the label or timeout bit is set.
+// sum; 0 when C = 0; NaN when the label, timeout or shard bit is set.
 __global__ void __launch_bounds__(1024)
     loss_reduce_kernel(const float* __restrict__ loss_rows, const int* __restrict__ C_dev,
                        int is_mean, float denom, const uint32_t* err, float* __restrict__ loss) {
@@ -179,7 +260,7 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) {
     const double den = is_mean ? static_cast<double>(C) : (denom > 0.f ? denom : 1.0);
     float L = (C > 0) ? static_cast<float>(red[0] / den) : 0.f;
-    if (*err & (kErrBitLabel | kErrBitTimeout)) L = __int_as_float(0x7fc00000);
+    if (*err & (kErrBitLabel | kErrBitTimeout | kErrBitShard)) L = __int_as_float(0x7fc00000);
     *loss = L;
   }
 }

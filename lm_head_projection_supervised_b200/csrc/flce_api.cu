@@ -28,6 +28,7 @@ namespace {
 constexpr int64_t kMaxN = int64_t(1) << 24;
 constexpr int64_t kMaxD = int64_t(1) << 16;
 constexpr int64_t kMaxV = int64_t(1) << 24;
+constexpr int kMaxShards = 4096;  // vocabulary slices merged by one combine
 #ifndef FLCE_PANEL_COLS
 #define FLCE_PANEL_COLS 8192
 #endif
@@ -68,13 +69,28 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.part = take(static_cast<size_t>(L.Np) * L.nvt * 8);
   L.tgt = take(static_cast<size_t>(L.Np) * 4);
   L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
-  L.fwd_total = off;
   L.pos = take(static_cast<size_t>(L.Np) * 4);
+  L.fwd_total = off;
   L.rs = take(static_cast<size_t>(L.Np) * 4);
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
   L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.vc * 2);
   L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.vc * 2);
   L.total = off;
+  return L;
+}
+
+// Workspace of flce_shard_combine: error word, C, idx [N], per-row losses [N].
+struct CombineLayout {
+  size_t C, idx, loss_rows, total;
+};
+
+CombineLayout combine_layout(int64_t N) {
+  CombineLayout L{};
+  const size_t n = static_cast<size_t>(roundup64(N > 0 ? N : 1, 64)) * 4;
+  L.C = 256;
+  L.idx = 512;
+  L.loss_rows = L.idx + n;
+  L.total = L.loss_rows + n;
   return L;
 }
 
@@ -286,12 +302,12 @@ WsPtrs carve(void* ws, const Layout& L) {
 
 // control block reset + compaction + gather of the supervised rows
 flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
-                     int64_t N, int64_t D, int64_t V, const Layout& L, const WsPtrs& p,
+                     int64_t N, int64_t D, int64_t V, int64_t v0, const Layout& L, const WsPtrs& p,
                      float* m_out, float* logs_out, int* pos, float* lossvec,
                      cudaStream_t s) {
   FLCE_CK(cudaMemsetAsync(p.err, 0, L.ctrl_bytes, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
-    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, p.idx, p.yc, p.C,
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, v0, p.idx, p.yc, p.C,
                                                  p.err, m_out, logs_out, pos, lossvec);
   }));
   const int64_t vec = D / 8;
@@ -302,96 +318,48 @@ flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, 
   return FLCE_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype) {
-  if (!shape_ok(N, D, V) || (dtype != FLCE_BF16 && dtype != FLCE_FP16)) return 0;
-  return make_layout(N, D, V).total;
-}
-
-const char* flce_status_string(int status) {
-  switch (status) {
-    case FLCE_OK: return "FLCE_OK";
-    case FLCE_ERR_NULL: return "FLCE_ERR_NULL: a required pointer is NULL";
-    case FLCE_ERR_SHAPE: return "FLCE_ERR_SHAPE: N, D or V out of range";
-    case FLCE_ERR_DTYPE: return "FLCE_ERR_DTYPE: dtype must be FLCE_BF16 or FLCE_FP16";
-    case FLCE_ERR_ALIGN: return "FLCE_ERR_ALIGN: misaligned pointer or D not a multiple of 8";
-    case FLCE_ERR_WORKSPACE: return "FLCE_ERR_WORKSPACE: workspace too small";
-    case FLCE_ERR_CUDA: return "FLCE_ERR_CUDA: a CUDA runtime call failed";
-    case FLCE_ERR_LABEL: return "FLCE_ERR_LABEL: supervised label outside [0, V)";
-    case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT: a device pipeline wait ran out";
-    case FLCE_ERR_NONFINITE: return "FLCE_ERR_NONFINITE: non-finite per-row statistic";
-    case FLCE_ERR_DEVICE: return "FLCE_ERR_DEVICE: current device is not sm_100";
-    case FLCE_ERR_ARG: return "FLCE_ERR_ARG: invalid argument value";
-    default: return "FLCE_ERR_UNKNOWN";
-  }
-}
-
-flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
-                         int64_t N, int64_t V, int32_t* idx, int32_t* C_out, void* ws,
-                         size_t ws_bytes, flce_stream stream) {
-  if ((N > 0 && (labels == nullptr || idx == nullptr)) || C_out == nullptr || ws == nullptr)
-    return FLCE_ERR_NULL;
-  if (N < 0 || N > kMaxN || V < 1 || V > kMaxV) return FLCE_ERR_SHAPE;
-  if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
-  if (ws_bytes < 256) return FLCE_ERR_WORKSPACE;
-  DevInfo di;
-  const flce_status st = device_setup(&di);
-  if (st != FLCE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t* err = static_cast<uint32_t*>(ws);
-  FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
-  FLCE_CK(timed_launch(kProfAux, s, [&] {
-    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, idx, nullptr,
-                                                 C_out, err, nullptr, nullptr, nullptr, nullptr);
-  }));
-  return FLCE_OK;
-}
-
-flce_status flce_forward(const void* H, const void* W, const void* b, const int64_t* labels,
+// Forward of the full vocabulary (shard false) or of the slice [v0, v0 + V)
+// of a vocabulary of V_total ids (shard true: per-row partial statistics in
+// `stats` instead of the loss; see flce_shard_forward).
+flce_status forward_impl(const void* H, const void* W, const void* b, const int64_t* labels,
                          const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
-                         int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
-                         size_t ws_bytes, flce_stream stream) {
-  return flce_forward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, nullptr,
-                         FLCE_REDUCE_MEAN, 0.f, 0u, loss, nullptr, m, logs, ws, ws_bytes,
-                         stream);
-}
-
-flce_status flce_forward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
-                            const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
-                            int64_t V, int dtype, const float* weight, int reduction, float denom,
-                            unsigned flags, float* loss, float* loss_rows, float* m, float* logs,
-                            void* ws,
-                            size_t ws_bytes, flce_stream stream) {
+                         int64_t V, int64_t v0, int64_t V_total, int dtype, const float* weight,
+                         int reduction, float denom, unsigned flags, float* loss,
+                         float* loss_rows, float* m, float* logs, bool shard, float4* stats,
+                         void* ws, size_t ws_bytes, cudaStream_t s) {
   if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
        reduction != FLCE_REDUCE_NONE) ||
       (flags & ~FLCE_FLAG_ROUND_LOGITS) != 0)
     return FLCE_ERR_ARG;
-  const bool none = reduction == FLCE_REDUCE_NONE;
-  if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
-                 (none && loss_rows == nullptr))) ||
-      W == nullptr || (!none && loss == nullptr) || ws == nullptr)
+  const bool none = !shard && reduction == FLCE_REDUCE_NONE;
+  if (shard) {
+    if ((N > 0 && (H == nullptr || labels == nullptr || stats == nullptr)) || W == nullptr ||
+        ws == nullptr)
+      return FLCE_ERR_NULL;
+  } else if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
+                        (none && loss_rows == nullptr))) ||
+             W == nullptr || (!none && loss == nullptr) || ws == nullptr) {
     return FLCE_ERR_NULL;
+  }
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
-  if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
+  if (!shape_ok(N, D, V) || v0 < 0 || V_total > kMaxV || v0 + V > V_total)
+    return FLCE_ERR_SHAPE;
   if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
       !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) || !aligned(loss, 4) ||
-      !aligned(weight, 4) || !aligned(loss_rows, 4))
+      !aligned(weight, 4) || !aligned(loss_rows, 4) || !aligned(stats, 16))
     return FLCE_ERR_ALIGN;
   const Layout L = make_layout(N, D, V);
   if (ws_bytes < L.fwd_total) return FLCE_ERR_WORKSPACE;
   DevInfo di;
   flce_status st = device_setup(&di);
   if (st != FLCE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsPtrs p = carve(ws, L);
   const bool bf16 = dtype == FLCE_BF16;
   const MapType mt = bf16 ? kMapBF16 : kMapFP16;
 
   float* lossvec = none ? loss_rows : nullptr;
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, m, logs, nullptr, lossvec, s);
+  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, L, p, shard ? nullptr : m,
+                shard ? nullptr : logs, shard ? p.pos : nullptr, lossvec, s);
   if (st != FLCE_OK) return st;
 
   GemmArgs a{};
@@ -415,8 +383,18 @@ flce_status flce_forward_ex(const void* H, const void* W, const void* b, const i
   a.err = p.err;
   FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
+  const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
+  if (shard) {
+    if (N > 0) {
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+        shard_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.yc, p.pos, N,
+            static_cast<int>(V), stats, p.err);
+      }));
+    }
+    return FLCE_OK;
+  }
   if (N > 0) {
-    const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
           p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
@@ -433,24 +411,15 @@ flce_status flce_forward_ex(const void* H, const void* W, const void* b, const i
   return FLCE_OK;
 }
 
-flce_status flce_backward(const void* H, const void* W, const void* b, const int64_t* labels,
+// Backward of the full vocabulary (v0 = 0, V_total = V) or of the slice
+// [v0, v0 + V): dW, db are the slice's rows and dH its term of the sum.
+flce_status backward_impl(const void* H, const void* W, const void* b, const int64_t* labels,
                           const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
-                          int64_t V, int dtype, const float* m, const float* logs, float lambda,
-                          const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
-                          size_t ws_bytes, flce_stream stream) {
-  return flce_backward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, m, logs, nullptr,
-                          FLCE_REDUCE_MEAN, 0.f, 0u, lambda, lambda_dev, nullptr, dH, dW, db, ws,
-                          ws_bytes, stream);
-}
-
-flce_status flce_backward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
-                             const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
-                             int64_t V, int dtype, const float* m, const float* logs,
-                             const float* weight, int reduction, float denom, unsigned flags,
-                             float lambda,
-                             const float* lambda_dev, const float* grad_rows, float* dH,
-                             float* dW, float* db, void* ws, size_t ws_bytes,
-                             flce_stream stream) {
+                          int64_t V, int64_t v0, int64_t V_total, int dtype, const float* m,
+                          const float* logs, const float* weight, int reduction, float denom,
+                          unsigned flags, float lambda, const float* lambda_dev,
+                          const float* grad_rows, float* dH, float* dW, float* db, void* ws,
+                          size_t ws_bytes, cudaStream_t s) {
   if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
        reduction != FLCE_REDUCE_NONE) ||
       (flags & ~FLCE_FLAG_ROUND_LOGITS) != 0)
@@ -461,7 +430,8 @@ flce_status flce_backward_ex(const void* H, const void* W, const void* b, const 
       W == nullptr || dW == nullptr || ws == nullptr || (b != nullptr && db == nullptr))
     return FLCE_ERR_NULL;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP16) return FLCE_ERR_DTYPE;
-  if (!shape_ok(N, D, V)) return FLCE_ERR_SHAPE;
+  if (!shape_ok(N, D, V) || v0 < 0 || V_total > kMaxV || v0 + V > V_total)
+    return FLCE_ERR_SHAPE;
   if (D % 8 != 0 || !aligned(H, 16) || !aligned(W, 16) || (b != nullptr && !aligned(b, 16)) ||
       !aligned(ws, 256) || !aligned(dH, 16) || !aligned(dW, 16) ||
       (db != nullptr && !aligned(db, 8)) || !aligned(m, 4) || !aligned(logs, 4) ||
@@ -472,14 +442,14 @@ flce_status flce_backward_ex(const void* H, const void* W, const void* b, const 
   DevInfo di;
   flce_status st = device_setup(&di);
   if (st != FLCE_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsPtrs p = carve(ws, L);
   const bool bf16 = dtype == FLCE_BF16;
   const MapType mt = bf16 ? kMapBF16 : kMapFP16;
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V, L, p, nullptr, nullptr, p.pos, nullptr,
+  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, L, p, nullptr, nullptr, p.pos,
+                nullptr,
                 s);
   if (st != FLCE_OK) return st;
   FLCE_CK(timed_launch(kProfAux, s, [&] {
@@ -568,6 +538,181 @@ flce_status flce_backward_ex(const void* H, const void* W, const void* b, const 
   return FLCE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype) {
+  if (!shape_ok(N, D, V) || (dtype != FLCE_BF16 && dtype != FLCE_FP16)) return 0;
+  return make_layout(N, D, V).total;
+}
+
+const char* flce_status_string(int status) {
+  switch (status) {
+    case FLCE_OK: return "FLCE_OK";
+    case FLCE_ERR_NULL: return "FLCE_ERR_NULL: a required pointer is NULL";
+    case FLCE_ERR_SHAPE: return "FLCE_ERR_SHAPE: N, D or V out of range";
+    case FLCE_ERR_DTYPE: return "FLCE_ERR_DTYPE: dtype must be FLCE_BF16 or FLCE_FP16";
+    case FLCE_ERR_ALIGN: return "FLCE_ERR_ALIGN: misaligned pointer or D not a multiple of 8";
+    case FLCE_ERR_WORKSPACE: return "FLCE_ERR_WORKSPACE: workspace too small";
+    case FLCE_ERR_CUDA: return "FLCE_ERR_CUDA: a CUDA runtime call failed";
+    case FLCE_ERR_LABEL: return "FLCE_ERR_LABEL: supervised label outside [0, V)";
+    case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT: a device pipeline wait ran out";
+    case FLCE_ERR_NONFINITE: return "FLCE_ERR_NONFINITE: non-finite per-row statistic";
+    case FLCE_ERR_DEVICE: return "FLCE_ERR_DEVICE: current device is not sm_100";
+    case FLCE_ERR_ARG: return "FLCE_ERR_ARG: invalid argument value";
+    case FLCE_ERR_SHARD:
+      return "FLCE_ERR_SHARD: a supervised label is held by no vocabulary slice or by several";
+    default: return "FLCE_ERR_UNKNOWN";
+  }
+}
+
+flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                         int64_t N, int64_t V, int32_t* idx, int32_t* C_out, void* ws,
+                         size_t ws_bytes, flce_stream stream) {
+  if ((N > 0 && (labels == nullptr || idx == nullptr)) || C_out == nullptr || ws == nullptr)
+    return FLCE_ERR_NULL;
+  if (N < 0 || N > kMaxN || V < 1 || V > kMaxV) return FLCE_ERR_SHAPE;
+  if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
+  if (ws_bytes < 256) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, 0, idx, nullptr,
+                                                 C_out, err, nullptr, nullptr, nullptr, nullptr);
+  }));
+  return FLCE_OK;
+}
+
+flce_status flce_forward(const void* H, const void* W, const void* b, const int64_t* labels,
+                         const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                         int64_t V, int dtype, float* loss, float* m, float* logs, void* ws,
+                         size_t ws_bytes, flce_stream stream) {
+  return flce_forward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, nullptr,
+                         FLCE_REDUCE_MEAN, 0.f, 0u, loss, nullptr, m, logs, ws, ws_bytes,
+                         stream);
+}
+
+flce_status flce_forward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
+                            const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                            int64_t V, int dtype, const float* weight, int reduction, float denom,
+                            unsigned flags, float* loss, float* loss_rows, float* m, float* logs,
+                            void* ws,
+                            size_t ws_bytes, flce_stream stream) {
+  return forward_impl(H, W, b, labels, mask, ignore_index, N, D, V, 0, V, dtype, weight,
+                      reduction, denom, flags, loss, loss_rows, m, logs, false, nullptr, ws,
+                      ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_shard_forward(const void* H, const void* W_slice, const void* b_slice,
+                               const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                               int64_t N, int64_t D, int64_t V_slice, int64_t v0,
+                               int64_t V_total, int dtype, unsigned flags, float* stats,
+                               void* ws, size_t ws_bytes, flce_stream stream) {
+  return forward_impl(H, W_slice, b_slice, labels, mask, ignore_index, N, D, V_slice, v0,
+                      V_total, dtype, nullptr, FLCE_REDUCE_MEAN, 0.f, flags, nullptr, nullptr,
+                      nullptr, nullptr, true, reinterpret_cast<float4*>(stats), ws, ws_bytes,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t flce_shard_combine_workspace_bytes(int64_t N) {
+  if (N < 0 || N > kMaxN) return 0;
+  return combine_layout(N).total;
+}
+
+flce_status flce_shard_combine(const float* stats_all, int P, const int64_t* labels,
+                               const uint8_t* mask, int64_t ignore_index, int64_t N,
+                               const float* weight, int reduction, float denom, float* loss,
+                               float* loss_rows, float* m, float* logs, void* ws,
+                               size_t ws_bytes, flce_stream stream) {
+  if (reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
+      reduction != FLCE_REDUCE_NONE)
+    return FLCE_ERR_ARG;
+  const bool none = reduction == FLCE_REDUCE_NONE;
+  if ((N > 0 && (stats_all == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
+                 (none && loss_rows == nullptr))) ||
+      (!none && loss == nullptr) || ws == nullptr)
+    return FLCE_ERR_NULL;
+  if (N < 0 || N > kMaxN || P < 1 || P > kMaxShards) return FLCE_ERR_SHAPE;
+  if (!aligned(stats_all, 16) || !aligned(ws, 256) || !aligned(m, 4) || !aligned(logs, 4) ||
+      !aligned(loss, 4) || !aligned(weight, 4) || !aligned(loss_rows, 4))
+    return FLCE_ERR_ALIGN;
+  const CombineLayout L = combine_layout(N);
+  if (ws_bytes < L.total) return FLCE_ERR_WORKSPACE;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(w);
+  int* C = reinterpret_cast<int*>(w + L.C);
+  int* idx = reinterpret_cast<int*>(w + L.idx);
+  float* rows = reinterpret_cast<float*>(w + L.loss_rows);
+  float* lossvec = none ? loss_rows : nullptr;
+  FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
+  // labels were range-checked by the slices' forwards; V here only bounds them again
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, kMaxV, 0, idx,
+                                                 nullptr, C, err, m, logs, nullptr, lossvec);
+  }));
+  if (N > 0) {
+    const int64_t blocks = cdiv64(N, 256) < 4LL * di.sms ? cdiv64(N, 256) : 4LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      shard_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(stats_all), P, N, C, idx, m, logs, rows, weight,
+          lossvec, err);
+    }));
+  }
+  if (!none) {
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      loss_reduce_kernel<<<1, 1024, 0, s>>>(rows, C, reduction == FLCE_REDUCE_MEAN ? 1 : 0,
+                                            denom, err, loss);
+    }));
+  }
+  return FLCE_OK;
+}
+
+flce_status flce_backward(const void* H, const void* W, const void* b, const int64_t* labels,
+                          const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                          int64_t V, int dtype, const float* m, const float* logs, float lambda,
+                          const float* lambda_dev, float* dH, float* dW, float* db, void* ws,
+                          size_t ws_bytes, flce_stream stream) {
+  return flce_backward_ex(H, W, b, labels, mask, ignore_index, N, D, V, dtype, m, logs, nullptr,
+                          FLCE_REDUCE_MEAN, 0.f, 0u, lambda, lambda_dev, nullptr, dH, dW, db, ws,
+                          ws_bytes, stream);
+}
+
+flce_status flce_backward_ex(const void* H, const void* W, const void* b, const int64_t* labels,
+                             const uint8_t* mask, int64_t ignore_index, int64_t N, int64_t D,
+                             int64_t V, int dtype, const float* m, const float* logs,
+                             const float* weight, int reduction, float denom, unsigned flags,
+                             float lambda,
+                             const float* lambda_dev, const float* grad_rows, float* dH,
+                             float* dW, float* db, void* ws, size_t ws_bytes,
+                             flce_stream stream) {
+  return backward_impl(H, W, b, labels, mask, ignore_index, N, D, V, 0, V, dtype, m, logs, weight,
+                       reduction, denom, flags, lambda, lambda_dev, grad_rows, dH, dW, db, ws,
+                       ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_shard_backward(const void* H, const void* W_slice, const void* b_slice,
+                                const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
+                                int64_t N, int64_t D, int64_t V_slice, int64_t v0,
+                                int64_t V_total, int dtype, const float* m, const float* logs,
+                                const float* weight, int reduction, float denom, unsigned flags,
+                                float lambda, const float* lambda_dev, const float* grad_rows,
+                                float* dH, float* dW_slice, float* db_slice, void* ws,
+                                size_t ws_bytes, flce_stream stream) {
+  return backward_impl(H, W_slice, b_slice, labels, mask, ignore_index, N, D, V_slice, v0,
+                       V_total, dtype, m, logs, weight, reduction, denom, flags, lambda,
+                       lambda_dev, grad_rows, dH, dW_slice, db_slice, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream));
+}
+
 flce_status flce_device_status(const void* ws, flce_stream stream) {
   if (ws == nullptr) return FLCE_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -576,6 +721,7 @@ flce_status flce_device_status(const void* ws, flce_stream stream) {
   if (cudaMemcpy(&e, ws, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return FLCE_ERR_CUDA;
   if (e & kErrBitLabel) return FLCE_ERR_LABEL;
   if (e & kErrBitTimeout) return FLCE_ERR_TIMEOUT;
+  if (e & kErrBitShard) return FLCE_ERR_SHARD;
   if (e & kErrBitNonfinite) return FLCE_ERR_NONFINITE;
   if (e != 0) return FLCE_ERR_CUDA;
   return FLCE_OK;

@@ -13,6 +13,7 @@ namespace flce {
 constexpr uint32_t kErrBitLabel = 1u << 7;
 constexpr uint32_t kErrBitTimeout = 1u << 8;
 constexpr uint32_t kErrBitNonfinite = 1u << 9;
+constexpr uint32_t kErrBitShard = 1u << 10;  // a label held by no slice or by several
 
 // Upper bound on any single pipeline wait inside a kernel.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s

@@ -16,6 +16,8 @@ floor does.
 import numpy as np
 import torch
 
+from oracle import flce_oracle as orc
+
 LOSS_RTOL = 1e-4
 STAT_RTOL = 1e-5
 GRAD_RTOL = 2e-3
@@ -67,3 +69,39 @@ def check_grad(name, got, ref):
     err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
     assert err <= GRAD_RTOL * scale, (name, err, scale)
     return err / scale if scale > 0 else 0.0
+
+
+def sampled_check(inp, got, n_rows=64, n_cols=192, full_stats=True):
+    rng = np.random.default_rng(0)
+    idx, C = orc.supervised_rows(inp.labels, inp.mask)
+    H64, W64, b64 = inp.H64(), inp.W64(), inp.b64()
+    rows = np.sort(rng.choice(idx, size=min(n_rows, C), replace=False))
+    r = orc.row_outputs(H64, W64, b64, inp.labels, inp.mask, -100, inp.lam, rows)
+    check_stats(got["m"][rows], r["m"])
+    check_stats(got["logs"][rows], r["logs"], floor=logs_floor(r["m"], inp.D))
+    if full_stats:
+        f = orc.forward(H64, W64, b64, inp.labels, inp.mask)
+        check_loss(got["loss"], f["loss"])
+        check_stats(got["m"], f["m"], idx)
+        check_stats(got["logs"], f["logs"], idx, floor=logs_floor(f["m"][idx], inp.D))
+        # vocabulary columns: the most frequent targets, the tail tile, random ids
+        ys, counts = np.unique(inp.labels[idx], return_counts=True)
+        hot = ys[np.argsort(-counts)[:32]]
+        cols = np.unique(np.concatenate([hot, [0, inp.V - 1],
+                                         rng.choice(inp.V, n_cols, replace=False)]))
+        dW, db = orc.vocab_outputs(H64, W64, b64, inp.labels, inp.mask, -100, inp.lam,
+                                   f["m"], f["logs"], cols)
+        # tolerance scale: the largest dW / db entry, which sits in a hot target row
+        check_grad("dW[cols]", got["dW"][cols], dW)
+        if b64 is not None:
+            check_grad("db[cols]", got["db"][cols], db)
+    # dH rows: the tolerance scale is the largest |dH| among the sampled rows,
+    # never above the largest over all rows, so this is at least as strict.
+    check_grad("dH[rows]", got["dH"][rows], r["dH"])
+    # a property of every size: sum_j p_ij = 1 gives sum_j dW_j = 0
+    dWd = got["dW"].astype(np.float64)
+    colsum = np.abs(dWd.sum(axis=0))
+    assert np.all(colsum <= 1e-3 * np.abs(dWd).sum(axis=0) + 1e-30), colsum.max()
+    unsup = np.setdiff1d(np.arange(inp.N), idx)
+    assert not got["dH"][unsup].any()
+    assert np.all(np.isneginf(got["m"][unsup]))

@@ -180,3 +180,80 @@ def test_forward_ex_argument_errors(L, kw, want):
 ])
 def test_backward_ex_argument_errors(L, kw, want):
     assert bwd_ex(L, **kw) == S[want]
+
+
+def sfwd(L, **kw):
+    a = dict(H=FAKE, W=FAKE, b=None, labels=FAKE, mask=None, ig=-100, N=64, D=32, V=1000, v0=0,
+             Vt=1000, dt=0, fl=0, st=FAKE, ws=FAKE, wsb=1 << 40, s=None)
+    a.update(kw)
+    return L.flce_shard_forward(P(a["H"]), P(a["W"]), P(a["b"]), P(a["labels"]), P(a["mask"]),
+                                a["ig"], a["N"], a["D"], a["V"], a["v0"], a["Vt"], a["dt"],
+                                a["fl"], P(a["st"]), P(a["ws"]), a["wsb"], P(a["s"]))
+
+
+def scomb(L, **kw):
+    a = dict(st=FAKE, Pn=2, labels=FAKE, mask=None, ig=-100, N=64, w=None, red=0, den=0.0,
+             loss=FAKE, rows=None, m=FAKE, logs=FAKE, ws=FAKE, wsb=1 << 40, s=None)
+    a.update(kw)
+    return L.flce_shard_combine(P(a["st"]), a["Pn"], P(a["labels"]), P(a["mask"]), a["ig"],
+                                a["N"], P(a["w"]), a["red"], a["den"], P(a["loss"]),
+                                P(a["rows"]), P(a["m"]), P(a["logs"]), P(a["ws"]), a["wsb"],
+                                P(a["s"]))
+
+
+def sbwd(L, **kw):
+    a = dict(H=FAKE, W=FAKE, b=None, labels=FAKE, mask=None, ig=-100, N=64, D=32, V=1000, v0=0,
+             Vt=1000, dt=0, m=FAKE, logs=FAKE, w=None, red=0, den=0.0, fl=0, lam=1.0, lamd=None,
+             g=None, dH=FAKE, dW=FAKE, db=None, ws=FAKE, wsb=1 << 40, s=None)
+    a.update(kw)
+    return L.flce_shard_backward(P(a["H"]), P(a["W"]), P(a["b"]), P(a["labels"]), P(a["mask"]),
+                                 a["ig"], a["N"], a["D"], a["V"], a["v0"], a["Vt"], a["dt"],
+                                 P(a["m"]), P(a["logs"]), P(a["w"]), a["red"], a["den"], a["fl"],
+                                 a["lam"], P(a["lamd"]), P(a["g"]), P(a["dH"]), P(a["dW"]),
+                                 P(a["db"]), P(a["ws"]), a["wsb"], P(a["s"]))
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(st=None), "FLCE_ERR_NULL"),
+    (dict(W=None), "FLCE_ERR_NULL"),
+    (dict(v0=-1), "FLCE_ERR_SHAPE"),
+    (dict(v0=1, Vt=1000), "FLCE_ERR_SHAPE"),          # slice runs past V_total
+    (dict(Vt=(1 << 24) + 1, v0=(1 << 24) - 999), "FLCE_ERR_SHAPE"),
+    (dict(st=FAKE + 8), "FLCE_ERR_ALIGN"),            # float4 rows need 16 bytes
+    (dict(fl=4), "FLCE_ERR_ARG"),
+    (dict(dt=5), "FLCE_ERR_DTYPE"),
+    (dict(wsb=2048), "FLCE_ERR_WORKSPACE"),
+])
+def test_shard_forward_argument_errors(L, kw, want):
+    assert sfwd(L, **kw) == S[want]
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(st=None), "FLCE_ERR_NULL"),
+    (dict(m=None), "FLCE_ERR_NULL"),
+    (dict(red=2, rows=None), "FLCE_ERR_NULL"),
+    (dict(red=4), "FLCE_ERR_ARG"),
+    (dict(Pn=0), "FLCE_ERR_SHAPE"),
+    (dict(N=-3), "FLCE_ERR_SHAPE"),
+    (dict(st=FAKE + 4), "FLCE_ERR_ALIGN"),
+    (dict(wsb=256), "FLCE_ERR_WORKSPACE"),
+])
+def test_shard_combine_argument_errors(L, kw, want):
+    assert scomb(L, **kw) == S[want]
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(dW=None), "FLCE_ERR_NULL"),
+    (dict(b=FAKE, db=None), "FLCE_ERR_NULL"),
+    (dict(v0=4, Vt=1004, wsb=4096), "FLCE_ERR_WORKSPACE"),
+    (dict(v0=10, Vt=1004), "FLCE_ERR_SHAPE"),
+    (dict(fl=2), "FLCE_ERR_ARG"),
+])
+def test_shard_backward_argument_errors(L, kw, want):
+    assert sbwd(L, **kw) == S[want]
+
+
+def test_shard_combine_workspace_bytes(L):
+    assert L.flce_shard_combine_workspace_bytes(-1) == 0
+    a = L.flce_shard_combine_workspace_bytes(1000)
+    assert a >= 2 * 1000 * 4 and a < L.flce_shard_combine_workspace_bytes(100000)

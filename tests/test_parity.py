@@ -8,7 +8,8 @@ from lm_head_projection_supervised_b200 import binding
 from lm_head_projection_supervised_b200 import workloads as wl
 from oracle import flce_oracle as orc
 
-from _gpu_helpers import check_grad, check_loss, check_stats, logs_floor, to_device
+from _gpu_helpers import (check_grad, check_loss, check_stats, logs_floor, sampled_check,
+                          to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -185,42 +186,6 @@ def test_autograd_wrapper_matches_abi():
 # --------------------------------------------------------------------------
 # full-size workloads, as the benchmark launches them
 # --------------------------------------------------------------------------
-def sampled_check(inp, got, n_rows=64, n_cols=192, full_stats=True):
-    rng = np.random.default_rng(0)
-    idx, C = orc.supervised_rows(inp.labels, inp.mask)
-    H64, W64, b64 = inp.H64(), inp.W64(), inp.b64()
-    rows = np.sort(rng.choice(idx, size=min(n_rows, C), replace=False))
-    r = orc.row_outputs(H64, W64, b64, inp.labels, inp.mask, -100, inp.lam, rows)
-    check_stats(got["m"][rows], r["m"])
-    check_stats(got["logs"][rows], r["logs"], floor=logs_floor(r["m"], inp.D))
-    if full_stats:
-        f = orc.forward(H64, W64, b64, inp.labels, inp.mask)
-        check_loss(got["loss"], f["loss"])
-        check_stats(got["m"], f["m"], idx)
-        check_stats(got["logs"], f["logs"], idx, floor=logs_floor(f["m"][idx], inp.D))
-        # vocabulary columns: the most frequent targets, the tail tile, random ids
-        ys, counts = np.unique(inp.labels[idx], return_counts=True)
-        hot = ys[np.argsort(-counts)[:32]]
-        cols = np.unique(np.concatenate([hot, [0, inp.V - 1],
-                                         rng.choice(inp.V, n_cols, replace=False)]))
-        dW, db = orc.vocab_outputs(H64, W64, b64, inp.labels, inp.mask, -100, inp.lam,
-                                   f["m"], f["logs"], cols)
-        # tolerance scale: the largest dW / db entry, which sits in a hot target row
-        check_grad("dW[cols]", got["dW"][cols], dW)
-        if b64 is not None:
-            check_grad("db[cols]", got["db"][cols], db)
-    # dH rows: the tolerance scale is the largest |dH| among the sampled rows,
-    # never above the largest over all rows, so this is at least as strict.
-    check_grad("dH[rows]", got["dH"][rows], r["dH"])
-    # a property of every size: sum_j p_ij = 1 gives sum_j dW_j = 0
-    dWd = got["dW"].astype(np.float64)
-    colsum = np.abs(dWd.sum(axis=0))
-    assert np.all(colsum <= 1e-3 * np.abs(dWd).sum(axis=0) + 1e-30), colsum.max()
-    unsup = np.setdiff1d(np.arange(inp.N), idx)
-    assert not got["dH"][unsup].any()
-    assert np.all(np.isneginf(got["m"][unsup]))
-
-
 @pytest.mark.parametrize("name", ["page2", "packed"])
 def test_full_size_sampled(name):
     inp = wl.make_inputs(name)

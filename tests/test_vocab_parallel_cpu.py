@@ -1,0 +1,163 @@
+"""Host logic of the vocabulary-parallel path on CPU: the cut of the
+vocabulary, and the exchange (all-gather of the statistics, all-reduce of dH)
+between gloo ranks, with the compute steps supplied by the oracle so that no
+GPU is needed.  The product path's compute steps are the CUDA calls; this
+file checks only what the module does around them."""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+from lm_head_projection_supervised_b200 import vocab_parallel as vp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("V,P", [(248320, 8), (248320, 3), (32000, 8), (1000, 7), (9, 9),
+                                 (257, 2), (512, 2), (100000, 1)])
+def test_vocab_slice_partitions_the_vocabulary(V, P):
+    cuts = [vp.vocab_slice(V, P, r) for r in range(P)]
+    v = 0
+    for v0, n in cuts:
+        assert v0 == v and n >= 1
+        v += n
+    assert v == V
+    if V >= 256 * P:
+        assert all(v0 % 256 == 0 for v0, _ in cuts)
+        sizes = [n for _, n in cuts[:-1]]
+        assert max(sizes) - min(sizes) <= 256 if sizes else True
+
+
+def test_vocab_slice_rejects_bad_arguments():
+    with pytest.raises(ValueError):
+        vp.vocab_slice(5, 6, 0)
+    with pytest.raises(ValueError):
+        vp.vocab_slice(100, 2, 2)
+
+
+class OracleOps:
+    """The three compute steps from the CPU oracle (float64 CPU tensors)."""
+
+    @staticmethod
+    def shard_forward(H, W_slice, b_slice, labels, mask=None, ignore_index=-100, v0=0,
+                      V_total=None, ws=None, round_logits=False):
+        from oracle import flce_shards as sh
+        st = sh.shard_partials(H.numpy(), W_slice.numpy(),
+                               None if b_slice is None else b_slice.numpy(), labels.numpy(),
+                               None if mask is None else mask.numpy(), ignore_index, v0=v0,
+                               V_total=V_total)
+        return torch.from_numpy(st)
+
+    @staticmethod
+    def shard_combine(stats_all, labels, mask=None, ignore_index=-100, weight=None,
+                      reduction="mean", denom=None):
+        from oracle import flce_shards as sh
+        r = sh.shard_combine(stats_all.numpy(), labels.numpy(),
+                             None if mask is None else mask.numpy(), ignore_index,
+                             None if weight is None else weight.numpy(), reduction, denom)
+        loss = torch.from_numpy(r["loss_vec"]) if reduction == "none" else \
+            torch.tensor(r["loss"], dtype=torch.float64)
+        return loss, torch.from_numpy(r["m"]), torch.from_numpy(r["logs"])
+
+    @staticmethod
+    def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index, m, logs, v0=0,
+                       V_total=None, lam=1.0, lam_dev=None, weight=None, reduction="mean",
+                       denom=None, grad_rows=None, round_logits=False, ws=None):
+        from oracle import flce_shards as sh
+        if lam_dev is not None:
+            lam = float(lam_dev)
+        out = sh.shard_backward(H.numpy(), W_slice.numpy(),
+                                None if b_slice is None else b_slice.numpy(), labels.numpy(),
+                                None if mask is None else mask.numpy(), ignore_index, v0=v0,
+                                V_total=V_total, lam=lam, m=m.numpy(), logs=logs.numpy(),
+                                weight=None if weight is None else weight.numpy(),
+                                reduction=reduction, denom=denom,
+                                grad_rows=None if grad_rows is None else grad_rows.numpy())
+        return tuple(None if t is None else torch.from_numpy(np.ascontiguousarray(t))
+                     for t in out)
+
+
+def _inputs(seed=11, N=37, D=9, V=611):
+    rng = np.random.default_rng(seed)
+    H = rng.standard_normal((N, D))
+    W = 0.6 * rng.standard_normal((V, D))
+    b = 0.2 * rng.standard_normal(V)
+    y = rng.integers(0, V, N)
+    y[rng.permutation(N)[:5]] = -100
+    mask = np.ones(N, dtype=np.uint8)
+    mask[rng.permutation(N)[:3]] = 0
+    w = rng.uniform(0.2, 1.8, N)
+    return H, W, b, y, mask, w
+
+
+def _worker(rank, world, port, reduction, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from lm_head_projection_supervised_b200 import vocab_parallel as vpar
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        H, W, b, y, mask, w = [torch.from_numpy(a) for a in _inputs()]
+        V = W.shape[0]
+        v0, n = vpar.vocab_slice(V, world, rank, align=64)
+        kw = dict(V_total=V, v0=v0, weight=w, reduction=reduction,
+                  denom=29.0 if reduction == "sum" else None, ops=OracleOps)
+        loss, m, logs = vpar.forward(H, W[v0:v0 + n], b[v0:v0 + n], y, mask, -100, **kw)
+        g = torch.linspace(-1.0, 2.0, H.shape[0], dtype=torch.float64)
+        bk = dict(kw, lam=0.8, grad_rows=g if reduction == "none" else None)
+        dH, dW, db = vpar.backward(H, W[v0:v0 + n], b[v0:v0 + n], y, mask, -100, m, logs, **bk)
+        q.put((rank, v0, n, loss.numpy(), m.numpy(), logs.numpy(), dH.numpy(), dW.numpy(),
+               db.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,reduction", [(2, "mean"), (3, "sum"), (2, "none")])
+def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
+    from oracle import flce_oracle as orc
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29600 + (os.getpid() + 7 * world) % 1000
+    procs = [ctx.Process(target=_worker, args=(r, world, port, reduction, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=180) for _ in range(world)], key=lambda t: t[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    H, W, b, y, mask, w = _inputs()
+    g = np.linspace(-1.0, 2.0, H.shape[0])
+    ref = orc.forward_backward(H, W, b, y, mask, lam=0.8, weight=w, reduction=reduction,
+                               denom=29.0 if reduction == "sum" else None,
+                               grad_rows=g if reduction == "none" else None)
+    idx = ref["idx"]
+    assert [r[1] for r in res] == sorted(r[1] for r in res)           # rank order = vocab order
+    for r in res:
+        _, v0, n, loss, m, logs, dH, dW, db = r
+        want = ref["loss_vec"] if reduction == "none" else ref["loss"]
+        assert np.max(np.abs(loss - want)) < 1e-12                    # same loss on every rank
+        assert np.max(np.abs(m[idx] - ref["m"][idx])) < 1e-13
+        assert np.max(np.abs(logs[idx] - ref["logs"][idx])) < 1e-12
+        assert np.max(np.abs(dH - ref["dH"])) < 1e-12                 # all-reduced dH
+        assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12     # local slice of dW
+        assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
+    assert sum(r[2] for r in res) == W.shape[0]
+
+
+def test_slices_on_one_device_with_oracle_ops():
+    """run_slices_on_one_device stacks and sums like the collectives do."""
+    from oracle import flce_oracle as orc
+    H, W, b, y, mask, w = _inputs(seed=12)
+    t = [torch.from_numpy(a) for a in (H, W, b, y, mask, w)]
+    got = vp.run_slices_on_one_device(*t[:5], P=4, lam=1.7, weight=t[5], ops=OracleOps)
+    ref = orc.forward_backward(H, W, b, y, mask, lam=1.7, weight=w)
+    assert abs(float(got["loss"]) - ref["loss"]) < 1e-12
+    assert np.max(np.abs(got["dH"].numpy() - ref["dH"])) < 1e-12
+    assert np.max(np.abs(got["dW"].numpy() - ref["dW"])) < 1e-12
+    assert np.max(np.abs(got["db"].numpy() - ref["db"])) < 1e-12
