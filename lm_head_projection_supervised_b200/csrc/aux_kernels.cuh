@@ -11,6 +11,7 @@
 namespace flce {
 
 constexpr int COMPACT_THREADS = 1024;
+constexpr int kNoColumn = -(1 << 30);  // y_c of a label that another vocabulary slice holds
 
 __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8_t* mask,
                                               int64_t ignore, int64_t i) {
@@ -23,14 +24,16 @@ __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8
 // contiguous slice, a block-wide exclusive scan of the slice counts gives
 // every thread its output offset.  Labels outside [0, V) on supervised rows
 // set the label error bit and are clamped to 0 so later indexing stays in
-// range.  y_c holds y - v0: the label's column in a vocabulary slice that
-// starts at v0 (v0 = 0 unsharded), outside [0, V_slice) when another slice
-// holds it.  Unsupervised rows get m = log s = -inf when m_out is given.
+// range.  y_c holds y - v0, the label's column in the vocabulary slice
+// [v0, v0 + V_slice) (the whole vocabulary unsharded), or kNoColumn when
+// another slice holds it, so that no column of this slice ever matches it.
+// Unsupervised rows get m = log s = -inf when m_out is given.
 // pos (optional) is the inverse map: pos[i] = compact row of i, or -1.
 // lossvec (optional) gets 0 on unsupervised rows (per-row loss output).
 __global__ void __launch_bounds__(COMPACT_THREADS)
     compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
-                   int64_t ignore, int64_t N, int64_t V, int64_t v0, int* __restrict__ idx,
+                   int64_t ignore, int64_t N, int64_t V, int64_t v0, int64_t V_slice,
+                   int* __restrict__ idx,
                    int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
                    float* __restrict__ m_out, float* __restrict__ logs_out,
                    int* __restrict__ pos, float* __restrict__ lossvec) {
@@ -73,7 +76,8 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
         y = 0;
       }
       idx[off] = static_cast<int>(i);
-      if (y_c != nullptr) y_c[off] = static_cast<int>(y - v0);
+      if (y_c != nullptr)
+        y_c[off] = (y >= v0 && y < v0 + V_slice) ? static_cast<int>(y - v0) : kNoColumn;
       if (pos != nullptr) pos[i] = off;
       ++off;
     } else {

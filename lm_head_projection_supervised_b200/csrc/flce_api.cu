@@ -302,12 +302,14 @@ WsPtrs carve(void* ws, const Layout& L) {
 
 // control block reset + compaction + gather of the supervised rows
 flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
-                     int64_t N, int64_t D, int64_t V, int64_t v0, const Layout& L, const WsPtrs& p,
+                     int64_t N, int64_t D, int64_t V, int64_t v0, int64_t V_slice,
+                     const Layout& L, const WsPtrs& p,
                      float* m_out, float* logs_out, int* pos, float* lossvec,
                      cudaStream_t s) {
   FLCE_CK(cudaMemsetAsync(p.err, 0, L.ctrl_bytes, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
-    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, v0, p.idx, p.yc, p.C,
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, v0, V_slice, p.idx,
+                                                 p.yc, p.C,
                                                  p.err, m_out, logs_out, pos, lossvec);
   }));
   const int64_t vec = D / 8;
@@ -358,7 +360,7 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   const MapType mt = bf16 ? kMapBF16 : kMapFP16;
 
   float* lossvec = none ? loss_rows : nullptr;
-  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, L, p, shard ? nullptr : m,
+  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, V, L, p, shard ? nullptr : m,
                 shard ? nullptr : logs, shard ? p.pos : nullptr, lossvec, s);
   if (st != FLCE_OK) return st;
 
@@ -448,9 +450,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
-  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, L, p, nullptr, nullptr, p.pos,
-                nullptr,
-                s);
+  st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, V, L, p, nullptr, nullptr,
+                p.pos, nullptr, s);
   if (st != FLCE_OK) return st;
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     row_scale_kernel<<<1, 1024, 0, s>>>(p.C, p.idx, weight, none ? grad_rows : nullptr,
@@ -582,7 +583,8 @@ flce_status flce_compact(const int64_t* labels, const uint8_t* mask, int64_t ign
   uint32_t* err = static_cast<uint32_t*>(ws);
   FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
-    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, 0, idx, nullptr,
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, V, 0, V, idx,
+                                                 nullptr,
                                                  C_out, err, nullptr, nullptr, nullptr, nullptr);
   }));
   return FLCE_OK;
@@ -656,8 +658,8 @@ flce_status flce_shard_combine(const float* stats_all, int P, const int64_t* lab
   FLCE_CK(cudaMemsetAsync(err, 0, 256, s));
   // labels were range-checked by the slices' forwards; V here only bounds them again
   FLCE_CK(timed_launch(kProfAux, s, [&] {
-    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, kMaxV, 0, idx,
-                                                 nullptr, C, err, m, logs, nullptr, lossvec);
+    compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore_index, N, kMaxV, 0, kMaxV,
+                                                 idx, nullptr, C, err, m, logs, nullptr, lossvec);
   }));
   if (N > 0) {
     const int64_t blocks = cdiv64(N, 256) < 4LL * di.sms ? cdiv64(N, 256) : 4LL * di.sms;
