@@ -44,6 +44,9 @@ def parse():
                    help="supervised rows per step of the reference (oracle) arm")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--vocab-shards", type=int, default=1,
+                   help="P > 1: the vocabulary-sliced form, all P slices on each GPU in turn "
+                        "(the kernels of a P-way vocabulary-parallel step, exchanges in place)")
     return p.parse_args()
 
 
@@ -275,10 +278,44 @@ def main():
     db = None if b is None else torch.empty(inp.V, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    P = args.vocab_shards
+    if P > 1:
+        from lm_head_projection_supervised_b200 import vocab_parallel as vpar
+        bounds = [vpar.vocab_slice(inp.V, P, r) for r in range(P)]
+        ws = binding.Workspace(inp.N, inp.D, max(n for _, n in bounds), tdt, dev)
+        stats = torch.empty((P, inp.N, 4), dtype=torch.float32, device=dev)
+        cws = binding.CombineWorkspace(inp.N, dev)
+        cfg["vocab_shards"] = P
+
+        def fwd():
+            for r, (v0, n) in enumerate(bounds):
+                binding.shard_forward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n], y,
+                                      mk, -100, v0=v0, V_total=inp.V, ws=ws, out=stats[r])
+            return binding.shard_combine(stats, y, mk, -100, ws=cws)
+
+        def bwd(m, logs):
+            for r, (v0, n) in enumerate(bounds):
+                binding.shard_backward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n], y,
+                                       mk, -100, m, logs, v0=v0, V_total=inp.V, lam=inp.lam,
+                                       ws=ws, accumulate_dh=r > 0,
+                                       out=(dH, dW[v0:v0 + n],
+                                            None if db is None else db[v0:v0 + n]))
+    else:
+        def fwd():
+            return binding.forward(H, W, b, y, mk, -100, ws=ws)
+
+        def bwd(m, logs):
+            binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws,
+                             out=(dH, dW, db))
+
     def step():
-        loss, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
-        binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws, out=(dH, dW, db))
+        loss, m, logs = fwd()
+        bwd(m, logs)
         return loss
+
+    def device_status():
+        st = binding.device_status(ws)
+        return st if st != 0 or P == 1 else binding.device_status(cws)
 
     def barrier():
         if world > 1:
@@ -288,7 +325,7 @@ def main():
     for _ in range(n_warm):
         step()
     torch.cuda.synchronize(dev)
-    st = binding.device_status(ws)
+    st = device_status()
     if st != 0:
         raise RuntimeError(f"device error during warm-up: {binding.status_string(st)}")
 
@@ -301,15 +338,15 @@ def main():
     for k in range(args.steps):
         e0, e1, e2 = evs[k]
         e0.record(stream)
-        loss, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
+        loss, m, logs = fwd()
         e1.record(stream)
-        binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws, out=(dH, dW, db))
+        bwd(m, logs)
         e2.record(stream)
     torch.cuda.synchronize(dev)
     prof = binding.profile_end()
     barrier()
     clocks = sampler.stop()
-    st = binding.device_status(ws)
+    st = device_status()
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {binding.status_string(st)}")
     total_ms = evs[0][0].elapsed_time(evs[-1][2])

@@ -190,6 +190,11 @@ typedef enum { FLCE_REDUCE_MEAN = 0, FLCE_REDUCE_SUM = 1, FLCE_REDUCE_NONE = 2 }
  *   ChunkedLinearCrossEntropy article).  The backward treats the rounding as
  *   the identity.  Pass the same flags to the forward and the backward. */
 #define FLCE_FLAG_ROUND_LOGITS 1u
+/* FLCE_FLAG_ACCUMULATE_DH (backward calls only): dH += this call's dH instead
+ *   of dH = this call's dH (rows of unsupervised positions are left as they
+ *   are).  With it the dH terms of several vocabulary slices, or of several
+ *   losses on one hidden state, sum in place. */
+#define FLCE_FLAG_ACCUMULATE_DH 2u
 
 /*
  * Forward with a reduction.  weight: device float [N] or NULL.  loss: device

@@ -23,6 +23,7 @@ STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DT
           11: "FLCE_ERR_ARG", 12: "FLCE_ERR_SHARD"}
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 FLAG_ROUND_LOGITS = 1
+FLAG_ACCUMULATE_DH = 2
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 _lib = None
@@ -157,6 +158,8 @@ def _prep(H, W, b, labels, mask):
         raise ValueError("labels must have one entry per row of H")
     y = y.contiguous()
     b2 = None if b is None else b.contiguous()
+    if b2 is not None and b2.data_ptr() % 16:
+        b2 = b2.clone()  # a vocabulary slice of a bias can start off the 16-byte grid
     return H2, W2, b2, y, _mask_u8(mask)
 
 
@@ -170,6 +173,11 @@ def _mask_u8(mask):
     elif mk.dtype != torch.uint8:
         mk = (mk != 0).view(torch.uint8)
     return mk.contiguous()
+
+
+def _flags(round_logits=False, accumulate_dh=False) -> int:
+    return (FLAG_ROUND_LOGITS if round_logits else 0) | \
+        (FLAG_ACCUMULATE_DH if accumulate_dh else 0)
 
 
 def _vec(t, N, device):
@@ -214,11 +222,12 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[W
 def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0, lam_dev=None,
              ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
              reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
-             round_logits: bool = False):
+             round_logits: bool = False, accumulate_dh: bool = False):
     """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex().
 
     For reduction "none", grad_rows [N] is the upstream gradient of each row's
-    loss; otherwise lam (or the device scalar lam_dev) is dJ/dL."""
+    loss; otherwise lam (or the device scalar lam_dev) is dJ/dL.  With
+    accumulate_dh the call adds its dH to out[0] instead of overwriting it."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
@@ -237,7 +246,7 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
     gr = _vec(grad_rows, N, H2.device)
     st = lib().flce_backward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
                                 D, V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red,
-                                float(denom or 0.0), FLAG_ROUND_LOGITS if round_logits else 0,
+                                float(denom or 0.0), _flags(round_logits, accumulate_dh),
                                 float(lam), _ptr(lam_dev), _ptr(gr),
                                 _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
                                 _stream(stream))
@@ -261,16 +270,19 @@ class CombineWorkspace:
 
 def shard_forward(H, W_slice, b_slice, labels, mask=None, ignore_index: int = -100, v0: int = 0,
                   V_total: Optional[int] = None, ws: Optional[Workspace] = None, stream=None,
-                  round_logits: bool = False):
+                  round_logits: bool = False, out=None):
     """Per-row partial statistics [N, 4] float32 (m_r, log s_r, t_r, o_r) of
-    the vocabulary slice [v0, v0 + V_slice) -- flce_shard_forward()."""
+    the vocabulary slice [v0, v0 + V_slice) -- flce_shard_forward().  out: an
+    optional contiguous float32 [N, 4] device tensor to write them to."""
     H2, W2, b2, y, mk = _prep(H, W_slice, b_slice, labels, mask)
     N, D = H2.shape
     Vs = W2.shape[0]
     V_total = v0 + Vs if V_total is None else int(V_total)
     if ws is None:
         ws = Workspace(N, D, Vs, H2.dtype, H2.device)
-    stats = torch.empty((N, 4), dtype=torch.float32, device=H2.device)
+    stats = torch.empty((N, 4), dtype=torch.float32, device=H2.device) if out is None else out
+    if stats.shape != (N, 4) or stats.dtype != torch.float32 or not stats.is_contiguous():
+        raise ValueError("out must be a contiguous float32 [N, 4] tensor")
     st = lib().flce_shard_forward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index,
                                   N, D, Vs, int(v0), V_total, dtype_code(H2.dtype),
                                   FLAG_ROUND_LOGITS if round_logits else 0, _ptr(stats),
@@ -314,9 +326,10 @@ def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index: int, m, logs
                    V_total: Optional[int] = None, lam: float = 1.0, lam_dev=None,
                    ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
                    reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
-                   round_logits: bool = False):
+                   round_logits: bool = False, accumulate_dh: bool = False):
     """(dH_r [N, D], dW_slice [V_slice, D], db_slice [V_slice] or None),
-    float32 -- flce_shard_backward().  dH_r is this slice's term of dH."""
+    float32 -- flce_shard_backward().  dH_r is this slice's term of dH (added
+    to out[0] with accumulate_dh)."""
     H2, W2, b2, y, mk = _prep(H, W_slice, b_slice, labels, mask)
     N, D = H2.shape
     Vs = W2.shape[0]
@@ -336,7 +349,7 @@ def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index: int, m, logs
     st = lib().flce_shard_backward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index,
                                    N, D, Vs, int(v0), V_total, dtype_code(H2.dtype), _ptr(m),
                                    _ptr(logs), _ptr(wt), REDUCTIONS[reduction],
-                                   float(denom or 0.0), FLAG_ROUND_LOGITS if round_logits else 0,
+                                   float(denom or 0.0), _flags(round_logits, accumulate_dh),
                                    float(lam), _ptr(lam_dev), _ptr(gr), _ptr(dH), _ptr(dW),
                                    _ptr(db), ws.ptr(), ws.nbytes, _stream(stream))
     _check(st, "flce_shard_backward")

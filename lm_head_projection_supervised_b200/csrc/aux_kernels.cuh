@@ -345,10 +345,18 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// dH[i] = dH_c[pos[i]] for supervised rows, 0 for the others (one warp per
-// row, 16-byte vectors).
+// dH[i] = dH_c[pos[i]] + (S / sigma) e_k W[y_k] for supervised rows (k =
+// pos[i]), 0 for the others.  e_k is what the 16-bit rounding took off the
+// row's target entry of the gradient panel, so this adds back the exact
+// target term in fp32; labels of another vocabulary slice (y_k outside
+// [0, V_slice)) carry none.  accumulate != 0: dH[i] += that value instead
+// (unsupervised rows unchanged).  One warp per row, 16-byte vectors of dH.
 __global__ void scatter_dh_kernel(const float4* __restrict__ dHc, const int* __restrict__ pos,
-                                  int64_t N, int64_t vec_per_row, float4* __restrict__ dH) {
+                                  int64_t N, int64_t vec_per_row, float4* __restrict__ dH,
+                                  const float* __restrict__ tgt_resid,
+                                  const int* __restrict__ y_c, const uint2* __restrict__ W,
+                                  int is_bf16, int V_slice, const float* __restrict__ scal,
+                                  float inv_sigma, int accumulate) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= N) return;
   const int lane = threadIdx.x & 31;
@@ -356,8 +364,43 @@ __global__ void scatter_dh_kernel(const float4* __restrict__ dHc, const int* __r
   float4* dst = dH + row * vec_per_row;
   if (p >= 0) {
     const float4* src = dHc + static_cast<int64_t>(p) * vec_per_row;
-    for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = src[k];
-  } else {
+    const int y = y_c[p];
+    const float c = tgt_resid[p] * (*scal) * inv_sigma;
+    if (c != 0.f && static_cast<unsigned>(y) < static_cast<unsigned>(V_slice)) {
+      const uint2* wr = W + static_cast<int64_t>(y) * vec_per_row;
+      for (int64_t k = lane; k < vec_per_row; k += 32) {
+        const uint2 wv = __ldg(wr + k);
+        float w0, w1, w2, w3;
+        if (is_bf16) {
+          w0 = __uint_as_float(wv.x << 16);
+          w1 = __uint_as_float(wv.x & 0xFFFF0000u);
+          w2 = __uint_as_float(wv.y << 16);
+          w3 = __uint_as_float(wv.y & 0xFFFF0000u);
+        } else {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&wv.x));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&wv.y));
+          w0 = a.x;
+          w1 = a.y;
+          w2 = b.x;
+          w3 = b.y;
+        }
+        float4 h = src[k];
+        if (accumulate) {
+          const float4 o = dst[k];
+          h = make_float4(h.x + o.x, h.y + o.y, h.z + o.z, h.w + o.w);
+        }
+        dst[k] = make_float4(fmaf(c, w0, h.x), fmaf(c, w1, h.y), fmaf(c, w2, h.z),
+                             fmaf(c, w3, h.w));
+      }
+    } else if (accumulate) {
+      for (int64_t k = lane; k < vec_per_row; k += 32) {
+        const float4 h = src[k], o = dst[k];
+        dst[k] = make_float4(h.x + o.x, h.y + o.y, h.z + o.z, h.w + o.w);
+      }
+    } else {
+      for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = src[k];
+    }
+  } else if (!accumulate) {
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
   }

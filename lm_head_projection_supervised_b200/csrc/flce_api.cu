@@ -33,6 +33,13 @@ constexpr int kMaxShards = 4096;  // vocabulary slices merged by one combine
 #define FLCE_PANEL_COLS 8192
 #endif
 constexpr int64_t kPanelCols = FLCE_PANEL_COLS;  // vocabulary columns per gradient panel
+#ifndef FLCE_G_PAD_COLS
+#define FLCE_G_PAD_COLS 0
+#endif
+// Extra 16-bit columns per gradient-panel row (row pitch = Vc + pad): a pitch
+// that is not a large power of two spreads a box's rows over more memory
+// channels.
+constexpr int64_t kPanelPad = FLCE_G_PAD_COLS;
 constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
 constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
@@ -41,8 +48,8 @@ int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, rs, dhc, gpanel[2], total;
-  int64_t Np, nvt, vc, panels;
+  size_t pos, rs, resid, dhc, gpanel[2], total;
+  int64_t Np, nvt, vc, gld, panels;
 };
 
 // Workspace carve-up.  The control block (error word, then one work counter
@@ -54,6 +61,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.nvt = cdiv64(V, BN);
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
   L.panels = cdiv64(V, L.vc);
+  L.gld = L.vc + kPanelPad;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -72,9 +80,10 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.pos = take(static_cast<size_t>(L.Np) * 4);
   L.fwd_total = off;
   L.rs = take(static_cast<size_t>(L.Np) * 4);
+  L.resid = take(static_cast<size_t>(L.Np) * 4);
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
-  L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.vc * 2);
-  L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.vc * 2);
+  L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.gld * 2);
+  L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.gld * 2);
   L.total = off;
   return L;
 }
@@ -275,6 +284,7 @@ struct WsPtrs {
   float* tgt;
   float* loss_rows;
   float* rs;
+  float* resid;
   float* dhc;
   uint16_t* gpanel[2];
 };
@@ -294,6 +304,7 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.tgt = reinterpret_cast<float*>(w + L.tgt);
   p.loss_rows = reinterpret_cast<float*>(w + L.loss_rows);
   p.rs = reinterpret_cast<float*>(w + L.rs);
+  p.resid = reinterpret_cast<float*>(w + L.resid);
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
   p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
   p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
@@ -424,7 +435,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
                           size_t ws_bytes, cudaStream_t s) {
   if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
        reduction != FLCE_REDUCE_NONE) ||
-      (flags & ~FLCE_FLAG_ROUND_LOGITS) != 0)
+      (flags & ~(FLCE_FLAG_ROUND_LOGITS | FLCE_FLAG_ACCUMULATE_DH)) != 0)
     return FLCE_ERR_ARG;
   const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
@@ -457,6 +468,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     row_scale_kernel<<<1, 1024, 0, s>>>(p.C, p.idx, weight, none ? grad_rows : nullptr,
                                         reduction, denom, lambda, lambda_dev, p.rs, p.scal);
   }));
+  // rows whose label another vocabulary slice holds keep a zero residual
+  FLCE_CK(cudaMemsetAsync(p.resid, 0, static_cast<size_t>(L.Np) * 4, s));
 
   // maps that do not depend on the panel
   CUtensorMap hcK, wK, hcMN, wMN, dwMap, dhMap;
@@ -485,12 +498,12 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.tmB[kClsDH] = wMN;
     a.tmDW = dwMap;
     a.tmDH = dhMap;
-    if (has_g && !make_map(&a.tmG, p.gpanel[Lp & 1], mt, w_g, L.Np, L.vc * 2, 64, BM))
+    if (has_g && !make_map(&a.tmG, p.gpanel[Lp & 1], mt, w_g, L.Np, L.gld * 2, 64, BM))
       return FLCE_ERR_CUDA;
     if (has_wh) {
       const uint16_t* gp = p.gpanel[(Lp - 1) & 1];
-      if (!make_map(&a.tmA[kClsDW], gp, mt, w_wh, L.Np, L.vc * 2, 64, BK) ||
-          !make_map(&a.tmA[kClsDH], gp, mt, w_wh, L.Np, L.vc * 2, BK, BM))
+      if (!make_map(&a.tmA[kClsDW], gp, mt, w_wh, L.Np, L.gld * 2, 64, BK) ||
+          !make_map(&a.tmA[kClsDH], gp, mt, w_wh, L.Np, L.gld * 2, BK, BM))
         return FLCE_ERR_CUDA;
     }
     a.is_bf16 = bf16;
@@ -513,6 +526,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.log2_sigma = log2_sigma;
     a.sigma = sigma;
     a.row_scale = p.rs;
+    a.tgt_resid = p.resid;
     a.scal = p.scal;
     a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
     a.inv_sigma = 1.f / sigma;
@@ -525,7 +539,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       const uint16_t* gp = p.gpanel[Lp & 1];
       FLCE_CK(timed_launch(kProfAux, s, [&] {
         bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w_g, 64)), 256, 0, s>>>(
-            gp, L.vc, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma, bf16 ? 1 : 0,
+            gp, L.gld, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma, bf16 ? 1 : 0,
             static_cast<int>(vp_g), db);
       }));
     }
@@ -533,7 +547,9 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
   if (N > 0) {
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       scatter_dh_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
-          reinterpret_cast<const float4*>(p.dhc), p.pos, N, D / 4, reinterpret_cast<float4*>(dH));
+          reinterpret_cast<const float4*>(p.dhc), p.pos, N, D / 4, reinterpret_cast<float4*>(dH),
+          p.resid, p.yc, static_cast<const uint2*>(W), bf16 ? 1 : 0, static_cast<int>(V), p.scal,
+          1.f / sigma, (flags & FLCE_FLAG_ACCUMULATE_DH) ? 1 : 0);
     }));
   }
   return FLCE_OK;

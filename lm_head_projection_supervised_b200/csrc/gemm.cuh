@@ -108,6 +108,8 @@ struct GemmArgs {
   float log2_sigma;        // bwd: the panel holds (p - onehot) * sigma
   float sigma;
   const float* row_scale;  // bwd: r_k, relative row scale of compact row k, in [-1, 1]
+  float* tgt_resid;        // bwd: per compact row, the target entry's value minus its 16-bit
+                           //      panel value (written by the tile that holds the label)
   const float* scal;       // bwd: S (device scalar); G = S r_k (p - onehot)
   float inv_sigma;
   float* out;              // plain
@@ -355,7 +357,8 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
                                            int vglob0, int vlim, int yl, bool valid, float mrow,
-                                           float krow, float rrow, uint32_t (&packed)[16]) {
+                                           float krow, float rrow, int row,
+                                           uint32_t (&packed)[16]) {
   float x[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(z[j]);
@@ -387,6 +390,17 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) gv[j] *= rrow;  // the row's scale relative to S
+  // The target entry r (p - 1) sigma dominates its row of dH; keep what the
+  // 16-bit rounding takes off it so that dH can add it back in fp32.
+  if (valid && static_cast<unsigned>(jt) < 32u) {
+    float resid = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j == jt)
+        resid = gv[j] - (g.is_bf16 ? __bfloat162float(__float2bfloat16_rn(gv[j]))
+                                   : __half2float(__float2half_rn(gv[j])));
+    g.tgt_resid[row] = resid;
+  }
   if (g.is_bf16) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -716,11 +730,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           named_bar_sync(1, NUM_EPI_THREADS);
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
-          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, pk);
+          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row, pk);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
           if (c + 2 < BN / 32) tmem_ld32(t_acc + (c + 2) * 32, za);
-          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, pk);
+          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row,
+                     pk);
           stage_row128(stg, r, 4, pk);
           if (c + 2 < BN / 32) tmem_wait_ld(za);
           fence_proxy_async_smem();

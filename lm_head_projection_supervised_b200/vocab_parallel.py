@@ -35,21 +35,22 @@ from . import binding
 def vocab_slice(V: int, P: int, r: int, align: int = 256) -> Tuple[int, int]:
     """(v0, V_r) of rank r when V vocabulary ids are cut into P slices.
 
-    Slice boundaries fall on multiples of `align` columns (the kernels' vocabulary
+    Slice boundaries fall on multiples of `align` ids (the kernels' vocabulary
     tile) when V >= align * P, so that only the last slice has a ragged tile;
-    otherwise the cut is the plain balanced one.  Slices are contiguous,
-    disjoint, cover [0, V) in rank order and are never empty."""
+    else on multiples of 8 ids (16 bytes of a 16-bit bias, so that a bias
+    slice stays on the TMA's 16-byte grid) when V >= 8 * P; else the plain
+    balanced cut.  Slices are contiguous, disjoint, cover [0, V) in rank
+    order and are never empty."""
     if P < 1 or not 0 <= r < P:
         raise ValueError("need 0 <= r < P")
     if V < P:
         raise ValueError("fewer vocabulary ids than slices")
-    if V >= align * P:
-        units = V // align
-        v0 = (r * units // P) * align
-        v1 = V if r == P - 1 else ((r + 1) * units // P) * align
-    else:
-        v0 = r * V // P
-        v1 = (r + 1) * V // P
+    for a in (align, 8, 1):
+        if V >= a * P:
+            break
+    units = V // a
+    v0 = (r * units // P) * a
+    v1 = V if r == P - 1 else ((r + 1) * units // P) * a
     return v0, v1 - v0
 
 
@@ -136,31 +137,35 @@ def vocab_parallel_cross_entropy(H, W_slice, labels, *, V_total: int, v0: int, g
 def run_slices_on_one_device(H, W, b, labels, mask=None, ignore_index: int = -100, P: int = 2,
                              lam: float = 1.0, weight=None, reduction: str = "mean",
                              denom: Optional[float] = None, grad_rows=None,
-                             round_logits: bool = False, ops=binding, ws=None):
-    """All P slices' calls on one device, one after the other, with the two
-    exchanges done as a local stack and a local sum: the same kernels and the
-    same data as a P-rank step, without a process group.
+                             round_logits: bool = False, ws=None, out=None):
+    """All P slices' calls on one device, one after the other: the same kernels
+    and data as a P-rank step, with the two exchanges done in place (each
+    slice writes its statistics into its row of one [P, N, 4] buffer, and adds
+    its dH term into one dH with FLCE_FLAG_ACCUMULATE_DH).
 
-    Returns dict(loss, m, logs, dH, dW, db) with dW and db the slices' results
-    concatenated back to [V, D] and [V].  ws, when given, is one workspace
-    large enough for the widest slice, shared by all calls."""
+    Returns dict(loss, m, logs, dH, dW, db); each slice writes its rows of dW
+    and db directly.  ws, when given, is one workspace large enough for the
+    widest slice, shared by all calls; out = (stats, dH, dW, db) preallocated
+    outputs (db None without bias)."""
+    N, D = H.reshape(-1, H.shape[-1]).shape
     V = W.shape[0]
     bounds = [vocab_slice(V, P, r) for r in range(P)]
-    stats = []
-    for v0, n in bounds:
-        stats.append(ops.shard_forward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n],
-                                       labels, mask, ignore_index, v0=v0, V_total=V,
-                                       ws=ws, round_logits=round_logits))
-    loss, m, logs = ops.shard_combine(torch.stack(stats), labels, mask, ignore_index,
-                                      weight=weight, reduction=reduction, denom=denom)
-    dH, dWs, dbs = None, [], []
-    for v0, n in bounds:
-        h, w, c = ops.shard_backward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n],
-                                     labels, mask, ignore_index, m, logs, v0=v0, V_total=V,
-                                     lam=lam, weight=weight, reduction=reduction, denom=denom,
-                                     grad_rows=grad_rows, round_logits=round_logits, ws=ws)
-        dH = h if dH is None else dH.add_(h)
-        dWs.append(w)
-        dbs.append(c)
-    return dict(loss=loss, m=m, logs=logs, dH=dH, dW=torch.cat(dWs),
-                db=None if b is None else torch.cat(dbs))
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=H.device)
+        out = (torch.empty((P, N, 4), **f32), torch.zeros((N, D), **f32),
+               torch.empty((V, D), **f32), None if b is None else torch.empty(V, **f32))
+    stats, dH, dW, db = out
+    for r, (v0, n) in enumerate(bounds):
+        binding.shard_forward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n], labels, mask,
+                              ignore_index, v0=v0, V_total=V, ws=ws, round_logits=round_logits,
+                              out=stats[r])
+    loss, m, logs = binding.shard_combine(stats, labels, mask, ignore_index, weight=weight,
+                                          reduction=reduction, denom=denom)
+    for r, (v0, n) in enumerate(bounds):
+        binding.shard_backward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n], labels,
+                               mask, ignore_index, m, logs, v0=v0, V_total=V, lam=lam,
+                               weight=weight, reduction=reduction, denom=denom,
+                               grad_rows=grad_rows, round_logits=round_logits, ws=ws,
+                               out=(dH, dW[v0:v0 + n], None if db is None else db[v0:v0 + n]),
+                               accumulate_dh=r > 0)
+    return dict(loss=loss, m=m, logs=logs, dH=dH, dW=dW, db=db)

@@ -161,7 +161,7 @@ def bwd_ex(L, **kw):
 @pytest.mark.parametrize("kw,want", [
     (dict(red=3), "FLCE_ERR_ARG"),
     (dict(red=-1), "FLCE_ERR_ARG"),
-    (dict(fl=2), "FLCE_ERR_ARG"),                    # unknown option bit
+    (dict(fl=2), "FLCE_ERR_ARG"),                    # dH accumulation: backward-only bit
     (dict(red=2, rows=None), "FLCE_ERR_NULL"),       # 'none' needs the per-row output
     (dict(red=1, loss=None), "FLCE_ERR_NULL"),       # 'sum' needs the scalar
     (dict(red=0, w=FAKE + 2), "FLCE_ERR_ALIGN"),
@@ -221,6 +221,7 @@ def sbwd(L, **kw):
     (dict(Vt=(1 << 24) + 1, v0=(1 << 24) - 999), "FLCE_ERR_SHAPE"),
     (dict(st=FAKE + 8), "FLCE_ERR_ALIGN"),            # float4 rows need 16 bytes
     (dict(fl=4), "FLCE_ERR_ARG"),
+    (dict(fl=2), "FLCE_ERR_ARG"),                    # dH accumulation: backward-only bit
     (dict(dt=5), "FLCE_ERR_DTYPE"),
     (dict(wsb=2048), "FLCE_ERR_WORKSPACE"),
 ])
@@ -247,7 +248,7 @@ def test_shard_combine_argument_errors(L, kw, want):
     (dict(b=FAKE, db=None), "FLCE_ERR_NULL"),
     (dict(v0=4, Vt=1004, wsb=4096), "FLCE_ERR_WORKSPACE"),
     (dict(v0=10, Vt=1004), "FLCE_ERR_SHAPE"),
-    (dict(fl=2), "FLCE_ERR_ARG"),
+    (dict(fl=4), "FLCE_ERR_ARG"),
 ])
 def test_shard_backward_argument_errors(L, kw, want):
     assert sbwd(L, **kw) == S[want]

@@ -1,7 +1,8 @@
 """GPU parity of the vocabulary-sharded calls (flce_shard_forward,
 flce_shard_combine, flce_shard_backward) against the oracle.  All slices run
-on one GPU, one after the other, with the two exchanges done as a local stack
-and a local sum (the same kernels and data as a multi-rank step)."""
+on one GPU, one after the other, with the two exchanges done in place (the
+statistics in one [P, N, 4] buffer, the dH terms summed by the backward's
+accumulate flag): the same kernels and data as a multi-rank step."""
 import numpy as np
 import pytest
 import torch
@@ -160,3 +161,20 @@ def test_packed_workload_eight_slices_sampled():
     res = dict(loss=got["loss"].item(), m=_np(got["m"]), logs=_np(got["logs"]),
                dH=_np(got["dH"]), dW=_np(got["dW"]), db=_np(got["db"]))
     sampled_check(inp, res, full_stats=True)
+
+
+def test_accumulate_dh_adds_in_place():
+    """FLCE_FLAG_ACCUMULATE_DH: dH += the call's dH; unsupervised rows keep
+    what they held."""
+    inp = wl.random_case(seed=62, N=300, D=64, V=4000)
+    H, W, b, y, mk = to_device(inp)
+    loss, m, logs = binding.forward(H, W, b, y, mk)
+    dH, dW, db = binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam)
+    base = torch.randn(inp.N, inp.D, device="cuda")
+    acc = base.clone()
+    binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, accumulate_dh=True,
+                     out=(acc, torch.empty_like(dW), torch.empty_like(db)))
+    idx, _ = orc.supervised_rows(inp.labels, inp.mask)
+    unsup = torch.from_numpy(np.setdiff1d(np.arange(inp.N), idx)).cuda()
+    assert torch.equal(acc[unsup], base[unsup])
+    assert (acc - (base + dH)).abs().max().item() <= 1e-6 * (base + dH).abs().max().item()

@@ -25,10 +25,10 @@ def test_vocab_slice_partitions_the_vocabulary(V, P):
         assert v0 == v and n >= 1
         v += n
     assert v == V
-    if V >= 256 * P:
-        assert all(v0 % 256 == 0 for v0, _ in cuts)
-        sizes = [n for _, n in cuts[:-1]]
-        assert max(sizes) - min(sizes) <= 256 if sizes else True
+    a = 256 if V >= 256 * P else 8 if V >= 8 * P else 1
+    assert all(v0 % a == 0 for v0, _ in cuts)
+    sizes = [n for _, n in cuts[:-1]]
+    assert max(sizes) - min(sizes) <= a if sizes else True
 
 
 def test_vocab_slice_rejects_bad_arguments():
@@ -148,16 +148,3 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
         assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12     # local slice of dW
         assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
     assert sum(r[2] for r in res) == W.shape[0]
-
-
-def test_slices_on_one_device_with_oracle_ops():
-    """run_slices_on_one_device stacks and sums like the collectives do."""
-    from oracle import flce_oracle as orc
-    H, W, b, y, mask, w = _inputs(seed=12)
-    t = [torch.from_numpy(a) for a in (H, W, b, y, mask, w)]
-    got = vp.run_slices_on_one_device(*t[:5], P=4, lam=1.7, weight=t[5], ops=OracleOps)
-    ref = orc.forward_backward(H, W, b, y, mask, lam=1.7, weight=w)
-    assert abs(float(got["loss"]) - ref["loss"]) < 1e-12
-    assert np.max(np.abs(got["dH"].numpy() - ref["dH"])) < 1e-12
-    assert np.max(np.abs(got["dW"].numpy() - ref["dW"])) < 1e-12
-    assert np.max(np.abs(got["db"].numpy() - ref["db"])) < 1e-12
