@@ -33,13 +33,6 @@ constexpr int kMaxShards = 4096;  // vocabulary slices merged by one combine
 #define FLCE_PANEL_COLS 8192
 #endif
 constexpr int64_t kPanelCols = FLCE_PANEL_COLS;  // vocabulary columns per gradient panel
-#ifndef FLCE_G_PAD_COLS
-#define FLCE_G_PAD_COLS 0
-#endif
-// Extra 16-bit columns per gradient-panel row (row pitch = Vc + pad): a pitch
-// that is not a large power of two spreads a box's rows over more memory
-// channels.
-constexpr int64_t kPanelPad = FLCE_G_PAD_COLS;
 constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
 constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
@@ -61,7 +54,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.nvt = cdiv64(V, BN);
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
   L.panels = cdiv64(V, L.vc);
-  L.gld = L.vc + kPanelPad;
+  L.gld = L.vc;  // gradient-panel row pitch in elements
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
