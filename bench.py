@@ -38,7 +38,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="flce", choices=["flce", "reference"])
     p.add_argument("--workload", default="packed")
-    p.add_argument("--cpu-rows", type=int, default=768,
+    p.add_argument("--cpu-rows", type=int, default=4096,
                    help="supervised rows in the CPU-oracle baseline sample")
     p.add_argument("--ref-rows", type=int, default=64,
                    help="supervised rows per step of the reference (oracle) arm")
