@@ -42,7 +42,7 @@ int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
   size_t pos, rs, resid, dhc, gpanel[2], total;
-  int64_t Np, nvt, vc, gld, panels;
+  int64_t Np, nvt, nparts, vc, gld, panels;
 };
 
 // Workspace carve-up.  The control block (error word, then one work counter
@@ -52,6 +52,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   Layout L{};
   L.Np = roundup64(N > 0 ? N : 1, PAIR_M);  // every half-tile of a CTA pair starts inside
   L.nvt = cdiv64(V, BN);
+  L.nparts = L.nvt * NUM_EPI_WG;  // forward (m, s) partials per row: one per half tile
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
   L.panels = cdiv64(V, L.vc);
   L.gld = L.vc;  // gradient-panel row pitch in elements
@@ -67,7 +68,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.idx = take(static_cast<size_t>(L.Np) * 4);
   L.yc = take(static_cast<size_t>(L.Np) * 4);
   L.hc = take(static_cast<size_t>(L.Np) * D * 2);
-  L.part = take(static_cast<size_t>(L.Np) * L.nvt * 8);
+  L.part = take(static_cast<size_t>(L.Np) * L.nparts * 8);
   L.tgt = take(static_cast<size_t>(L.Np) * 4);
   L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
   L.pos = take(static_cast<size_t>(L.Np) * 4);
@@ -174,6 +175,17 @@ flce_status device_setup(DevInfo* out) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(ModeCfg<kModePlain>::SMEM_BYTES)) != cudaSuccess)
         return FLCE_ERR_CUDA;
+      // The GEMM kernels split registers between warpgroups with setmaxnreg;
+      // the split only fits if the block was launched with enough of them.
+      for (const void* fn : {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd>),
+                             reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd>),
+                             reinterpret_cast<const void*>(flce_gemm_kernel<kModePlain>)}) {
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return FLCE_ERR_CUDA;
+        if (fa.numRegs < static_cast<int>(kRegsAtLaunch)) d.ok = false;
+      }
+    }
+    if (d.ok) {
       // how many CTA pairs can be resident together (one CTA per SM)
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -383,7 +395,7 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   a.idx = p.idx;
   a.bias = static_cast<const uint16_t*>(b);
   a.part = p.part;
-  a.part_ld = static_cast<int>(L.nvt);
+  a.part_ld = static_cast<int>(L.nparts);
   a.tgt = p.tgt;
   a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
   a.err = p.err;
@@ -394,7 +406,7 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
     if (N > 0) {
       FLCE_CK(timed_launch(kProfAux, s, [&] {
         shard_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.yc, p.pos, N,
+            p.part, static_cast<int>(L.nparts), static_cast<int>(L.nparts), p.tgt, p.yc, p.pos, N,
             static_cast<int>(V), stats, p.err);
       }));
     }
@@ -403,7 +415,7 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   if (N > 0) {
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-          p.part, static_cast<int>(L.nvt), static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs,
+          p.part, static_cast<int>(L.nparts), static_cast<int>(L.nparts), p.tgt, p.C, p.idx, m, logs,
           p.loss_rows, weight, lossvec, p.err);
     }));
   }

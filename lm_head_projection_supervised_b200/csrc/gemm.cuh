@@ -56,19 +56,35 @@ constexpr uint32_t B_STAGE_BYTES = BN_HALF * BK * 2;  // 16 KiB
 constexpr uint32_t PAIR_TX_BYTES = 2 * (A_STAGE_BYTES + B_STAGE_BYTES);  // both CTAs' loads
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;   // 8 KiB: 64 MN-elements x 64 K rows
 constexpr uint32_t STG_BYTES = BM * 128;         // 16 KiB: 128 rows x 128 bytes
-constexpr int NUM_THREADS = 256;
+// Warps 0-3 form the first warpgroup: scheduler + producer (warp 0), MMA
+// issuer (warp 1), two idle warps.  Warps 4-11 are the epilogue: two
+// warpgroups, each draining half of the accumulator's columns (warp w reads
+// TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, the rows of its quadrant).
+constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
-constexpr int NUM_EPI_THREADS = 128;
+constexpr int NUM_EPI_WG = 2;
+constexpr int EPI_WG_THREADS = 128;
+constexpr int NUM_EPI_THREADS = NUM_EPI_WG * EPI_WG_THREADS;
+constexpr int EPI_CHUNKS = BN / 32 / NUM_EPI_WG;  // 32-column chunks per epilogue warpgroup
+// Registers per thread after the split: the first warpgroup gives up what the
+// epilogue takes.  The block is launched with at least kRegsAtLaunch per
+// thread (checked on the host before any launch), which covers the split.
+constexpr uint32_t kRegsLow = 56;
+constexpr uint32_t kRegsHigh = 216;
+constexpr uint32_t kRegsAtLaunch =
+    (128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh + NUM_THREADS - 1) / NUM_THREADS;
+static_assert(128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr float kLog2e = 1.4426950408889634f;
 enum GemmMode : int { kModeFwd = 0, kModeBwd = 1, kModePlain = 2 };
 
-// Ring depth per mode: the backward epilogue stages TMA stores through two
-// 16 KiB boxes, the other modes use that shared memory for a 7th stage.
+// Ring depth per mode: the backward epilogue stages TMA stores through one
+// 16 KiB box per epilogue warpgroup, the other modes use that shared memory
+// for a 7th stage.
 template <int MODE>
 struct ModeCfg {
   static constexpr int STAGES = (MODE == kModeBwd) ? 6 : 7;
-  static constexpr uint32_t STAGING = (MODE == kModeBwd) ? 2 * STG_BYTES : 0;
+  static constexpr uint32_t STAGING = (MODE == kModeBwd) ? NUM_EPI_WG * STG_BYTES : 0;
   static constexpr size_t SMEM_BYTES =
       1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + STAGING + 512;
 };
@@ -331,6 +347,9 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
 #pragma unroll
   for (int j = 1; j < 32; ++j) cm = fmaxf(cm, x[j]);
   const float mn = fmaxf(st.m, cm);
+  // nothing seen yet and this chunk is all padding (a half tile past V): the
+  // state stays (-inf, 0) instead of exp(-inf + inf)
+  if (mn == -INFINITY) return;
   const float nb = -mn * kLog2e;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
@@ -516,6 +535,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   const int C = (MODE == kModePlain) ? g.M : *g.C_dev;
   const UnitSpace us = make_unit_space<MODE>(g, C);
 
+  if (warp < EPI_WARP0) {
+  setmaxnreg_dec<kRegsLow>();  // the whole first warpgroup
   if (warp == 0) {
     // ------------------------------------------------------------ scheduler + producer
     if (lane == 0) {
@@ -618,19 +639,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       umma_commit_pair_mc(done_bar, 0x1);
       mbar_wait(done_bar, 0, nullptr, nullptr, kDrainLimitNs);
     }
-  } else if (warp >= EPI_WARP0) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsHigh>();  // each epilogue warpgroup
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;              // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;         // row within this CTA's half of the tile
     const int rbase = static_cast<int>(rank) * BM;
     const int epi_tid = threadIdx.x - EPI_WARP0 * 32;
+    const int wg = epi_tid / EPI_WG_THREADS;   // epilogue warpgroup: columns [128 wg, 128 wg + 128)
+    const int wtid = epi_tid % EPI_WG_THREADS;
+    const int c0 = wg * EPI_CHUNKS;            // first 32-column chunk of this warpgroup
+    const uint32_t wg_bar = 2 + static_cast<uint32_t>(wg);  // named barrier of this warpgroup
+    uint8_t* stg = sStg + wg * STG_BYTES;      // this warpgroup's staging box (backward)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int acc = 0;
     uint32_t acc_phase = 0;
-    uint32_t nstore = 0;  // TMA stores issued by this CTA (staging buffer parity)
     float wh_scale = 0.f;
     if (MODE == kModeBwd) wh_scale = (C > 0) ? *g.scal * g.inv_sigma : 0.f;
-    // Shared decision of the four epilogue warps (they pass named barriers
+    // Shared decision of the eight epilogue warps (they pass named barriers
     // together, so they leave the loop together).
     int round = 0;
     auto decide_abort = [&]() -> bool {
@@ -639,16 +666,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       named_bar_sync(1, NUM_EPI_THREADS);
       return decision[(round++) & 1] != 0;
     };
-    // Stages one 128 x 128-byte box and hands it to the TMA engine.
+    // Stages one 128 x 128-byte box in this warpgroup's staging buffer and
+    // hands it to the TMA engine.
     auto emit_box = [&](const uint32_t (&w)[32], const CUtensorMap* map, int x, int y,
                         bool reduce, bool issue) {
-      uint8_t* stg = sStg + (nstore & 1u) * STG_BYTES;
-      if (epi_tid == 0) bulk_wait_group_read<1>();  // the box stored two boxes ago left smem
-      named_bar_sync(1, NUM_EPI_THREADS);
+      if (wtid == 0) bulk_wait_group_read<0>();  // the previous box has left the buffer
+      named_bar_sync(wg_bar, EPI_WG_THREADS);
       stage_row128(stg, r, 0, w);
       fence_proxy_async_smem();
-      named_bar_sync(1, NUM_EPI_THREADS);
-      if (epi_tid == 0) {
+      named_bar_sync(wg_bar, EPI_WG_THREADS);
+      if (wtid == 0) {
         if (issue) {
           if (reduce)
             tma_reduce_add_2d(map, smem_addr(stg), x, y);
@@ -657,7 +684,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         }
         bulk_commit_group();
       }
-      ++nstore;
     };
 
     for (int it = 0;; ++it) {
@@ -698,54 +724,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       const uint32_t t_acc = lane_base + static_cast<uint32_t>(acc * BN);
 
       if (MODE == kModeFwd) {
+        // (m, s) of this warpgroup's 128 columns: one partial per half tile
         FwdRowState st{-INFINITY, 0.f, 0.f, false};
         uint32_t za[32], zb[32];
-        tmem_ld32(t_acc, za);
+        tmem_ld32(t_acc + c0 * 32, za);
         tmem_wait_ld(za);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; c += 2) {
+        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           fwd_chunk(g, za, c * 32, vglob0, vlim, yl, st);
           tmem_wait_ld(zb);
-          if (c + 2 < BN / 32) tmem_ld32(t_acc + (c + 2) * 32, za);
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
           fwd_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          if (c + 2 < BN / 32) tmem_wait_ld(za);
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_on_leader(&tempty[acc]);
         if (valid) {
-          g.part[static_cast<size_t>(row) * g.part_ld + un.n0 / BN] = make_float2(st.m, st.s);
+          g.part[static_cast<size_t>(row) * g.part_ld + (un.n0 / BN) * NUM_EPI_WG + wg] =
+              make_float2(st.m, st.s);
           if (st.have_tgt) g.tgt[row] = st.tgt;
         }
       } else if (MODE == kModeBwd && un.cls == kClsGrad) {
         uint32_t za[32], zb[32];
-        tmem_ld32(t_acc, za);
+        tmem_ld32(t_acc + c0 * 32, za);
         tmem_wait_ld(za);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; c += 2) {
+        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
           // chunks c, c+1 form one 64-column box of the 16-bit panel
-          uint8_t* stg = sStg + (nstore & 1u) * STG_BYTES;
-          if (epi_tid == 0) bulk_wait_group_read<1>();
-          named_bar_sync(1, NUM_EPI_THREADS);
+          if (wtid == 0) bulk_wait_group_read<0>();  // the previous box has left the buffer
+          named_bar_sync(wg_bar, EPI_WG_THREADS);
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
           grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row, pk);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
-          if (c + 2 < BN / 32) tmem_ld32(t_acc + (c + 2) * 32, za);
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
           grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row,
                      pk);
           stage_row128(stg, r, 4, pk);
-          if (c + 2 < BN / 32) tmem_wait_ld(za);
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
           fence_proxy_async_smem();
-          named_bar_sync(1, NUM_EPI_THREADS);
-          if (epi_tid == 0) {
+          named_bar_sync(wg_bar, EPI_WG_THREADS);
+          if (wtid == 0) {
             // a box that starts past the panel's last column holds only padding
             if (un.n0 + c * 32 < g.w_g) tma_store_2d(&g.tmG, smem_addr(stg), un.n0 + c * 32, tm0);
             bulk_commit_group();
           }
-          ++nstore;
         }
         tc_fence_before();
         __syncwarp();
@@ -759,14 +785,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         const bool zero = (un.nk == 0);
         // a dW half that starts past the panel's last row has nothing to store
         const bool issue = !is_dw || tm0 < g.w_wh;
-        const int nch = min(BN / 32, cdiv_i(g.D - un.n0, 32));
+        // this warpgroup's chunks [c0, ce) of the ones inside D
+        const int ce = min(c0 + EPI_CHUNKS, cdiv_i(g.D - un.n0, 32));
+        const int nch = ce;
         uint32_t za[32], zb[32], w[32];
-        if (!zero) {
-          tmem_ld32(t_acc, za);
+        if (!zero && c0 < ce) {
+          tmem_ld32(t_acc + c0 * 32, za);
           tmem_wait_ld(za);
         }
 #pragma unroll 1
-        for (int c = 0; c < nch; c += 2) {
+        for (int c = c0; c < ce; c += 2) {
           // za holds chunk c; chunk c+1 loads into zb meanwhile
           if (!zero && c + 1 < nch) tmem_ld32(t_acc + (c + 1) * 32, zb);
 #pragma unroll
@@ -788,17 +816,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else {  // kModePlain
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int c0 = un.n0 + c * 32;
-          if (c0 >= g.ncols) break;
+        for (int c = c0; c < c0 + EPI_CHUNKS; ++c) {
+          const int col0 = un.n0 + c * 32;
+          if (col0 >= g.ncols) break;
           uint32_t z[32];
           tmem_ld32(t_acc + c * 32, z);
           tmem_wait_ld(z);
           if (valid) {
-            float* dst = g.out + static_cast<size_t>(row) * g.ncols + c0;
+            float* dst = g.out + static_cast<size_t>(row) * g.ncols + col0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (c0 + j < g.ncols) dst[j] = __uint_as_float(z[j]) * g.scale;
+              if (col0 + j < g.ncols) dst[j] = __uint_as_float(z[j]) * g.scale;
           }
         }
         tc_fence_before();
@@ -810,7 +838,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         acc_phase ^= 1u;
       }
     }
-    if (MODE == kModeBwd && epi_tid == 0) bulk_wait_group<0>();
+    if (MODE == kModeBwd && wtid == 0) bulk_wait_group<0>();
   }
 
   // Neither CTA frees its TMEM (or exits) while the pair still uses it.

@@ -59,6 +59,13 @@ SPECS = {
                           bias_std=0.01, ignore_frac=0.10, mask_false_frac=0.05, lam=0.5),
     "packed": WorkloadSpec("packed", 3, N=16384, D=1024, V=248320, dtype="bf16", w_std=0.02,
                            label_dist="zipf", segments=8, prefix_frac=0.3),
+    # the packed recipe at the two smaller hidden sizes the method is compared on
+    # (w_std scaled by sqrt(1024 / D) so that the logits keep the same spread)
+    "packed_d256": WorkloadSpec("packed_d256", 5, N=16384, D=256, V=248320, dtype="bf16",
+                                w_std=0.04, label_dist="zipf", segments=8, prefix_frac=0.3),
+    "packed_d512": WorkloadSpec("packed_d512", 6, N=16384, D=512, V=248320, dtype="bf16",
+                                w_std=0.02 * 2 ** 0.5, label_dist="zipf", segments=8,
+                                prefix_frac=0.3),
     "stress": WorkloadSpec("stress", 4, N=32768, D=4096, V=248320, dtype="bf16", w_std=0.02,
                            h_scale=4.0, big_row_frac=0.01, big_row_scale=50.0,
                            ignore_frac=0.5),
