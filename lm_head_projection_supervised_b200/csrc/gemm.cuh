@@ -343,9 +343,15 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
     for (int j = 0; j < 32; ++j)
       if (cb + j >= vlim) x[j] = -INFINITY;
   }
-  float cm = x[0];
+  // chunk max as a tree (depth 5 instead of a chain of 31)
+  float t[16];
 #pragma unroll
-  for (int j = 1; j < 32; ++j) cm = fmaxf(cm, x[j]);
+  for (int j = 0; j < 16; ++j) t[j] = fmaxf(x[j], x[j + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+  const float cm = t[0];
   const float mn = fmaxf(st.m, cm);
   // nothing seen yet and this chunk is all padding (a half tile past V): the
   // state stays (-inf, 0) instead of exp(-inf + inf)
@@ -536,110 +542,110 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   const UnitSpace us = make_unit_space<MODE>(g, C);
 
   if (warp < EPI_WARP0) {
-  setmaxnreg_dec<kRegsLow>();  // the whole first warpgroup
-  if (warp == 0) {
-    // ------------------------------------------------------------ scheduler + producer
-    if (lane == 0) {
-      uint32_t n_issued = 0;
-      bool ok = true;
-      const uint32_t full_c0 = leader_addr(&full[0]);
-      for (int it = 0; ok; ++it) {
-        const int slot = it % UQ;
-        const uint32_t ph = (it / UQ) & 1;
-        int u;
-        if (leader) {
-          if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
-          u = atomicAdd(g.counter, 1);
-          if (u >= us.total) u = -1;
-          s_unit[slot] = u;
-          st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<int*>(&s_unit[slot])), 1),
-                                static_cast<uint32_t>(u));
-          mbar_arrive(&uq_full[slot]);
-          mbar_arrive_cluster(mapa_shared(smem_addr(&uq_full[slot]), 1));
-        } else {
-          if (!mbar_wait_cluster(&uq_full[slot], ph, abort_flag, g.err)) break;
-          u = s_unit[slot];
-          arrive_on_leader(&uq_empty[slot]);
-        }
-        if (u < 0) break;
-        const Unit un = decode_unit<MODE>(g, us, C, u);
-        for (int kb = 0; kb < un.nk; ++kb) {
-          const uint32_t stage = n_issued % STAGES;
-          const uint32_t phase = (n_issued / STAGES) & 1u;
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, g.err)) {
-            ok = false;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
-          issue_stage_loads<MODE>(g, un, kb, rank, smem_addr(sA + stage * A_STAGE_BYTES),
-                                  smem_addr(sB + stage * B_STAGE_BYTES),
-                                  full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)));
-          ++n_issued;
-        }
-      }
-      // The even CTA lets every copy still in flight (its own and its peer's)
-      // land before the pair can exit.
-      if (leader) {
-        const uint32_t first = n_issued > STAGES ? n_issued - STAGES : 0u;
-        for (uint32_t i = first; i < n_issued; ++i)
-          mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, nullptr, nullptr, kDrainLimitNs);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (lane == 0 && leader) {
-      uint32_t n_used = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      for (int it = 0;; ++it) {
-        const int slot = it % UQ;
-        if (!mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err)) break;
-        const int u = s_unit[slot];
-        mbar_arrive(&uq_empty[slot]);
-        if (u < 0) break;
-        const Unit un = decode_unit<MODE>(g, us, C, u);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, g.err)) break;
-        tc_fence_after();
-        const bool a_mn = unit_a_mn<MODE>(g, un);
-        const bool b_mn = unit_b_mn<MODE>(g, un);
-        const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, PAIR_M, BN);
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        const uint32_t a_lbo = a_mn ? MN_BOX_BYTES : 16u;
-        const uint32_t b_lbo = b_mn ? MN_BOX_BYTES : 16u;
-        const uint32_t a_step = a_mn ? 16u * 128u : 32u;  // bytes per K=16 slice
-        const uint32_t b_step = b_mn ? 16u * 128u : 32u;
+    setmaxnreg_dec<kRegsLow>();  // the whole first warpgroup
+    if (warp == 0) {
+      // ------------------------------------------------------------ scheduler + producer
+      if (lane == 0) {
+        uint32_t n_issued = 0;
         bool ok = true;
-        for (int kb = 0; kb < un.nk; ++kb) {
-          const uint32_t stage = n_used % STAGES;
-          const uint32_t phase = (n_used / STAGES) & 1u;
-          if (!mbar_wait(&full[stage], phase, abort_flag, g.err)) {
-            ok = false;
-            break;
+        const uint32_t full_c0 = leader_addr(&full[0]);
+        for (int it = 0; ok; ++it) {
+          const int slot = it % UQ;
+          const uint32_t ph = (it / UQ) & 1;
+          int u;
+          if (leader) {
+            if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
+            u = atomicAdd(g.counter, 1);
+            if (u >= us.total) u = -1;
+            s_unit[slot] = u;
+            st_shared_cluster_u32(mapa_shared(smem_addr(const_cast<int*>(&s_unit[slot])), 1),
+                                  static_cast<uint32_t>(u));
+            mbar_arrive(&uq_full[slot]);
+            mbar_arrive_cluster(mapa_shared(smem_addr(&uq_full[slot]), 1));
+          } else {
+            if (!mbar_wait_cluster(&uq_full[slot], ph, abort_flag, g.err)) break;
+            u = s_unit[slot];
+            arrive_on_leader(&uq_empty[slot]);
           }
-          tc_fence_after();
-          const uint32_t sa = smem_addr(sA + stage * A_STAGE_BYTES);
-          const uint32_t sb = smem_addr(sB + stage * B_STAGE_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024u);
-            const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024u);
-            umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          if (u < 0) break;
+          const Unit un = decode_unit<MODE>(g, us, C, u);
+          for (int kb = 0; kb < un.nk; ++kb) {
+            const uint32_t stage = n_issued % STAGES;
+            const uint32_t phase = (n_issued / STAGES) & 1u;
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, g.err)) {
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
+            issue_stage_loads<MODE>(g, un, kb, rank, smem_addr(sA + stage * A_STAGE_BYTES),
+                                    smem_addr(sB + stage * B_STAGE_BYTES),
+                                    full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)));
+            ++n_issued;
           }
-          umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
-          ++n_used;
         }
-        if (!ok) break;
-        umma_commit_pair_mc(&tfull[acc], 0x3);  // accumulator ready in both CTAs
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        // The even CTA lets every copy still in flight (its own and its peer's)
+        // land before the pair can exit.
+        if (leader) {
+          const uint32_t first = n_issued > STAGES ? n_issued - STAGES : 0u;
+          for (uint32_t i = first; i < n_issued; ++i)
+            mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, nullptr, nullptr, kDrainLimitNs);
         }
       }
-      // All pair MMAs complete before either CTA releases its TMEM.
-      umma_commit_pair_mc(done_bar, 0x1);
-      mbar_wait(done_bar, 0, nullptr, nullptr, kDrainLimitNs);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer (even CTA)
+      if (lane == 0 && leader) {
+        uint32_t n_used = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int it = 0;; ++it) {
+          const int slot = it % UQ;
+          if (!mbar_wait(&uq_full[slot], (it / UQ) & 1, abort_flag, g.err)) break;
+          const int u = s_unit[slot];
+          mbar_arrive(&uq_empty[slot]);
+          if (u < 0) break;
+          const Unit un = decode_unit<MODE>(g, us, C, u);
+          if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, g.err)) break;
+          tc_fence_after();
+          const bool a_mn = unit_a_mn<MODE>(g, un);
+          const bool b_mn = unit_b_mn<MODE>(g, un);
+          const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, PAIR_M, BN);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+          const uint32_t a_lbo = a_mn ? MN_BOX_BYTES : 16u;
+          const uint32_t b_lbo = b_mn ? MN_BOX_BYTES : 16u;
+          const uint32_t a_step = a_mn ? 16u * 128u : 32u;  // bytes per K=16 slice
+          const uint32_t b_step = b_mn ? 16u * 128u : 32u;
+          bool ok = true;
+          for (int kb = 0; kb < un.nk; ++kb) {
+            const uint32_t stage = n_used % STAGES;
+            const uint32_t phase = (n_used / STAGES) & 1u;
+            if (!mbar_wait(&full[stage], phase, abort_flag, g.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_addr(sA + stage * A_STAGE_BYTES);
+            const uint32_t sb = smem_addr(sB + stage * B_STAGE_BYTES);
+  #pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024u);
+              const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024u);
+              umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+            ++n_used;
+          }
+          if (!ok) break;
+          umma_commit_pair_mc(&tfull[acc], 0x3);  // accumulator ready in both CTAs
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
+        // All pair MMAs complete before either CTA releases its TMEM.
+        umma_commit_pair_mc(done_bar, 0x1);
+        mbar_wait(done_bar, 0, nullptr, nullptr, kDrainLimitNs);
+      }
     }
-  }
   } else {
     setmaxnreg_inc<kRegsHigh>();  // each epilogue warpgroup
     // ------------------------------------------------------------ epilogue
