@@ -241,22 +241,34 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
 // TMA loads of k-block kb of unit `un` into this CTA's ring stage: its 128
 // A rows (16 KiB) and its 128 of the 256 B rows (16 KiB).  Completion is
 // counted on the even CTA's barrier `bar_cluster`.
+// Which operand boxes a producer thread issues: the backward splits A and B
+// between two threads, because issuing a stage's 2-4 boxes from one thread
+// takes about as long as the stage's MMAs.
+enum LoadPart : int { kLoadA = 0, kLoadB = 1, kLoadAB = 2 };
+template <int MODE>
+struct LoadSplit {
+  static constexpr bool kSplit = MODE == kModeBwd;
+};
+
 template <int MODE>
 __device__ __forceinline__ void issue_stage_loads(const GemmArgs& g, const Unit& un, int kb,
                                                   uint32_t rank, uint32_t sa, uint32_t sb,
-                                                  uint32_t bar_cluster) {
+                                                  uint32_t bar_cluster, int part) {
   const int mapi = (MODE == kModeBwd) ? un.cls : 0;
   const CUtensorMap* tA = &g.tmA[mapi];
   const CUtensorMap* tB = &g.tmB[mapi];
   const int k0 = kb * BK;
   const int am0 = un.m0 + static_cast<int>(rank) * BM;       // this CTA's A rows
   const int bn0 = un.n0 + static_cast<int>(rank) * BN_HALF;  // this CTA's B rows
-  if (unit_a_mn<MODE>(g, un)) {
-    tma_load_2d_pair(sa, tA, bar_cluster, am0, k0);
-    tma_load_2d_pair(sa + MN_BOX_BYTES, tA, bar_cluster, am0 + 64, k0);
-  } else {
-    tma_load_2d_pair(sa, tA, bar_cluster, k0, am0);
+  if (part != kLoadB) {
+    if (unit_a_mn<MODE>(g, un)) {
+      tma_load_2d_pair(sa, tA, bar_cluster, am0, k0);
+      tma_load_2d_pair(sa + MN_BOX_BYTES, tA, bar_cluster, am0 + 64, k0);
+    } else {
+      tma_load_2d_pair(sa, tA, bar_cluster, k0, am0);
+    }
   }
+  if (part == kLoadA) return;
   if (unit_b_mn<MODE>(g, un)) {
     // dH: the k index is a vocabulary id of the panel
     const int kB = (MODE == kModeBwd && un.cls == kClsDH) ? g.vp_wh + k0 : k0;
@@ -508,7 +520,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     for (int q = 0; q < UQ; ++q) {
       mbar_init(&uq_full[q], 1);
       // even CTA: its MMA lane and epilogue warps; odd CTA: its producer and epilogue warps
-      mbar_init(&uq_empty[q], 2 * (1 + NUM_EPI_THREADS / 32));
+      // + the second producer of each CTA when the loads are split
+      mbar_init(&uq_empty[q], 2 * (1 + NUM_EPI_THREADS / 32) + (LoadSplit<MODE>::kSplit ? 2 : 0));
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -543,8 +556,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 
   if (warp < EPI_WARP0) {
     setmaxnreg_dec<kRegsLow>();  // the whole first warpgroup
-    if (warp == 0) {
-      // ------------------------------------------------------------ scheduler + producer
+    if (warp == 0 || (LoadSplit<MODE>::kSplit && warp == 2)) {
+      // ------------------------------------------------------------ scheduler + producers
+      // warp 0: the scheduler (even CTA) and the A loads (all loads when not split);
+      // warp 2: the B loads when split
+      const int part = !LoadSplit<MODE>::kSplit ? kLoadAB : (warp == 0 ? kLoadA : kLoadB);
+      const bool scheduler = leader && warp == 0;
       if (lane == 0) {
         uint32_t n_issued = 0;
         bool ok = true;
@@ -553,7 +570,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           const int slot = it % UQ;
           const uint32_t ph = (it / UQ) & 1;
           int u;
-          if (leader) {
+          if (scheduler) {
             if (!mbar_wait(&uq_empty[slot], ph ^ 1u, abort_flag, g.err)) break;
             u = atomicAdd(g.counter, 1);
             if (u >= us.total) u = -1;
@@ -563,7 +580,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             mbar_arrive(&uq_full[slot]);
             mbar_arrive_cluster(mapa_shared(smem_addr(&uq_full[slot]), 1));
           } else {
-            if (!mbar_wait_cluster(&uq_full[slot], ph, abort_flag, g.err)) break;
+            const bool got = leader ? mbar_wait(&uq_full[slot], ph, abort_flag, g.err)
+                                    : mbar_wait_cluster(&uq_full[slot], ph, abort_flag, g.err);
+            if (!got) break;
             u = s_unit[slot];
             arrive_on_leader(&uq_empty[slot]);
           }
@@ -576,16 +595,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
               ok = false;
               break;
             }
-            if (leader) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
+            // one arrival (with both CTAs' bytes) per stage, from the scheduler
+            if (scheduler) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
             issue_stage_loads<MODE>(g, un, kb, rank, smem_addr(sA + stage * A_STAGE_BYTES),
                                     smem_addr(sB + stage * B_STAGE_BYTES),
-                                    full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)));
+                                    full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)),
+                                    part);
             ++n_issued;
           }
         }
-        // The even CTA lets every copy still in flight (its own and its peer's)
-        // land before the pair can exit.
-        if (leader) {
+        // The even CTA lets every copy still in flight (its own and its peer's,
+        // both producers') land before the pair can exit.
+        if (scheduler) {
           const uint32_t first = n_issued > STAGES ? n_issued - STAGES : 0u;
           for (uint32_t i = first; i < n_issued; ++i)
             mbar_wait(&full[i % STAGES], (i / STAGES) & 1u, nullptr, nullptr, kDrainLimitNs);
