@@ -186,7 +186,7 @@ def test_autograd_wrapper_matches_abi():
 # --------------------------------------------------------------------------
 # full-size workloads, as the benchmark launches them
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("name", ["page2", "packed"])
+@pytest.mark.parametrize("name", ["page2", "packed", "packed_d256", "packed_d512"])
 def test_full_size_sampled(name):
     inp = wl.make_inputs(name)
     got = run_gpu(inp)
