@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     if (leader)
       mbar_arrive(bar);
     else
-      mbar_arrive_cluster(mapa_shared(smem_addr(bar), 0));
+      mbar_arrive_cluster_release_cta(mapa_shared(smem_addr(bar), 0));
   };
 
   if (threadIdx.x == 0) {

@@ -111,6 +111,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+// Consumer release on a peer CTA's barrier (an accumulator or a unit slot is
+// free again): the default semantics, release at CTA scope.  The data it
+// hands back is ordered by the tcgen05 fences and the waits before it, and
+// unlike the cluster-scope form it does not wait for this thread's earlier
+// global stores (the forward's per-row partials) to be performed.
+__device__ __forceinline__ void mbar_arrive_cluster_release_cta(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
