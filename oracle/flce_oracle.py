@@ -30,7 +30,7 @@ the recurrence against the dense definition (§02: exact in the reals) and to
 plant the two fault modes that §04 names, so that the tests can show they are
 caught.
 
-Readings where the pages are silent (each is listed in the design notes):
+Readings where the pages are silent:
   * m and log s of a row with a_i = 0 are the recurrence's initial state:
     m = -inf, s = 0, so log s = -inf.
   * Z is not rounded to the input dtype; it is exact (float64 here).
