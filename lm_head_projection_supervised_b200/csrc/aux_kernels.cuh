@@ -20,16 +20,20 @@ __device__ __forceinline__ bool is_supervised(const int64_t* labels, const uint8
 
 // a_i = 1[mask_i] 1[y_i != ignore]; idx = supervised rows ascending (stable),
 // y_c = their labels (optional), C = count ("分块交叉熵" page §01; the supervised-row
-// filter of "ChunkedLinearCrossEntropy").  One block: each thread scans a
-// contiguous slice, a block-wide exclusive scan of the slice counts gives
-// every thread its output offset.  Labels outside [0, V) on supervised rows
-// set the label error bit and are clamped to 0 so later indexing stays in
-// range.  y_c holds y - v0, the label's column in the vocabulary slice
-// [v0, v0 + V_slice) (the whole vocabulary unsharded), or kNoColumn when
-// another slice holds it, so that no column of this slice ever matches it.
-// Unsupervised rows get m = log s = -inf when m_out is given.
+// filter of "ChunkedLinearCrossEntropy").  One block walks the rows in
+// batches of COMPACT_BATCH chunks of COMPACT_THREADS consecutive rows (thread t
+// takes row base + k * COMPACT_THREADS + t, so loads are coalesced and a batch's
+// loads are all in flight at once); within a chunk a warp ballot and a scan of
+// the 32 warp counts give each supervised row its output slot, chunks follow
+// one another, so the order is ascending.  Labels outside [0, V) on
+// supervised rows set the label error bit and are clamped to 0 so later
+// indexing stays in range.  y_c holds y - v0, the label's column in the
+// vocabulary slice [v0, v0 + V_slice) (the whole vocabulary unsharded), or
+// kNoColumn when another slice holds it, so that no column of this slice ever
+// matches it.  Unsupervised rows get m = log s = -inf when m_out is given.
 // pos (optional) is the inverse map: pos[i] = compact row of i, or -1.
 // lossvec (optional) gets 0 on unsupervised rows (per-row loss output).
+constexpr int COMPACT_BATCH = 4;
 __global__ void __launch_bounds__(COMPACT_THREADS)
     compact_kernel(const int64_t* __restrict__ labels, const uint8_t* __restrict__ mask,
                    int64_t ignore, int64_t N, int64_t V, int64_t v0, int64_t V_slice,
@@ -37,58 +41,73 @@ __global__ void __launch_bounds__(COMPACT_THREADS)
                    int* __restrict__ y_c, int* __restrict__ C_out, uint32_t* err,
                    float* __restrict__ m_out, float* __restrict__ logs_out,
                    int* __restrict__ pos, float* __restrict__ lossvec) {
-  __shared__ int warp_tot[COMPACT_THREADS / 32];
+  constexpr int NW = COMPACT_THREADS / 32;
+  static_assert(NW == 32 && COMPACT_BATCH <= NW, "one scanning warp per chunk of the batch");
+  __shared__ int warp_cnt[COMPACT_BATCH][NW];
+  __shared__ int warp_off[COMPACT_BATCH][NW];
+  __shared__ int chunk_tot[COMPACT_BATCH];
   const int t = threadIdx.x;
-  const int64_t per = (N + COMPACT_THREADS - 1) / COMPACT_THREADS;
-  const int64_t beg = min(N, t * per);
-  const int64_t end = min(N, beg + per);
-  int cnt = 0;
-  for (int64_t i = beg; i < end; ++i) cnt += is_supervised(labels, mask, ignore, i) ? 1 : 0;
-  // block exclusive scan of cnt
   const int lane = t & 31, warp = t >> 5;
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_tot[lane];
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += v;
-    }
-    warp_tot[lane] = wi - w;  // exclusive warp offsets
-    if (lane == 31) *C_out = wi;
-  }
-  __syncthreads();
-  int off = warp_tot[warp] + incl - cnt;
+  const unsigned lanes_below = (1u << lane) - 1u;
+  int running = 0;  // rows written by the previous batches (the same in every thread)
   bool bad = false;
-  for (int64_t i = beg; i < end; ++i) {
-    if (is_supervised(labels, mask, ignore, i)) {
-      int64_t y = labels[i];
-      if (y < 0 || y >= V) {
-        bad = true;
-        y = 0;
-      }
-      idx[off] = static_cast<int>(i);
-      if (y_c != nullptr)
-        y_c[off] = (y >= v0 && y < v0 + V_slice) ? static_cast<int>(y - v0) : kNoColumn;
-      if (pos != nullptr) pos[i] = off;
-      ++off;
-    } else {
-      if (m_out != nullptr) {
-        m_out[i] = -INFINITY;
-        logs_out[i] = -INFINITY;
-      }
-      if (pos != nullptr) pos[i] = -1;
-      if (lossvec != nullptr) lossvec[i] = 0.f;
+  for (int64_t base = 0; base < N; base += static_cast<int64_t>(COMPACT_THREADS) * COMPACT_BATCH) {
+    int64_t y[COMPACT_BATCH];
+    bool sup[COMPACT_BATCH];
+    unsigned bal[COMPACT_BATCH];
+#pragma unroll
+    for (int k = 0; k < COMPACT_BATCH; ++k) {
+      const int64_t i = base + static_cast<int64_t>(k) * COMPACT_THREADS + t;
+      sup[k] = i < N && is_supervised(labels, mask, ignore, i);
+      y[k] = sup[k] ? labels[i] : 0;
     }
+#pragma unroll
+    for (int k = 0; k < COMPACT_BATCH; ++k) {
+      bal[k] = __ballot_sync(0xffffffffu, sup[k]);
+      if (lane == 0) warp_cnt[k][warp] = __popc(bal[k]);
+    }
+    __syncthreads();
+    if (warp < COMPACT_BATCH) {  // warp k: exclusive scan of chunk k's warp counts
+      const int c = warp_cnt[warp][lane];
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      warp_off[warp][lane] = incl - c;
+      if (lane == 31) chunk_tot[warp] = incl;
+    }
+    __syncthreads();
+    int off = running;
+#pragma unroll
+    for (int k = 0; k < COMPACT_BATCH; ++k) {
+      const int64_t i = base + static_cast<int64_t>(k) * COMPACT_THREADS + t;
+      if (sup[k]) {
+        const int o = off + warp_off[k][warp] + __popc(bal[k] & lanes_below);
+        int64_t yy = y[k];
+        if (yy < 0 || yy >= V) {
+          bad = true;
+          yy = 0;
+        }
+        idx[o] = static_cast<int>(i);
+        if (y_c != nullptr)
+          y_c[o] = (yy >= v0 && yy < v0 + V_slice) ? static_cast<int>(yy - v0) : kNoColumn;
+        if (pos != nullptr) pos[i] = o;
+      } else if (i < N) {
+        if (m_out != nullptr) {
+          m_out[i] = -INFINITY;
+          logs_out[i] = -INFINITY;
+        }
+        if (pos != nullptr) pos[i] = -1;
+        if (lossvec != nullptr) lossvec[i] = 0.f;
+      }
+      off += chunk_tot[k];
+    }
+    running = off;
+    __syncthreads();  // the next batch reuses warp_cnt / warp_off / chunk_tot
   }
+  if (t == 0) *C_out = running;
   if (bad) atomicOr(err, kErrBitLabel);
 }
 
