@@ -325,12 +325,15 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) *scal = S;
 }
 
-// db[vp + j] = (S / sigma) * sum_{i < C} Gp[i][j] for the panel's columns, in a
-// fixed order: 8 row groups per block, combined in group order.
+// db[vp + j] = (S / sigma) * sum_{i < C} (Gp[i][j] + [y_i = vp + j] e_i) for the
+// panel's columns, in a fixed order: 8 row groups per block, combined in
+// group order.  e_i is what the 16-bit rounding took off row i's target entry
+// (recorded by the gradient units), so the target terms enter db exactly.
 __global__ void __launch_bounds__(256)
     bias_grad_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
                      const int* __restrict__ C_dev, const float* __restrict__ scal,
-                     float inv_sigma, int is_bf16, int vp, float* __restrict__ db) {
+                     float inv_sigma, int is_bf16, int vp, const int* __restrict__ y_c,
+                     const float* __restrict__ tgt_resid, float* __restrict__ db) {
   __shared__ float2 part[8][32];
   const int C = *C_dev;
   const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
@@ -339,15 +342,20 @@ __global__ void __launch_bounds__(256)
   if (j < w) {
     for (int i = grp; i < C; i += 8) {
       const uint32_t v = *reinterpret_cast<const uint32_t*>(Gp + static_cast<int64_t>(i) * ldg + j);
+      float gx, gy;
       if (is_bf16) {
-        acc.x += __uint_as_float((v & 0xFFFFu) << 16);
-        acc.y += __uint_as_float(v & 0xFFFF0000u);
+        gx = __uint_as_float((v & 0xFFFFu) << 16);
+        gy = __uint_as_float(v & 0xFFFF0000u);
       } else {
-        const __half2 h = *reinterpret_cast<const __half2*>(&v);
-        const float2 f = __half22float2(h);
-        acc.x += f.x;
-        acc.y += f.y;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+        gx = f.x;
+        gy = f.y;
       }
+      const int yc = __ldg(y_c + i) - vp;  // the row's label as a column of this panel
+      if (yc == j) gx += __ldg(tgt_resid + i);
+      if (yc == j + 1) gy += __ldg(tgt_resid + i);
+      acc.x += gx;
+      acc.y += gy;
     }
   }
   part[grp][lane] = acc;
@@ -422,6 +430,89 @@ __global__ void scatter_dh_kernel(const float4* __restrict__ dHc, const int* __r
   } else if (!accumulate) {
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int64_t k = lane; k < vec_per_row; k += 32) dst[k] = z;
+  }
+}
+
+// Sort keys for grouping the supervised rows by label: key = the row's label
+// as a column of this vocabulary slice, or V_slice (sorts last, ignored) for
+// padding rows and labels another slice holds; value = the compact row.
+__global__ void label_sort_prep_kernel(const int* __restrict__ C_dev, const int* __restrict__ y_c,
+                                       int64_t Np, int V_slice, uint32_t* __restrict__ keys,
+                                       int* __restrict__ vals) {
+  const int C = *C_dev;
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < Np;
+       k += static_cast<int64_t>(blockDim.x) * gridDim.x) {
+    const int y = k < C ? y_c[k] : -1;
+    keys[k] = (y >= 0 && y < V_slice) ? static_cast<uint32_t>(y) : static_cast<uint32_t>(V_slice);
+    vals[k] = static_cast<int>(k);
+  }
+}
+
+// dW[v] += (S / sigma) sum_{k: y_k = v} e_k H_c[k], over the rows grouped by
+// label (keys sorted stably, so each group's rows are in ascending order):
+// the fp32 residuals of the 16-bit target entries (see scatter_dh_kernel),
+// added once per label after every panel's dW is written.  One warp per
+// (group start, 128-column chunk): a lane owns 4 columns; the group's row
+// ids and residuals are read 32 at a time and broadcast by shuffles, so the
+// H loads of consecutive rows are independent.  Fixed order: deterministic.
+__global__ void dw_target_resid_kernel(const uint32_t* __restrict__ keys,
+                                       const int* __restrict__ rows, int64_t Np, int V_slice,
+                                       const uint2* __restrict__ Hc, int64_t vec_per_row,
+                                       int is_bf16, const float* __restrict__ tgt_resid,
+                                       const float* __restrict__ scal, float inv_sigma,
+                                       float4* __restrict__ dW) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nchunk = (vec_per_row + 31) / 32;
+  const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
+  const float scale = (*scal) * inv_sigma;
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < Np * nchunk; w += warps) {
+    const int64_t p = w / nchunk;
+    const int64_t c = (w % nchunk) * 32 + lane;  // this lane's 4-column group
+    const uint32_t v = keys[p];
+    if (v >= static_cast<uint32_t>(V_slice) || (p > 0 && keys[p - 1] == v)) continue;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int64_t q0 = p;; q0 += 32) {
+      // up to 32 rows of the group: row id and residual in lane order
+      const int64_t q = q0 + lane;
+      const bool in = q < Np && keys[q] == v;
+      const int k = in ? rows[q] : 0;
+      const float e = in ? tgt_resid[k] : 0.f;
+      const unsigned live = __ballot_sync(0xffffffffu, in);
+      const int n = __popc(live);  // the group's rows are contiguous from q0
+      for (int j = 0; j < n; ++j) {
+        const int kj = __shfl_sync(0xffffffffu, k, j);
+        const float ej = __shfl_sync(0xffffffffu, e, j);
+        if (c < vec_per_row) {
+          const uint2 hv = __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c);
+          float h0, h1, h2, h3;
+          if (is_bf16) {
+            h0 = __uint_as_float(hv.x << 16);
+            h1 = __uint_as_float(hv.x & 0xFFFF0000u);
+            h2 = __uint_as_float(hv.y << 16);
+            h3 = __uint_as_float(hv.y & 0xFFFF0000u);
+          } else {
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+            h0 = lo.x;
+            h1 = lo.y;
+            h2 = hi.x;
+            h3 = hi.y;
+          }
+          a0 = fmaf(ej, h0, a0);
+          a1 = fmaf(ej, h1, a1);
+          a2 = fmaf(ej, h2, a2);
+          a3 = fmaf(ej, h3, a3);
+        }
+      }
+      if (n < 32) break;
+    }
+    if (c < vec_per_row) {
+      float4* dst = dW + static_cast<int64_t>(v) * vec_per_row + c;
+      const float4 o = *dst;
+      *dst = make_float4(fmaf(scale, a0, o.x), fmaf(scale, a1, o.y), fmaf(scale, a2, o.z),
+                         fmaf(scale, a3, o.w));
+    }
   }
 }
 

@@ -16,6 +16,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cub/device/device_radix_sort.cuh>
+
 #include "../../include/flce.h"
 #include "../../include/flce_diag.h"
 #include "aux_kernels.cuh"
@@ -41,7 +43,7 @@ int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, rs, resid, dhc, gpanel[2], total;
+  size_t pos, rs, resid, skeys[2], svals[2], cubtmp, cub_bytes, dhc, gpanel[2], total;
   int64_t Np, nvt, nparts, vc, gld, panels;
 };
 
@@ -75,6 +77,13 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.fwd_total = off;
   L.rs = take(static_cast<size_t>(L.Np) * 4);
   L.resid = take(static_cast<size_t>(L.Np) * 4);
+  // rows grouped by label (stable radix sort, ping-pong buffers + CUB's scratch)
+  for (int i = 0; i < 2; ++i) {
+    L.skeys[i] = take(static_cast<size_t>(L.Np) * 4);
+    L.svals[i] = take(static_cast<size_t>(L.Np) * 4);
+  }
+  L.cub_bytes = static_cast<size_t>(L.Np) * 4 + (size_t(4) << 20);
+  L.cubtmp = take(L.cub_bytes);
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
   L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.gld * 2);
   L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.gld * 2);
@@ -290,6 +299,9 @@ struct WsPtrs {
   float* loss_rows;
   float* rs;
   float* resid;
+  uint32_t* skeys[2];
+  int* svals[2];
+  void* cubtmp;
   float* dhc;
   uint16_t* gpanel[2];
 };
@@ -310,6 +322,11 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.loss_rows = reinterpret_cast<float*>(w + L.loss_rows);
   p.rs = reinterpret_cast<float*>(w + L.rs);
   p.resid = reinterpret_cast<float*>(w + L.resid);
+  for (int i = 0; i < 2; ++i) {
+    p.skeys[i] = reinterpret_cast<uint32_t*>(w + L.skeys[i]);
+    p.svals[i] = reinterpret_cast<int*>(w + L.svals[i]);
+  }
+  p.cubtmp = w + L.cubtmp;
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
   p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
   p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
@@ -545,11 +562,38 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       FLCE_CK(timed_launch(kProfAux, s, [&] {
         bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w_g, 64)), 256, 0, s>>>(
             gp, L.gld, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma, bf16 ? 1 : 0,
-            static_cast<int>(vp_g), db);
+            static_cast<int>(vp_g), p.yc, p.resid, db);
       }));
     }
   }
   if (N > 0) {
+    // dW's target terms in fp32: group the rows by label (stable sort), then
+    // add each group's residuals times its H rows to the label's dW row
+    const int64_t pblocks = cdiv64(L.Np, 256) < 4LL * di.sms ? cdiv64(L.Np, 256) : 4LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      label_sort_prep_kernel<<<static_cast<unsigned>(pblocks), 256, 0, s>>>(
+          p.C, p.yc, L.Np, static_cast<int>(V), p.skeys[0], p.svals[0]);
+    }));
+    int end_bit = 1;
+    while ((int64_t(1) << end_bit) <= V) ++end_bit;  // keys are 0 .. V
+    cub::DoubleBuffer<uint32_t> dkeys(p.skeys[0], p.skeys[1]);
+    cub::DoubleBuffer<int> dvals(p.svals[0], p.svals[1]);
+    size_t need = 0;
+    FLCE_CK(cub::DeviceRadixSort::SortPairs(nullptr, need, dkeys, dvals, static_cast<int>(L.Np), 0,
+                                            end_bit, s));
+    if (need > L.cub_bytes) return FLCE_ERR_WORKSPACE;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      cub::DeviceRadixSort::SortPairs(p.cubtmp, need, dkeys, dvals, static_cast<int>(L.Np), 0,
+                                      end_bit, s);
+    }));
+    const int64_t rwarps = L.Np * cdiv64(D / 4, 32);
+    const int64_t rblocks = cdiv64(rwarps, 8) < 16LL * di.sms ? cdiv64(rwarps, 8) : 16LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      dw_target_resid_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+          dkeys.Current(), dvals.Current(), L.Np, static_cast<int>(V),
+          reinterpret_cast<const uint2*>(p.hc), D / 4, bf16 ? 1 : 0, p.resid, p.scal,
+          1.f / sigma, reinterpret_cast<float4*>(dW));
+    }));
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       scatter_dh_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
           reinterpret_cast<const float4*>(p.dhc), p.pos, N, D / 4, reinterpret_cast<float4*>(dH),
