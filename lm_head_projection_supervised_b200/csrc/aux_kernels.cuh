@@ -480,29 +480,39 @@ __global__ void dw_target_resid_kernel(const uint32_t* __restrict__ keys,
       const float e = in ? tgt_resid[k] : 0.f;
       const unsigned live = __ballot_sync(0xffffffffu, in);
       const int n = __popc(live);  // the group's rows are contiguous from q0
-      for (int j = 0; j < n; ++j) {
-        const int kj = __shfl_sync(0xffffffffu, k, j);
-        const float ej = __shfl_sync(0xffffffffu, e, j);
-        if (c < vec_per_row) {
-          const uint2 hv = __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c);
+      for (int j0 = 0; j0 < n; j0 += 16) {
+        // sixteen rows' loads in flight, then their terms in row order
+        uint2 hv[16];
+        float ej[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int kj = __shfl_sync(0xffffffffu, k, j0 + u);
+          ej[u] = __shfl_sync(0xffffffffu, e, j0 + u);
+          hv[u] = (j0 + u < n && c < vec_per_row)
+                      ? __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c)
+                      : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (j0 + u >= n) break;
           float h0, h1, h2, h3;
           if (is_bf16) {
-            h0 = __uint_as_float(hv.x << 16);
-            h1 = __uint_as_float(hv.x & 0xFFFF0000u);
-            h2 = __uint_as_float(hv.y << 16);
-            h3 = __uint_as_float(hv.y & 0xFFFF0000u);
+            h0 = __uint_as_float(hv[u].x << 16);
+            h1 = __uint_as_float(hv[u].x & 0xFFFF0000u);
+            h2 = __uint_as_float(hv[u].y << 16);
+            h3 = __uint_as_float(hv[u].y & 0xFFFF0000u);
           } else {
-            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
-            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].y));
             h0 = lo.x;
             h1 = lo.y;
             h2 = hi.x;
             h3 = hi.y;
           }
-          a0 = fmaf(ej, h0, a0);
-          a1 = fmaf(ej, h1, a1);
-          a2 = fmaf(ej, h2, a2);
-          a3 = fmaf(ej, h3, a3);
+          a0 = fmaf(ej[u], h0, a0);
+          a1 = fmaf(ej[u], h1, a1);
+          a2 = fmaf(ej[u], h2, a2);
+          a3 = fmaf(ej[u], h3, a3);
         }
       }
       if (n < 32) break;
