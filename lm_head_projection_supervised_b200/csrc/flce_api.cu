@@ -483,6 +483,17 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
+  // the label sort's scratch (checked before any work is enqueued)
+  int end_bit = 1;
+  while ((int64_t(1) << end_bit) <= V) ++end_bit;  // sort keys are 0 .. V
+  size_t need = 0;
+  {
+    cub::DoubleBuffer<uint32_t> k0(p.skeys[0], p.skeys[1]);
+    cub::DoubleBuffer<int> v0buf(p.svals[0], p.svals[1]);
+    FLCE_CK(cub::DeviceRadixSort::SortPairs(nullptr, need, k0, v0buf, static_cast<int>(L.Np), 0,
+                                            end_bit, s));
+    if (need > L.cub_bytes) return FLCE_ERR_WORKSPACE;
+  }
   st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, V, L, p, nullptr, nullptr,
                 p.pos, nullptr, s);
   if (st != FLCE_OK) return st;
@@ -574,14 +585,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       label_sort_prep_kernel<<<static_cast<unsigned>(pblocks), 256, 0, s>>>(
           p.C, p.yc, L.Np, static_cast<int>(V), p.skeys[0], p.svals[0]);
     }));
-    int end_bit = 1;
-    while ((int64_t(1) << end_bit) <= V) ++end_bit;  // keys are 0 .. V
     cub::DoubleBuffer<uint32_t> dkeys(p.skeys[0], p.skeys[1]);
     cub::DoubleBuffer<int> dvals(p.svals[0], p.svals[1]);
-    size_t need = 0;
-    FLCE_CK(cub::DeviceRadixSort::SortPairs(nullptr, need, dkeys, dvals, static_cast<int>(L.Np), 0,
-                                            end_bit, s));
-    if (need > L.cub_bytes) return FLCE_ERR_WORKSPACE;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       cub::DeviceRadixSort::SortPairs(p.cubtmp, need, dkeys, dvals, static_cast<int>(L.Np), 0,
                                       end_bit, s);
