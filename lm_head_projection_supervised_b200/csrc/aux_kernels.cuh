@@ -473,16 +473,17 @@ __global__ void __launch_bounds__(RESID_WARPS * 32)
     const int64_t c = (item % nchunk) * 32 + lane;  // this lane's 4-column group
     const uint32_t v = keys[p];
     if (v >= static_cast<uint32_t>(V_slice) || (p > 0 && keys[p - 1] == v)) continue;
-    // end of the group: first position past p whose key differs (keys ascend)
-    int64_t lo = p + 1, hi = Np;
-    while (lo < hi) {
-      const int64_t mid = (lo + hi) >> 1;
-      if (keys[mid] == v)
-        lo = mid + 1;
-      else
-        hi = mid;
+    // group length: 32 keys per step, until one differs (most groups are short)
+    int64_t len = 1;
+    for (;;) {
+      const int64_t q = p + len + lane;
+      const unsigned same = __ballot_sync(0xffffffffu, q < Np && keys[q] == v);
+      if (same != 0xffffffffu) {
+        len += __ffs(~same) - 1;  // the run of equal keys from lane 0 on
+        break;
+      }
+      len += 32;
     }
-    const int64_t len = lo - p;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     for (int64_t b = warp; b * 16 < len; b += RESID_WARPS) {
       const int64_t q0 = p + b * 16;
