@@ -451,91 +451,91 @@ __global__ void label_sort_prep_kernel(const int* __restrict__ C_dev, const int*
 // dW[v] += (S / sigma) sum_{k: y_k = v} e_k H_c[k], over the rows grouped by
 // label (keys sorted stably, so each group's rows are in ascending order):
 // the fp32 residuals of the 16-bit target entries (see scatter_dh_kernel),
-// added once per label after every panel's dW is written.  One block of
-// RESID_WARPS warps per (group start, 128-column chunk): a lane owns 4
-// columns; warp w takes the group's 16-row batches w, w + RESID_WARPS, ...
-// (row ids and residuals read once per batch and broadcast by shuffles, so
-// the batch's H loads are in flight together), and the warps' partial sums
-// are added in warp order.  Fixed order throughout: deterministic.
-constexpr int RESID_WARPS = 8;
-__global__ void __launch_bounds__(RESID_WARPS * 32)
-    dw_target_resid_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ rows,
-                           int64_t Np, int V_slice, const uint2* __restrict__ Hc,
-                           int64_t vec_per_row, int is_bf16, const float* __restrict__ tgt_resid,
-                           const float* __restrict__ scal, float inv_sigma,
-                           float4* __restrict__ dW) {
-  __shared__ float4 part[RESID_WARPS][32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// added once per label after every panel's dW is written.  One warp per
+// (group start, 128-column chunk): a lane owns 4 columns; the group's row
+// ids and residuals are read 32 at a time (one step ahead) and broadcast by
+// shuffles, so the H loads of consecutive rows are independent.  Fixed
+// order: deterministic.
+__global__ void dw_target_resid_kernel(const uint32_t* __restrict__ keys,
+                                       const int* __restrict__ rows, int64_t Np, int V_slice,
+                                       const uint2* __restrict__ Hc, int64_t vec_per_row,
+                                       int is_bf16, const float* __restrict__ tgt_resid,
+                                       const float* __restrict__ scal, float inv_sigma,
+                                       float4* __restrict__ dW) {
+  const int lane = threadIdx.x & 31;
   const int64_t nchunk = (vec_per_row + 31) / 32;
+  const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
   const float scale = (*scal) * inv_sigma;
-  for (int64_t item = blockIdx.x; item < Np * nchunk; item += gridDim.x) {
-    const int64_t p = item / nchunk;
-    const int64_t c = (item % nchunk) * 32 + lane;  // this lane's 4-column group
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < Np * nchunk; w += warps) {
+    const int64_t p = w / nchunk;
+    const int64_t c = (w % nchunk) * 32 + lane;  // this lane's 4-column group
     const uint32_t v = keys[p];
     if (v >= static_cast<uint32_t>(V_slice) || (p > 0 && keys[p - 1] == v)) continue;
-    // group length: 32 keys per step, until one differs (most groups are short)
-    int64_t len = 1;
-    for (;;) {
-      const int64_t q = p + len + lane;
-      const unsigned same = __ballot_sync(0xffffffffu, q < Np && keys[q] == v);
-      if (same != 0xffffffffu) {
-        len += __ffs(~same) - 1;  // the run of equal keys from lane 0 on
-        break;
-      }
-      len += 32;
-    }
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int64_t b = warp; b * 16 < len; b += RESID_WARPS) {
-      const int64_t q0 = p + b * 16;
-      const int n = static_cast<int>(len - b * 16 < 16 ? len - b * 16 : 16);
-      const int k = lane < n ? rows[q0 + lane] : 0;
-      const float e = lane < n ? tgt_resid[k] : 0.f;
-      uint2 hv[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int kj = __shfl_sync(0xffffffffu, k, u);
-        hv[u] = (u < n && c < vec_per_row) ? __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c)
-                                           : make_uint2(0u, 0u);
+    // up to 32 rows of the group per step: row id and residual in lane order;
+    // the next step's are fetched while this step's H rows load
+    bool in = p + lane < Np && keys[p + lane] == v;
+    int k = in ? rows[p + lane] : 0;
+    float e = in ? tgt_resid[k] : 0.f;
+    for (int64_t q0 = p;; q0 += 32) {
+      const unsigned live = __ballot_sync(0xffffffffu, in);
+      const int n = __popc(live);  // the group's rows are contiguous from q0
+      bool in_next = false;
+      int k_next = 0;
+      float e_next = 0.f;
+      if (n == 32) {
+        const int64_t qn = q0 + 32 + lane;
+        in_next = qn < Np && keys[qn] == v;
+        k_next = in_next ? rows[qn] : 0;
+        e_next = in_next ? tgt_resid[k_next] : 0.f;
       }
+      for (int j0 = 0; j0 < n; j0 += 16) {
+        // sixteen rows' loads in flight, then their terms in row order
+        uint2 hv[16];
+        float ej[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float eu = __shfl_sync(0xffffffffu, e, u);
-        if (u >= n) continue;
-        float h0, h1, h2, h3;
-        if (is_bf16) {
-          h0 = __uint_as_float(hv[u].x << 16);
-          h1 = __uint_as_float(hv[u].x & 0xFFFF0000u);
-          h2 = __uint_as_float(hv[u].y << 16);
-          h3 = __uint_as_float(hv[u].y & 0xFFFF0000u);
-        } else {
-          const float2 l2 = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].x));
-          const float2 h2v = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].y));
-          h0 = l2.x;
-          h1 = l2.y;
-          h2 = h2v.x;
-          h3 = h2v.y;
+        for (int u = 0; u < 16; ++u) {
+          const int kj = __shfl_sync(0xffffffffu, k, j0 + u);
+          ej[u] = __shfl_sync(0xffffffffu, e, j0 + u);
+          hv[u] = (j0 + u < n && c < vec_per_row)
+                      ? __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c)
+                      : make_uint2(0u, 0u);
         }
-        a0 = fmaf(eu, h0, a0);
-        a1 = fmaf(eu, h1, a1);
-        a2 = fmaf(eu, h2, a2);
-        a3 = fmaf(eu, h3, a3);
-      }
-    }
-    part[warp][lane] = make_float4(a0, a1, a2, a3);
-    __syncthreads();
-    if (warp == 0 && c < vec_per_row) {
-      float4 t = part[0][lane];
 #pragma unroll
-      for (int w = 1; w < RESID_WARPS; ++w) {
-        const float4 x = part[w][lane];
-        t = make_float4(t.x + x.x, t.y + x.y, t.z + x.z, t.w + x.w);
+        for (int u = 0; u < 16; ++u) {
+          if (j0 + u >= n) break;
+          float h0, h1, h2, h3;
+          if (is_bf16) {
+            h0 = __uint_as_float(hv[u].x << 16);
+            h1 = __uint_as_float(hv[u].x & 0xFFFF0000u);
+            h2 = __uint_as_float(hv[u].y << 16);
+            h3 = __uint_as_float(hv[u].y & 0xFFFF0000u);
+          } else {
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].y));
+            h0 = lo.x;
+            h1 = lo.y;
+            h2 = hi.x;
+            h3 = hi.y;
+          }
+          a0 = fmaf(ej[u], h0, a0);
+          a1 = fmaf(ej[u], h1, a1);
+          a2 = fmaf(ej[u], h2, a2);
+          a3 = fmaf(ej[u], h3, a3);
+        }
       }
+      if (n < 32) break;
+      in = in_next;
+      k = k_next;
+      e = e_next;
+    }
+    if (c < vec_per_row) {
       float4* dst = dW + static_cast<int64_t>(v) * vec_per_row + c;
       const float4 o = *dst;
-      *dst = make_float4(fmaf(scale, t.x, o.x), fmaf(scale, t.y, o.y), fmaf(scale, t.z, o.z),
-                         fmaf(scale, t.w, o.w));
+      *dst = make_float4(fmaf(scale, a0, o.x), fmaf(scale, a1, o.y), fmaf(scale, a2, o.z),
+                         fmaf(scale, a3, o.w));
     }
-    __syncthreads();  // part[] is reused by the next item
   }
 }
 

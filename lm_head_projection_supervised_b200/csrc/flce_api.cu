@@ -591,10 +591,10 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       cub::DeviceRadixSort::SortPairs(p.cubtmp, need, dkeys, dvals, static_cast<int>(L.Np), 0,
                                       end_bit, s);
     }));
-    const int64_t ritems = L.Np * cdiv64(D / 4, 32);
-    const int64_t rblocks = ritems < 8LL * di.sms ? ritems : 8LL * di.sms;
+    const int64_t rwarps = L.Np * cdiv64(D / 4, 32);
+    const int64_t rblocks = cdiv64(rwarps, 8) < 16LL * di.sms ? cdiv64(rwarps, 8) : 16LL * di.sms;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
-      dw_target_resid_kernel<<<static_cast<unsigned>(rblocks), RESID_WARPS * 32, 0, s>>>(
+      dw_target_resid_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
           dkeys.Current(), dvals.Current(), L.Np, static_cast<int>(V),
           reinterpret_cast<const uint2*>(p.hc), D / 4, bf16 ? 1 : 0, p.resid, p.scal,
           1.f / sigma, reinterpret_cast<float4*>(dW));
