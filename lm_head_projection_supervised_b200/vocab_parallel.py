@@ -96,20 +96,21 @@ class VocabParallelLinearCrossEntropy(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, H, W_slice, b_slice, labels, mask, ignore_index, V_total, v0, group,
-                weight=None, reduction="mean", denom=None, round_logits=False):
+                weight=None, reduction="mean", denom=None, round_logits=False, ops=binding):
         loss, m, logs = forward(H, W_slice, b_slice, labels, mask, ignore_index,
                                 V_total=V_total, v0=v0, group=group, weight=weight,
-                                reduction=reduction, denom=denom, round_logits=round_logits)
+                                reduction=reduction, denom=denom, round_logits=round_logits,
+                                ops=ops)
         ctx.save_for_backward(H, W_slice, b_slice, labels, mask, weight, m, logs)
-        ctx.cfg = (ignore_index, V_total, v0, group, reduction, denom, round_logits)
+        ctx.cfg = (ignore_index, V_total, v0, group, reduction, denom, round_logits, ops)
         return loss
 
     @staticmethod
     def backward(ctx, grad_out):
         H, W_slice, b_slice, labels, mask, weight, m, logs = ctx.saved_tensors
-        ignore_index, V_total, v0, group, reduction, denom, round_logits = ctx.cfg
+        ignore_index, V_total, v0, group, reduction, denom, round_logits, ops = ctx.cfg
         kw = dict(V_total=V_total, v0=v0, group=group, weight=weight, reduction=reduction,
-                  denom=denom, round_logits=round_logits)
+                  denom=denom, round_logits=round_logits, ops=ops)
         if reduction == "none":
             kw["grad_rows"] = grad_out.reshape(-1)
         else:
@@ -117,20 +118,20 @@ class VocabParallelLinearCrossEntropy(torch.autograd.Function):
         dH, dW, db = backward(H, W_slice, b_slice, labels, mask, ignore_index, m, logs, **kw)
         return (dH.reshape(H.shape).to(H.dtype), dW.to(W_slice.dtype),
                 None if db is None else db.to(b_slice.dtype),
-                None, None, None, None, None, None, None, None, None, None)
+                None, None, None, None, None, None, None, None, None, None, None)
 
 
 def vocab_parallel_cross_entropy(H, W_slice, labels, *, V_total: int, v0: int, group=None,
                                  b_slice=None, mask=None, ignore_index: int = -100, weight=None,
                                  reduction: str = "mean", denom: Optional[float] = None,
-                                 round_logits: bool = False):
+                                 round_logits: bool = False, ops=binding):
     """Loss of the full vocabulary from this rank's slice, differentiable in
     H, W_slice and b_slice.  H: [N, D] (or [..., D]) replicated on the group."""
     D = H.shape[-1]
     loss = VocabParallelLinearCrossEntropy.apply(
         H.reshape(-1, D), W_slice, b_slice, labels.reshape(-1),
         None if mask is None else mask.reshape(-1), ignore_index, V_total, v0, group,
-        None if weight is None else weight.reshape(-1), reduction, denom, round_logits)
+        None if weight is None else weight.reshape(-1), reduction, denom, round_logits, ops)
     return loss.reshape(labels.shape) if reduction == "none" else loss
 
 

@@ -16,6 +16,14 @@ from lm_head_projection_supervised_b200 import vocab_parallel as vp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _free_port():
+    """A TCP port on 127.0.0.1 that the OS reports free (for the rendezvous)."""
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 @pytest.mark.parametrize("V,P", [(248320, 8), (248320, 3), (32000, 8), (1000, 7), (9, 9),
                                  (257, 2), (512, 2), (100000, 1)])
 def test_vocab_slice_partitions_the_vocabulary(V, P):
@@ -122,7 +130,7 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
     from oracle import flce_oracle as orc
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29600 + (os.getpid() + 7 * world) % 1000
+    port = _free_port()
     procs = [ctx.Process(target=_worker, args=(r, world, port, reduction, q))
              for r in range(world)]
     for p in procs:
@@ -148,3 +156,59 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
         assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12     # local slice of dW
         assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
     assert sum(r[2] for r in res) == W.shape[0]
+
+
+def _autograd_worker(rank, world, port, reduction, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from lm_head_projection_supervised_b200 import vocab_parallel as vpar
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        H, W, b, y, mask, w = [torch.from_numpy(a) for a in _inputs(seed=13)]
+        V = W.shape[0]
+        v0, n = vpar.vocab_slice(V, world, rank, align=64)
+        Hp = H.clone().requires_grad_(True)
+        Wp = W[v0:v0 + n].clone().requires_grad_(True)
+        bp = b[v0:v0 + n].clone().requires_grad_(True)
+        loss = vpar.vocab_parallel_cross_entropy(Hp, Wp, y, V_total=V, v0=v0, b_slice=bp,
+                                                 mask=mask, weight=w, reduction=reduction,
+                                                 ops=OracleOps)
+        g = torch.linspace(-1.0, 2.0, H.shape[0], dtype=torch.float64)
+        (loss if reduction != "none" else loss * g).sum().mul(0.8).backward()
+        q.put((rank, v0, n, loss.detach().numpy(), Hp.grad.numpy(), Wp.grad.numpy(),
+               bp.grad.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("reduction", ["mean", "none"])
+def test_gloo_autograd_wrapper(reduction):
+    """vocab_parallel_cross_entropy through torch.autograd on 2 gloo ranks:
+    the upstream gradient reaches the slice calls as the device-scalar lambda
+    (mean) or as per-row gradients (none), and the gradients equal the dense
+    oracle's."""
+    from oracle import flce_oracle as orc
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_autograd_worker, args=(r, 2, port, reduction, q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted([q.get(timeout=180) for _ in range(2)], key=lambda t: t[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    H, W, b, y, mask, w = _inputs(seed=13)
+    g = np.linspace(-1.0, 2.0, H.shape[0])
+    ref = orc.forward_backward(H, W, b, y, mask, lam=0.8, weight=w, reduction=reduction,
+                               grad_rows=0.8 * g if reduction == "none" else None)
+    for _, v0, n, loss, dH, dW, db in res:
+        want = ref["loss_vec"] if reduction == "none" else ref["loss"]
+        assert np.max(np.abs(loss - want)) < 1e-12
+        assert np.max(np.abs(dH - ref["dH"])) < 1e-12
+        assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12
+        assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
