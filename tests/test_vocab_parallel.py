@@ -178,3 +178,34 @@ def test_accumulate_dh_adds_in_place():
     unsup = torch.from_numpy(np.setdiff1d(np.arange(inp.N), idx)).cuda()
     assert torch.equal(acc[unsup], base[unsup])
     assert (acc - (base + dH)).abs().max().item() <= 1e-6 * (base + dH).abs().max().item()
+
+
+def test_autograd_wrapper_on_a_one_rank_nccl_group():
+    """vocab_parallel_cross_entropy with the real NCCL collectives (one rank:
+    the whole vocabulary is the slice) equals the unsharded call, through
+    torch.autograd."""
+    import socket
+
+    import torch.distributed as dist
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        inp = wl.random_case(seed=63, N=200, D=64, V=3000)
+        H, W, b, y, mk = to_device(inp)
+        Hp = H.clone().requires_grad_(True)
+        Wp = W.clone().requires_grad_(True)
+        bp = b.clone().requires_grad_(True)
+        loss = vp.vocab_parallel_cross_entropy(Hp, Wp, y, V_total=inp.V, v0=0, b_slice=bp,
+                                               mask=mk)
+        (0.5 * loss).backward()
+        ref_loss, m, logs = binding.forward(H, W, b, y, mk)
+        dH, dW, db = binding.backward(H, W, b, y, mk, -100, m, logs, lam=0.5)
+        check_loss(loss.item(), ref_loss.item())
+        for got, ref in ((Hp.grad, dH), (Wp.grad, dW), (bp.grad, db)):
+            g = got.float()
+            assert (g - ref).abs().max().item() <= 1e-2 * ref.abs().max().item()
+    finally:
+        dist.destroy_process_group()
