@@ -10,23 +10,27 @@
 // warp 1 issues tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256, K=16),
 // which reads both CTAs' stages and writes both CTAs' TMEM, into one of two
 // accumulators (512 columns).  In each CTA, warp 0 streams that CTA's halves
-// of the operands and warps 4..7 read a finished accumulator with
-// tcgen05.ld (thread = TMEM lane = tile row) and run the epilogue while the
-// next unit accumulates in the other.
+// of the operands (in the backward warp 0 the A boxes and warp 2 the B
+// boxes), and two epilogue warpgroups (warps 4..7 and 8..11, each on half of
+// the columns) read a finished accumulator with tcgen05.ld (thread = TMEM
+// lane = tile row) and run the epilogue while the next unit accumulates in
+// the other.
 //
 // Modes (one launch = one mode):
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
 //              running max / rescaled exp-sum over the tile's columns and
 //              captures the target logit from the tile that holds it
 //              ("分块交叉熵" page, §02), writing one (m, s) partial per row
-//              and vocabulary tile.
+//              and half tile (one per epilogue warpgroup).
 //   kModeBwd   three unit classes in one launch, with no dependency between
 //              them:
 //              class 2 (grad): the tile of vocabulary panel p recomputed; the
 //                 epilogue rebuilds p = exp((Z - m) - log s) from the saved
 //                 statistics, subtracts the one-hot target (§04), rounds to
 //                 the 16-bit input type, stages 128 x 64 boxes in shared
-//                 memory and stores them with TMA into gradient buffer p % 2;
+//                 memory and stores them with TMA into gradient buffer p % 2,
+//                 and records what the rounding took off each row's target
+//                 entry (added back in fp32 to dH, dW and db later);
 //              The panel holds r_k (p - onehot) sigma with the row scale
 //              s_k = S r_k (S = max |s_k|), the contractions multiply by S / sigma.
 //              class 0 (dW): dW[panel p-1 rows] = G^T H_c  (K = C), stored by TMA;
