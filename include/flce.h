@@ -152,10 +152,10 @@ FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
  * process exits).  It calls no cudaMalloc, cudaFree or other allocating
  * routine.  The caller still passes all inputs and outputs.
  *
- *  - Size limit: the forward's scratch, about (N rounded up to 128) x
- *    (2 D + 8 ceil(V / 256) + 16) bytes, must fit in FLCE_NOALLOC_SCRATCH_BYTES
- *    (the small workload, N=2048 D=512 V=32000, needs about 4 MiB; the
- *    16k-row, 248320-vocabulary case needs about 160 MiB and does not fit);
+ *  - Size limit: the forward's scratch, about (N rounded up to 256) x
+ *    (2 D + 16 ceil(V / 256) + 20) bytes, must fit in FLCE_NOALLOC_SCRATCH_BYTES
+ *    (the small workload, N=2048 D=512 V=32000, needs about 6 MiB; the
+ *    16k-row, 248320-vocabulary case needs about 275 MiB and does not fit);
  *    larger problems get FLCE_ERR_WORKSPACE before anything is enqueued.
  *  - The first call on each device looks up the buffer's device address with
  *    that device current; make that first call before any stream capture.

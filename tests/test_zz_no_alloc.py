@@ -34,7 +34,7 @@ def test_oversized_problem_is_rejected_before_any_gpu_work():
     """Sizes whose workspace exceeds the fixed buffer get FLCE_ERR_WORKSPACE."""
     f = _noalloc_fn()
     fake = ctypes.c_void_p(0x100000)
-    N, D, V = 16384, 1024, 248320   # forward scratch ~160 MiB
+    N, D, V = 16384, 1024, 248320   # forward scratch ~275 MiB
     st = f(fake, fake, None, fake, None, -100, N, D, V, 0, fake, fake, fake, None)
     assert binding.STATUS[st] == "FLCE_ERR_WORKSPACE"
 
