@@ -326,21 +326,28 @@ __global__ void __launch_bounds__(1024)
 }
 
 // db[vp + j] = (S / sigma) * sum_{i < C} (Gp[i][j] + [y_i = vp + j] e_i) for the
-// panel's columns, in a fixed order: 8 row groups per block, combined in
-// group order.  e_i is what the 16-bit rounding took off row i's target entry
-// (recorded by the gradient units), so the target terms enter db exactly.
+// panel's columns, in two passes with a fixed order.  e_i is what the 16-bit
+// rounding took off row i's target entry (recorded by the gradient units), so
+// the target terms enter db exactly.
+// Pass 1: block (x, s) sums 64 columns over the rows of split s (rows
+// s * ceil(C / gridDim.y) ...), 8 row groups per block combined in group
+// order, into bpart[s][j].
+constexpr int BIAS_SPLITS = 16;
 __global__ void __launch_bounds__(256)
-    bias_grad_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
-                     const int* __restrict__ C_dev, const float* __restrict__ scal,
-                     float inv_sigma, int is_bf16, int vp, const int* __restrict__ y_c,
-                     const float* __restrict__ tgt_resid, float* __restrict__ db) {
+    bias_partial_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
+                        const int* __restrict__ C_dev, int is_bf16, int vp,
+                        const int* __restrict__ y_c, const float* __restrict__ tgt_resid,
+                        float* __restrict__ bpart) {
   __shared__ float2 part[8][32];
   const int C = *C_dev;
   const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
   const int j = blockIdx.x * 64 + 2 * lane;  // two adjacent columns per thread
+  const int per = (C + static_cast<int>(gridDim.y) - 1) / static_cast<int>(gridDim.y);
+  const int r0 = static_cast<int>(blockIdx.y) * per;
+  const int r1 = min(C, r0 + per);
   float2 acc = make_float2(0.f, 0.f);
   if (j < w) {
-    for (int i = grp; i < C; i += 8) {
+    for (int i = r0 + grp; i < r1; i += 8) {
       const uint32_t v = *reinterpret_cast<const uint32_t*>(Gp + static_cast<int64_t>(i) * ldg + j);
       float gx, gy;
       if (is_bf16) {
@@ -366,10 +373,22 @@ __global__ void __launch_bounds__(256)
       t.x += part[k][lane].x;
       t.y += part[k][lane].y;
     }
-    const float scale = (C > 0) ? *scal * inv_sigma : 0.f;
-    db[vp + j] = t.x * scale;
-    if (j + 1 < w) db[vp + j + 1] = t.y * scale;
+    float* dst = bpart + static_cast<int64_t>(blockIdx.y) * w;
+    dst[j] = t.x;
+    if (j + 1 < w) dst[j + 1] = t.y;
   }
+}
+
+// Pass 2: db[vp + j] = (S / sigma) * sum_s bpart[s][j], splits in order.
+__global__ void bias_finish_kernel(const float* __restrict__ bpart, int splits, int w,
+                                   const int* __restrict__ C_dev, const float* __restrict__ scal,
+                                   float inv_sigma, int vp, float* __restrict__ db) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= w) return;
+  float t = 0.f;
+  for (int sp = 0; sp < splits; ++sp) t += bpart[static_cast<int64_t>(sp) * w + j];
+  const float scale = (*C_dev > 0) ? *scal * inv_sigma : 0.f;
+  db[vp + j] = t * scale;
 }
 
 // dH[i] = dH_c[pos[i]] + (S / sigma) e_k W[y_k] for supervised rows (k =

@@ -43,7 +43,7 @@ int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, rs, resid, skeys[2], svals[2], cubtmp, cub_bytes, dhc, gpanel[2], total;
+  size_t pos, rs, resid, skeys[2], svals[2], cubtmp, cub_bytes, bpart, dhc, gpanel[2], total;
   int64_t Np, nvt, nparts, vc, gld, panels;
 };
 
@@ -84,6 +84,7 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   }
   L.cub_bytes = static_cast<size_t>(L.Np) * 4 + (size_t(4) << 20);
   L.cubtmp = take(L.cub_bytes);
+  L.bpart = take(static_cast<size_t>(BIAS_SPLITS) * L.vc * 4);  // db partials of one panel
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
   L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.gld * 2);
   L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.gld * 2);
@@ -302,6 +303,7 @@ struct WsPtrs {
   uint32_t* skeys[2];
   int* svals[2];
   void* cubtmp;
+  float* bpart;
   float* dhc;
   uint16_t* gpanel[2];
 };
@@ -327,6 +329,7 @@ WsPtrs carve(void* ws, const Layout& L) {
     p.svals[i] = reinterpret_cast<int*>(w + L.svals[i]);
   }
   p.cubtmp = w + L.cubtmp;
+  p.bpart = reinterpret_cast<float*>(w + L.bpart);
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
   p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
   p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
@@ -571,9 +574,14 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     if (b != nullptr && has_g) {
       const uint16_t* gp = p.gpanel[Lp & 1];
       FLCE_CK(timed_launch(kProfAux, s, [&] {
-        bias_grad_kernel<<<static_cast<unsigned>(cdiv64(w_g, 64)), 256, 0, s>>>(
-            gp, L.gld, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma, bf16 ? 1 : 0,
-            static_cast<int>(vp_g), p.yc, p.resid, db);
+        bias_partial_kernel<<<dim3(static_cast<unsigned>(cdiv64(w_g, 64)), BIAS_SPLITS), 256, 0,
+                              s>>>(gp, L.gld, static_cast<int>(w_g), p.C, bf16 ? 1 : 0,
+                                   static_cast<int>(vp_g), p.yc, p.resid, p.bpart);
+      }));
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+        bias_finish_kernel<<<static_cast<unsigned>(cdiv64(w_g, 256)), 256, 0, s>>>(
+            p.bpart, BIAS_SPLITS, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma,
+            static_cast<int>(vp_g), db);
       }));
     }
   }
