@@ -3,14 +3,16 @@
 //
 // Forward  (one stream, no host synchronisation):
 //   compact -> gather H_c -> gemm<fwd> (Z tiles + online (m, s) + target)
-//   -> merge partials per row -> fixed-order loss mean
+//   -> merge partials per row -> fixed-order loss reduction
 // Backward, with P vocabulary panels of Vc columns and two panel buffers:
 //   compact -> gather H_c ->
 //   for L = 0 .. P:   gemm<bwd> with
 //                       grad units of panel L     (if L < P) -> buffer L % 2
 //                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 2
-//                     bias_grad of panel L (bias only, if L < P)
-//   -> scatter dH_c to dH (zero rows for unsupervised positions)
+//                     db of panel L in two passes (bias only, if L < P)
+//   -> rows grouped by label (stable radix sort) -> dW target terms in fp32
+//   -> scatter dH_c to dH with its target terms (zero rows for unsupervised
+//      positions)
 //   with row scales s_k = S r_k computed first (row_scale_kernel); the panels
 //   hold r_k (p - onehot) sigma and the dW / dH epilogues multiply by S / sigma.
 #include <mutex>
