@@ -329,53 +329,74 @@ __global__ void __launch_bounds__(1024)
 // panel's columns, in two passes with a fixed order.  e_i is what the 16-bit
 // rounding took off row i's target entry (recorded by the gradient units), so
 // the target terms enter db exactly.
-// Pass 1: block (x, s) sums 64 columns over the rows of split s (rows
-// s * ceil(C / gridDim.y) ...), 8 row groups per block combined in group
-// order, into bpart[s][j].
-constexpr int BIAS_SPLITS = 16;
+// Pass 1: block (x, s) sums 256 columns over the rows of split s (rows
+// s * ceil(C / gridDim.y) ...): warp g takes rows g, g + 8, ... of the split
+// (four rows' 16-byte loads in flight per lane, 8 columns each); the 8 warps'
+// sums are added in warp order into bpart[s][j].  A lane reads up to 7
+// columns past the panel width, inside the panel row (whose pitch is a
+// multiple of 256 columns); those columns are never written out.
+constexpr int BIAS_SPLITS = 32;
 __global__ void __launch_bounds__(256)
     bias_partial_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
                         const int* __restrict__ C_dev, int is_bf16, int vp,
                         const int* __restrict__ y_c, const float* __restrict__ tgt_resid,
                         float* __restrict__ bpart) {
-  __shared__ float2 part[8][32];
+  __shared__ float part[8][256];
   const int C = *C_dev;
   const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const int j = blockIdx.x * 64 + 2 * lane;  // two adjacent columns per thread
+  const int j0 = blockIdx.x * 256 + lane * 8;  // this lane's 8 columns
   const int per = (C + static_cast<int>(gridDim.y) - 1) / static_cast<int>(gridDim.y);
   const int r0 = static_cast<int>(blockIdx.y) * per;
   const int r1 = min(C, r0 + per);
-  float2 acc = make_float2(0.f, 0.f);
-  if (j < w) {
-    for (int i = r0 + grp; i < r1; i += 8) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(Gp + static_cast<int64_t>(i) * ldg + j);
-      float gx, gy;
+  float acc[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+  auto add_row = [&](const uint4& v, int i) {
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    float g[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
       if (is_bf16) {
-        gx = __uint_as_float((v & 0xFFFFu) << 16);
-        gy = __uint_as_float(v & 0xFFFF0000u);
+        g[2 * h] = __uint_as_float(wv[h] << 16);
+        g[2 * h + 1] = __uint_as_float(wv[h] & 0xFFFF0000u);
       } else {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
-        gx = f.x;
-        gy = f.y;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h]));
+        g[2 * h] = f.x;
+        g[2 * h + 1] = f.y;
       }
-      const int yc = __ldg(y_c + i) - vp;  // the row's label as a column of this panel
-      if (yc == j) gx += __ldg(tgt_resid + i);
-      if (yc == j + 1) gy += __ldg(tgt_resid + i);
-      acc.x += gx;
-      acc.y += gy;
     }
+    const int yc = __ldg(y_c + i) - vp - j0;  // the row's label among this lane's columns
+    if (static_cast<unsigned>(yc) < 8u) {
+      const float e = __ldg(tgt_resid + i);
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        if (t == yc) g[t] += e;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] += g[t];
+  };
+  if (j0 < w) {
+    int i = r0 + grp;
+    for (; i + 24 < r1; i += 32) {  // four rows per step, loads first
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = __ldg(reinterpret_cast<const uint4*>(Gp + static_cast<int64_t>(i + 8 * u) * ldg + j0));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) add_row(v[u], i + 8 * u);
+    }
+    for (; i < r1; i += 8)
+      add_row(__ldg(reinterpret_cast<const uint4*>(Gp + static_cast<int64_t>(i) * ldg + j0)), i);
   }
-  part[grp][lane] = acc;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) part[grp][lane * 8 + t] = acc[t];
   __syncthreads();
-  if (grp == 0 && j < w) {
-    float2 t = part[0][lane];
-    for (int k = 1; k < 8; ++k) {
-      t.x += part[k][lane].x;
-      t.y += part[k][lane].y;
-    }
-    float* dst = bpart + static_cast<int64_t>(blockIdx.y) * w;
-    dst[j] = t.x;
-    if (j + 1 < w) dst[j + 1] = t.y;
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j < w) {
+    float t = part[0][threadIdx.x];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) t += part[k][threadIdx.x];
+    bpart[static_cast<int64_t>(blockIdx.y) * w + j] = t;
   }
 }
 

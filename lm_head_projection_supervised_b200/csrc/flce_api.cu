@@ -576,7 +576,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     if (b != nullptr && has_g) {
       const uint16_t* gp = p.gpanel[Lp & 1];
       FLCE_CK(timed_launch(kProfAux, s, [&] {
-        bias_partial_kernel<<<dim3(static_cast<unsigned>(cdiv64(w_g, 64)), BIAS_SPLITS), 256, 0,
+        bias_partial_kernel<<<dim3(static_cast<unsigned>(cdiv64(w_g, 256)), BIAS_SPLITS), 256, 0,
                               s>>>(gp, L.gld, static_cast<int>(w_g), p.C, bf16 ? 1 : 0,
                                    static_cast<int>(vp_g), p.yc, p.resid, p.bpart);
       }));
