@@ -363,9 +363,7 @@ def device_status(ws: Workspace, stream=None) -> int:
 def compact(labels, mask, ignore_index: int, V: int, stream=None):
     """idx (int32, first C valid) and C (int32 device scalar) -- flce_compact()."""
     y = labels.reshape(-1).to(torch.int64).contiguous()
-    mk = None
-    if mask is not None:
-        mk = mask.reshape(-1).to(torch.uint8).contiguous()
+    mk = _mask_u8(mask)
     N = y.numel()
     idx = torch.empty(max(N, 1), dtype=torch.int32, device=y.device)
     C = torch.empty((), dtype=torch.int32, device=y.device)

@@ -258,3 +258,14 @@ def test_shard_combine_workspace_bytes(L):
     assert L.flce_shard_combine_workspace_bytes(-1) == 0
     a = L.flce_shard_combine_workspace_bytes(1000)
     assert a >= 2 * 1000 * 4 and a < L.flce_shard_combine_workspace_bytes(100000)
+
+
+def test_mask_conversion_keeps_every_nonzero_entry():
+    """Any nonzero mask value means "takes part", also for integer masks whose
+    values do not fit in a byte (a plain uint8 cast would wrap 256 to 0)."""
+    import torch
+    from lm_head_projection_supervised_b200.binding import _mask_u8
+    m = _mask_u8(torch.tensor([0, 1, 256, -3, 7]))
+    assert m.dtype == torch.uint8 and m.tolist() == [0, 1, 1, 1, 1]
+    assert _mask_u8(torch.tensor([True, False])).tolist() == [1, 0]
+    assert _mask_u8(None) is None
