@@ -5,7 +5,6 @@ tilings and vocabulary partitions, the identities the pages state hold.
   [p5] AIInfraGuide ch. 2 "数学基础" (maths basics)
 """
 import numpy as np
-import pytest
 import scipy.special
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
@@ -91,11 +90,40 @@ def test_any_vocabulary_partition_merges_to_dense(prob, data):
 @settings(**SETTINGS)
 @given(problems())
 def test_gradient_rows_sum_to_zero(prob):
-    """sum_j p_ij = 1 ([p5] §5.2), so each supervised row of G sums to 0 and
-    db sums to 0; with a bias, dW's column sums are the H-weighted same."""
+    """sum_j p_ij = 1 ([p5] §5.2), so each supervised row of G sums to 0: db
+    sums to 0 and so does every column of dW (sum_j dW_j = sum_i (sum_j G_ij) H_i)."""
     H, W, b, y, mask = prob
     d = orc.forward_backward(H, W, b, y, mask, lam=1.0)
     if b is not None:
         assert abs(np.sum(d["db"])) <= 1e-13 * max(1.0, np.max(np.abs(d["db"])) * W.shape[0])
     assert np.max(np.abs(d["dW"].sum(axis=0)), initial=0.0) <= 1e-12 * max(
         1.0, np.max(np.abs(d["dW"])) * W.shape[0])
+
+
+@settings(**SETTINGS)
+@given(problems(), st.integers(0, 2**31 - 1))
+def test_reductions_are_consistent(prob, seed):
+    """The NeMo-style reductions of the same per-row losses agree with one
+    another: sum over 'none' rows = 'sum'; 'mean' = 'sum' with denom = C; and
+    the gradients scale the same way (per-row upstream gradients of 1/C give
+    the mean's gradients)."""
+    H, W, b, y, mask = prob
+    rng = np.random.default_rng(seed)
+    w = rng.uniform(0.0, 2.0, H.shape[0])
+    none = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="none",
+                                grad_rows=np.ones(H.shape[0]))
+    summ = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="sum", lam=1.0)
+    C = none["C"]
+    assert abs(np.sum(none["loss_vec"]) - summ["loss"]) <= 1e-12 * max(1.0, abs(summ["loss"]))
+    for k in ("dH", "dW"):
+        assert np.max(np.abs(none[k] - summ[k]), initial=0.0) <= 1e-12 * max(
+            1.0, np.max(np.abs(summ[k]), initial=0.0))
+    if C:
+        mean = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="mean", lam=1.0)
+        den = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="sum", denom=float(C),
+                                   lam=1.0)
+        assert abs(mean["loss"] - den["loss"]) <= 1e-13 * max(1.0, abs(mean["loss"]))
+        g = orc.forward_backward(H, W, b, y, mask, weight=w, reduction="none",
+                                 grad_rows=np.full(H.shape[0], 1.0 / C))
+        assert np.max(np.abs(g["dW"] - mean["dW"]), initial=0.0) <= 1e-12 * max(
+            1.0, np.max(np.abs(mean["dW"]), initial=0.0))
