@@ -6,8 +6,9 @@ benchmark's CPU-baseline leg.  It shares no code with the CUDA path.
 from .flce_oracle import (IGNORE_INDEX, backward, chunked, forward, forward_backward,
                           objective, row_outputs, row_scales, supervised_rows,
                           vocab_outputs)
+from .flce_filtered import backward_filtered
 from .flce_shards import shard_backward, shard_combine, shard_partials
 
-__all__ = ["IGNORE_INDEX", "backward", "chunked", "forward", "forward_backward",
+__all__ = ["IGNORE_INDEX", "backward", "backward_filtered", "chunked", "forward", "forward_backward",
            "objective", "row_outputs", "row_scales", "shard_backward", "shard_combine",
            "shard_partials", "supervised_rows", "vocab_outputs"]
