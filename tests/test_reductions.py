@@ -61,8 +61,9 @@ def test_reduction_parity(name, kw, reduction, weighted, denom):
         assert np.all(got[unsup] == 0.0)
     else:
         check_loss(loss.item(), ref["loss"])
-    check_stats(m.cpu().numpy(), ref["m"], idx)
-    check_stats(logs.cpu().numpy(), ref["logs"], idx, floor=logs_floor(ref["m"][idx], inp.D))
+    check_stats(m.cpu().numpy(), ref["m"], idx, quantity="m")
+    check_stats(logs.cpu().numpy(), ref["logs"], idx, floor=logs_floor(ref["m"][idx], inp.D),
+                quantity="logs")
     check_grad("dH", dH.cpu().numpy(), ref["dH"])
     check_grad("dW", dW.cpu().numpy(), ref["dW"])
     if inp.b is not None:
@@ -138,9 +139,9 @@ def test_rounded_logits_parity(kw):
     # the variant is visible: the rounded-logit loss is not the exact one
     assert abs(ref["loss"] - plain["loss"]) > 10 * abs(loss.item() - ref["loss"])
     ulp = ulp16(ref["m"][idx], inp.dtype)
-    check_stats(m.cpu().numpy(), ref["m"], idx, floor=ulp)
+    check_stats(m.cpu().numpy(), ref["m"], idx, floor=ulp, quantity="m")
     check_stats(logs.cpu().numpy(), ref["logs"], idx,
-                floor=np.maximum(ulp, logs_floor(ref["m"][idx], inp.D)))
+                floor=np.maximum(ulp, logs_floor(ref["m"][idx], inp.D)), quantity="logs")
     check_grad("dH", dH.cpu().numpy(), ref["dH"])
     check_grad("dW", dW.cpu().numpy(), ref["dW"])
     if inp.b is not None:

@@ -99,8 +99,8 @@ def test_slices_reproduce_the_dense_oracle(name, kw, P, extra):
         frac = 7 if inp.dtype == "bf16" else 10
         floor = np.maximum(floor, 2.0 ** (np.floor(np.log2(np.maximum(
             np.abs(ref["m"][idx]), 2.0 ** -14))) - frac))
-    check_stats(_np(got["m"]), ref["m"], idx, floor=floor if rl else None)
-    check_stats(_np(got["logs"]), ref["logs"], idx, floor=floor)
+    check_stats(_np(got["m"]), ref["m"], idx, floor=floor if rl else None, quantity="m")
+    check_stats(_np(got["logs"]), ref["logs"], idx, floor=floor, quantity="logs")
     check_grad("dH", _np(got["dH"]), ref["dH"])
     check_grad("dW", _np(got["dW"]), ref["dW"])
     if inp.b is not None:
@@ -118,7 +118,7 @@ def test_one_slice_equals_the_unsharded_call():
     dH, dW, db = binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam)
     idx, _ = orc.supervised_rows(inp.labels, inp.mask)
     assert torch.equal(got["m"], m)
-    check_stats(_np(got["logs"]), _np(logs).astype(np.float64), idx)
+    check_stats(_np(got["logs"]), _np(logs).astype(np.float64), idx, quantity="logs")
     check_loss(got["loss"].item(), loss.item())
     for a, c in ((got["dH"], dH), (got["dW"], dW), (got["db"], db)):
         assert (a - c).abs().max().item() <= 1e-5 * c.abs().max().item()
