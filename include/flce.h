@@ -153,12 +153,16 @@ FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
  * routine.  The caller still passes all inputs and outputs.
  *
  *  - Size limit: the forward's scratch, about (N rounded up to 256) x
- *    (2 D + 16 ceil(V / 256) + 20) bytes, must fit in FLCE_NOALLOC_SCRATCH_BYTES
- *    (the small workload, N=2048 D=512 V=32000, needs about 6 MiB; the
- *    16k-row, 248320-vocabulary case needs about 275 MiB and does not fit);
+ *    (2 D + 8 ceil(V / 256) + 20) bytes, must fit in FLCE_NOALLOC_SCRATCH_BYTES
+ *    (the small workload, N=2048 D=512 V=32000, needs about 4 MiB; the
+ *    16k-row, 248320-vocabulary case needs about 154 MiB and does not fit);
  *    larger problems get FLCE_ERR_WORKSPACE before anything is enqueued.
- *  - The first call on each device looks up the buffer's device address with
- *    that device current; make that first call before any stream capture.
+ *  - Every call looks up the buffer's device address on the current device
+ *    (cudaGetSymbolAddress, which allocates nothing; no address is kept
+ *    between calls, so a reset of the device's primary context, which loads
+ *    the library's module and the buffer again, cannot leave a stale one).
+ *    The first call on a device also loads the kernels there: make that
+ *    first call before any stream capture.
  *  - All calls on a device share the one buffer, which keeps the previous
  *    call's contents; the call clears what has to start at zero.  Calls that
  *    overlap on the GPU (different streams or host threads) race on the
@@ -195,6 +199,15 @@ typedef enum { FLCE_REDUCE_MEAN = 0, FLCE_REDUCE_SUM = 1, FLCE_REDUCE_NONE = 2 }
  *   are).  With it the dH terms of several vocabulary slices, or of several
  *   losses on one hidden state, sum in place. */
 #define FLCE_FLAG_ACCUMULATE_DH 2u
+/* FLCE_FLAG_REUSE_FORWARD (backward calls only): the workspace still holds
+ *   what a forward call (flce_forward, flce_forward_ex or flce_shard_forward)
+ *   left there for the same H, labels, mask, ignore_index, N, D and V (the
+ *   supervised-row list, C, the gathered rows H_c and the row map), and
+ *   nothing has written to the workspace since: the backward skips the
+ *   compaction and the gather and uses them.  The caller guarantees that
+ *   H, labels and mask did not change in between; the result is undefined
+ *   otherwise.  A device error recorded by that forward stays recorded. */
+#define FLCE_FLAG_REUSE_FORWARD 4u
 
 /*
  * Forward with a reduction.  weight: device float [N] or NULL.  loss: device
@@ -228,6 +241,34 @@ FLCE_API flce_status flce_backward_ex(const void* H, const void* W, const void* 
                                       unsigned flags, float lambda, const float* lambda_dev,
                                       const float* grad_rows, float* dH, float* dW, float* db,
                                       void* ws, size_t ws_bytes, flce_stream stream);
+
+/*
+ * Backward with opt-in gradient filtering, an approximation: the
+ * "分块交叉熵 / Output projection / exact cross entropy" page (§07, on Apple's
+ * Cut Cross-Entropy) describes skipping the blocks of the softmax whose
+ * probabilities are all negligible in the backward contractions.  Here a
+ * block is 128 consecutive supervised rows (ascending row order) by 64
+ * consecutive vocabulary ids, aligned to multiples of 128 and 64; a block
+ * whose every |p_ij - 1[j = y_i]| is below filter_eps contributes nothing to
+ * dH and dW (the dW / dH contractions skip it), while db keeps every entry.
+ * The test is made in fp32 on the kernel's p.  filter_eps = 0 is the exact
+ * backward, identical to flce_backward_ex(); filter_eps < 0 or not finite:
+ * FLCE_ERR_ARG.  Every other argument as in flce_backward_ex().  The result is
+ * reported against the exact oracle in the tests; how far it departs from the
+ * exact gradient depends on the inputs (for logits with a few dominant
+ * entries per row, little; for flat logits, p ~ 1 / V everywhere, it drops
+ * almost everything off the target entries).
+ */
+FLCE_API flce_status flce_backward_filtered(const void* H, const void* W, const void* b,
+                                            const int64_t* labels, const uint8_t* mask,
+                                            int64_t ignore_index, int64_t N, int64_t D,
+                                            int64_t V, int dtype, const float* m,
+                                            const float* logs, const float* weight,
+                                            int reduction, float denom, unsigned flags,
+                                            float lambda, const float* lambda_dev,
+                                            const float* grad_rows, float filter_eps, float* dH,
+                                            float* dW, float* db, void* ws, size_t ws_bytes,
+                                            flce_stream stream);
 
 /*
  * Vocabulary-sharded (tensor-parallel over V) form.

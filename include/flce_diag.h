@@ -42,13 +42,23 @@ FLCE_API flce_status flce_diag_gemm(const void* A, const void* B, float* out,
 FLCE_API flce_status flce_diag_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, flce_stream stream);
 
 /*
+ * Computes y_poly[i] = ex2_poly(x[i]) (the exponential the epilogues evaluate
+ * on the FMA pipe for small hidden sizes) and y_sfu[i] = ex2.approx(x[i])
+ * (the special-function unit's), for accuracy tests.  Device pointers, n >= 0.
+ */
+FLCE_API flce_status flce_diag_exp2(const float* x, float* y_poly, float* y_sfu, int64_t n,
+                                    flce_stream stream);
+
+/*
  * Per-launch timing of the library's own kernels.  Between begin and end,
  * every kernel the library enqueues is bracketed by two CUDA events on the
- * caller's stream (this adds no synchronisation).  end() waits for those
- * events and returns, per kind k in [0, nkinds), the summed duration in ms
- * and the number of launches:
- *   0 = forward tile GEMM, 1 = gradient-panel GEMM, 2 = dW/dH GEMM,
- *   3 = every other kernel (compaction, gather, merge, loss, zeroing, db).
+ * caller's stream (this adds no synchronisation), except the backward's chain
+ * of GEMM launches, which overlap one another (programmatic dependent launch)
+ * and are timed as one span from before the first to after the last.  end()
+ * waits for those events and returns, per kind k in [0, nkinds), the summed
+ * duration in ms and the number of launches:
+ *   0 = forward GEMM, 1 = backward GEMM chain, 2 = plain GEMM (diagnostic),
+ *   3 = every other kernel (compaction, gather, merge, loss, sort, db, scatter).
  */
 FLCE_API flce_status flce_diag_profile_begin(void);
 FLCE_API flce_status flce_diag_profile_end(double* ms, int64_t* launches, int nkinds);

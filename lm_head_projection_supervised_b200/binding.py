@@ -24,6 +24,7 @@ STATUS = {0: "FLCE_OK", 1: "FLCE_ERR_NULL", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_DT
 REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 FLAG_ROUND_LOGITS = 1
 FLAG_ACCUMULATE_DH = 2
+FLAG_REUSE_FORWARD = 4
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 _lib = None
@@ -65,6 +66,9 @@ def lib() -> ctypes.CDLL:
     L.flce_backward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp, i32,
                                    f32, u32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
     L.flce_backward_ex.restype = i32
+    L.flce_backward_filtered.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, vp, vp, vp,
+                                         i32, f32, u32, f32, vp, vp, f32, vp, vp, vp, vp, sz, vp]
+    L.flce_backward_filtered.restype = i32
     L.flce_shard_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, u32,
                                      vp, vp, sz, vp]
     L.flce_shard_forward.restype = i32
@@ -80,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.flce_device_status.restype = i32
     L.flce_diag_gemm.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, f32, vp, sz, vp]
     L.flce_diag_gemm.restype = i32
+    L.flce_diag_exp2.argtypes = [vp, vp, vp, i64, vp]
+    L.flce_diag_exp2.restype = i32
     L.flce_diag_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
     L.flce_diag_timeout.restype = i32
     L.flce_diag_profile_begin.argtypes = []
@@ -175,9 +181,10 @@ def _mask_u8(mask):
     return mk.contiguous()
 
 
-def _flags(round_logits=False, accumulate_dh=False) -> int:
+def _flags(round_logits=False, accumulate_dh=False, reuse_forward=False) -> int:
     return (FLAG_ROUND_LOGITS if round_logits else 0) | \
-        (FLAG_ACCUMULATE_DH if accumulate_dh else 0)
+        (FLAG_ACCUMULATE_DH if accumulate_dh else 0) | \
+        (FLAG_REUSE_FORWARD if reuse_forward else 0)
 
 
 def _vec(t, N, device):
@@ -222,12 +229,18 @@ def forward(H, W, b, labels, mask=None, ignore_index: int = -100, ws: Optional[W
 def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0, lam_dev=None,
              ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
              reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
-             round_logits: bool = False, accumulate_dh: bool = False):
-    """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex().
+             round_logits: bool = False, accumulate_dh: bool = False,
+             reuse_forward: bool = False, filter_eps: float = 0.0):
+    """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex(), or
+    flce_backward_filtered() when filter_eps > 0 (gradient filtering: 128-row x
+    64-id blocks whose |p - onehot| are all below filter_eps are left out of
+    dH and dW; an approximation).
 
     For reduction "none", grad_rows [N] is the upstream gradient of each row's
     loss; otherwise lam (or the device scalar lam_dev) is dJ/dL.  With
-    accumulate_dh the call adds its dH to out[0] instead of overwriting it."""
+    accumulate_dh the call adds its dH to out[0] instead of overwriting it.
+    reuse_forward: `ws` holds the compaction of a forward() on the same
+    inputs, untouched since; the backward skips redoing it."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
@@ -244,13 +257,17 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
         lam_dev = lam_dev.reshape(()).to(torch.float32).contiguous()
     wt = _vec(weight, N, H2.device)
     gr = _vec(grad_rows, N, H2.device)
-    st = lib().flce_backward_ex(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N,
-                                D, V, dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red,
-                                float(denom or 0.0), _flags(round_logits, accumulate_dh),
-                                float(lam), _ptr(lam_dev), _ptr(gr),
-                                _ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes,
-                                _stream(stream))
-    _check(st, "flce_backward_ex")
+    common = (_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D, V,
+              dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red, float(denom or 0.0),
+              _flags(round_logits, accumulate_dh, reuse_forward), float(lam), _ptr(lam_dev),
+              _ptr(gr))
+    tail = (_ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes, _stream(stream))
+    if filter_eps:
+        st = lib().flce_backward_filtered(*common, float(filter_eps), *tail)
+        _check(st, "flce_backward_filtered")
+    else:
+        st = lib().flce_backward_ex(*common, *tail)
+        _check(st, "flce_backward_ex")
     return dH, dW, db
 
 
@@ -386,6 +403,15 @@ def diag_gemm(A, B, M: int, N: int, K: int, a_mn: bool, b_mn: bool, scale: float
     return out
 
 
+def diag_exp2(x: torch.Tensor, stream=None):
+    """(ex2_poly(x), ex2.approx(x)) element-wise, float32 -- flce_diag_exp2()."""
+    x = x.to(torch.float32).contiguous()
+    yp, ys = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().flce_diag_exp2(_ptr(x), _ptr(yp), _ptr(ys), x.numel(), _stream(stream)),
+           "flce_diag_exp2")
+    return yp, ys
+
+
 def diag_timeout(limit_ns: int, device="cuda", stream=None) -> int:
     ws = torch.zeros(256, dtype=torch.uint8, device=device)
     _check(lib().flce_diag_timeout(_ptr(ws), 256, int(limit_ns), _stream(stream)),
@@ -411,30 +437,34 @@ def profile_end():
 class FusedLinearCrossEntropy(torch.autograd.Function):
     """L = reduce_i w_i CE(H W^T + b, y)_i over the supervised rows; gradients
     from the library's backward, with the upstream gradient kept on the
-    device (no host round trip)."""
+    device (no host round trip).  One workspace serves both passes: the
+    forward's compaction and gathered rows are kept in it for the backward."""
 
     @staticmethod
     def forward(ctx, H, W, b, labels, mask, ignore_index, weight=None, reduction="mean",
                 denom=None, round_logits=False):
-        loss, m, logs = forward(H, W, b, labels, mask, ignore_index, weight=weight,
+        H2 = H.reshape(-1, H.shape[-1])
+        ws = Workspace(H2.shape[0], H2.shape[1], W.shape[0], H.dtype, H.device)
+        loss, m, logs = forward(H, W, b, labels, mask, ignore_index, ws=ws, weight=weight,
                                 reduction=reduction, denom=denom, round_logits=round_logits)
         ctx.save_for_backward(H, W, b, labels, mask, m, logs, weight)
         ctx.ignore_index, ctx.reduction, ctx.denom = ignore_index, reduction, denom
         ctx.round_logits = round_logits
+        ctx.ws = ws
         return loss
 
     @staticmethod
     def backward(ctx, grad_out):
         H, W, b, labels, mask, m, logs, weight = ctx.saved_tensors
+        ws, ctx.ws = ctx.ws, None
         g = grad_out.detach()
+        common = dict(weight=weight, round_logits=ctx.round_logits, ws=ws, reuse_forward=True)
         if ctx.reduction == "none":
             dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs,
-                                  weight=weight, reduction="none", grad_rows=g,
-                                  round_logits=ctx.round_logits)
+                                  reduction="none", grad_rows=g, **common)
         else:
             dH, dW, db = backward(H, W, b, labels, mask, ctx.ignore_index, m, logs, lam_dev=g,
-                                  weight=weight, reduction=ctx.reduction, denom=ctx.denom,
-                                  round_logits=ctx.round_logits)
+                                  reduction=ctx.reduction, denom=ctx.denom, **common)
         return (dH.reshape(H.shape).to(H.dtype), dW.to(W.dtype),
                 None if db is None else db.to(b.dtype), None, None, None, None, None, None, None)
 

@@ -132,7 +132,8 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ H, const int* __res
 
 // Online-softmax merge of two partial states (m, s): the running update of
 // the "分块交叉熵" page §02, in the two-state form of the maths-basics page
-// (online softmax block merge).  -inf marks an empty state.
+// (online softmax block merge).  -inf marks an empty state.  Only the
+// smaller state is rescaled, so one exponential per merge.
 __device__ __forceinline__ void merge_state(float& m, float& s, float om, float os) {
   if (om == -INFINITY) return;
   if (m == -INFINITY) {
@@ -140,39 +141,73 @@ __device__ __forceinline__ void merge_state(float& m, float& s, float om, float 
     s = os;
     return;
   }
-  const float mn = fmaxf(m, om);
-  s = s * expf(m - mn) + os * expf(om - mn);
-  m = mn;
+  if (om <= m) {
+    s += os * expf(om - m);
+  } else {
+    s = s * expf(m - om) + os;
+    m = om;
+  }
 }
 
-// Per supervised row: merge the per-vocabulary-tile partials (lane-strided,
-// then a butterfly of warp shuffles, symmetric so that every lane ends with
-// the same state), then m_i, log s_i and l_i = (m_i - target_i) + log s_i.
-// loss_rows[i] = w_i l_i (compact order); lossvec[orig] = w_i l_i if given.
-__global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld, int nvt,
-                                   const float* __restrict__ tgt, const int* __restrict__ C_dev,
-                                   const int* __restrict__ idx, float* __restrict__ m_out,
-                                   float* __restrict__ logs_out, float* __restrict__ loss_rows,
-                                   const float* __restrict__ weight,
-                                   float* __restrict__ lossvec, uint32_t* err) {
-  const int C = *C_dev;
-  const int lane = threadIdx.x & 31;
-  const int warps = (blockDim.x >> 5) * gridDim.x;
-  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < C; i += warps) {
-    const float2* pr = part + static_cast<size_t>(i) * part_ld;
-    float m = -INFINITY, s = 0.f;
-    for (int v = lane; v < nvt; v += 32) {
-      const float2 ps = pr[v];
-      merge_state(m, s, ps.x, ps.y);
-    }
+// Per-tile forward partials are stored tile-major: part[v * ld + k] is the
+// (m, s) of compact row k over vocabulary tile v.  A block of 256 threads
+// merges the partials of 32 rows: thread (t, r) = (threadIdx.x / 32,
+// threadIdx.x % 32) takes tiles t, t + 8, ... of row r (each warp reads 32
+// consecutive rows of one tile: 256 contiguous bytes), then thread (0, r)
+// merges the 8 lane states in t order.  Fixed order: deterministic.
+constexpr int MERGE_ROWS = 32;
+constexpr int MERGE_SPLIT = 8;
+
+__device__ __forceinline__ float2 merge_row_tiles(const float2* __restrict__ part, int64_t ld,
+                                                  int nvt, int k, bool live,
+                                                  float2 (&sh)[MERGE_SPLIT][MERGE_ROWS]) {
+  const int r = threadIdx.x & 31, t = threadIdx.x >> 5;
+  float m = -INFINITY, s = 0.f;
+  if (live) {
+    int v = t;
+    for (; v + 3 * MERGE_SPLIT < nvt; v += 4 * MERGE_SPLIT) {  // four loads in flight
+      float2 q[4];
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const float om = __shfl_xor_sync(0xffffffffu, m, o);
-      const float os = __shfl_xor_sync(0xffffffffu, s, o);
-      merge_state(m, s, om, os);
+      for (int u = 0; u < 4; ++u) q[u] = part[static_cast<int64_t>(v + u * MERGE_SPLIT) * ld + k];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) merge_state(m, s, q[u].x, q[u].y);
     }
-    if (lane == 0) {
-      const float logs = logf(s);
+    for (; v < nvt; v += MERGE_SPLIT) {
+      const float2 q = part[static_cast<int64_t>(v) * ld + k];
+      merge_state(m, s, q.x, q.y);
+    }
+  }
+  sh[t][r] = make_float2(m, s);
+  __syncthreads();
+  float2 out = make_float2(-INFINITY, 0.f);
+  if (t == 0) {
+    float mm = -INFINITY, ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < MERGE_SPLIT; ++j) merge_state(mm, ss, sh[j][r].x, sh[j][r].y);
+    out = make_float2(mm, ss);
+  }
+  __syncthreads();
+  return out;
+}
+
+// Per supervised row: merge the per-vocabulary-tile partials, then m_i,
+// log s_i and l_i = (m_i - target_i) + log s_i.  loss_rows[i] = w_i l_i
+// (compact order); lossvec[orig] = w_i l_i if given.
+__global__ void __launch_bounds__(MERGE_ROWS * MERGE_SPLIT)
+    merge_stats_kernel(const float2* __restrict__ part, int64_t ld, int nvt,
+                       const float* __restrict__ tgt, const int* __restrict__ C_dev,
+                       const int* __restrict__ idx, float* __restrict__ m_out,
+                       float* __restrict__ logs_out, float* __restrict__ loss_rows,
+                       const float* __restrict__ weight, float* __restrict__ lossvec,
+                       uint32_t* err) {
+  __shared__ float2 sh[MERGE_SPLIT][MERGE_ROWS];
+  const int C = *C_dev;
+  for (int base = blockIdx.x * MERGE_ROWS; base < C; base += gridDim.x * MERGE_ROWS) {
+    const int i = base + (threadIdx.x & 31);
+    const float2 ms = merge_row_tiles(part, ld, nvt, i, i < C, sh);
+    if (threadIdx.x < 32 && i < C) {
+      const float m = ms.x;
+      const float logs = logf(ms.y);
       const float li = (m - tgt[i]) + logs;
       const int o = idx[i];
       m_out[o] = m;
@@ -189,37 +224,28 @@ __global__ void merge_stats_kernel(const float2* __restrict__ part, int part_ld,
 // statistics (m_r, log s_r, t_r, o_r) of the slice's columns: the merged
 // tile partials, the target logit when the slice holds the label (y_c in
 // [0, V_slice)) else 0, and the ownership flag.  Unsupervised rows (pos < 0)
-// get the recurrence's initial state (-inf, -inf, 0, 0).  One warp per row.
-__global__ void shard_stats_kernel(const float2* __restrict__ part, int part_ld, int nvt,
-                                   const float* __restrict__ tgt, const int* __restrict__ y_c,
-                                   const int* __restrict__ pos, int64_t N, int V_slice,
-                                   float4* __restrict__ stats, uint32_t* err) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       i < N; i += warps) {
-    const int k = pos[i];
-    if (k < 0) {
-      if (lane == 0) stats[i] = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
-      continue;
-    }
-    const float2* pr = part + static_cast<size_t>(k) * part_ld;
-    float m = -INFINITY, s = 0.f;
-    for (int v = lane; v < nvt; v += 32) {
-      const float2 ps = pr[v];
-      merge_state(m, s, ps.x, ps.y);
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const float om = __shfl_xor_sync(0xffffffffu, m, o);
-      const float os = __shfl_xor_sync(0xffffffffu, s, o);
-      merge_state(m, s, om, os);
-    }
-    if (lane == 0) {
-      const float logs = logf(s);
-      const bool own = static_cast<unsigned>(y_c[k]) < static_cast<unsigned>(V_slice);
-      stats[i] = make_float4(m, logs, own ? tgt[k] : 0.f, own ? 1.f : 0.f);
-      if (!isfinite(m) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
+// get the recurrence's initial state (-inf, -inf, 0, 0).  32 rows per block
+// pass, as in merge_stats_kernel.
+__global__ void __launch_bounds__(MERGE_ROWS * MERGE_SPLIT)
+    shard_stats_kernel(const float2* __restrict__ part, int64_t ld, int nvt,
+                       const float* __restrict__ tgt, const int* __restrict__ y_c,
+                       const int* __restrict__ pos, int64_t N, int V_slice,
+                       float4* __restrict__ stats, uint32_t* err) {
+  __shared__ float2 sh[MERGE_SPLIT][MERGE_ROWS];
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * MERGE_ROWS; base < N;
+       base += static_cast<int64_t>(gridDim.x) * MERGE_ROWS) {
+    const int64_t i = base + (threadIdx.x & 31);
+    const int k = i < N ? pos[i] : -1;
+    const float2 ms = merge_row_tiles(part, ld, nvt, k, k >= 0, sh);
+    if (threadIdx.x < 32 && i < N) {
+      if (k < 0) {
+        stats[i] = make_float4(-INFINITY, -INFINITY, 0.f, 0.f);
+      } else {
+        const float logs = logf(ms.y);
+        const bool own = static_cast<unsigned>(y_c[k]) < static_cast<unsigned>(V_slice);
+        stats[i] = make_float4(ms.x, logs, own ? tgt[k] : 0.f, own ? 1.f : 0.f);
+        if (!isfinite(ms.x) || !isfinite(logs)) atomicOr(err, kErrBitNonfinite);
+      }
     }
   }
 }
@@ -325,91 +351,17 @@ __global__ void __launch_bounds__(1024)
   if (threadIdx.x == 0) *scal = S;
 }
 
-// db[vp + j] = (S / sigma) * sum_{i < C} (Gp[i][j] + [y_i = vp + j] e_i) for the
-// panel's columns, in two passes with a fixed order.  e_i is what the 16-bit
-// rounding took off row i's target entry (recorded by the gradient units), so
-// the target terms enter db exactly.
-// Pass 1: block (x, s) sums 256 columns over the rows of split s (rows
-// s * ceil(C / gridDim.y) ...): warp g takes rows g, g + 8, ... of the split
-// (four rows' 16-byte loads in flight per lane, 8 columns each); the 8 warps'
-// sums are added in warp order into bpart[s][j].  A lane reads up to 7
-// columns past the panel width, inside the panel row (whose pitch is a
-// multiple of 256 columns); those columns are never written out.
-constexpr int BIAS_SPLITS = 32;
-__global__ void __launch_bounds__(256)
-    bias_partial_kernel(const uint16_t* __restrict__ Gp, int64_t ldg, int w,
-                        const int* __restrict__ C_dev, int is_bf16, int vp,
-                        const int* __restrict__ y_c, const float* __restrict__ tgt_resid,
-                        float* __restrict__ bpart) {
-  __shared__ float part[8][256];
-  const int C = *C_dev;
-  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
-  const int j0 = blockIdx.x * 256 + lane * 8;  // this lane's 8 columns
-  const int per = (C + static_cast<int>(gridDim.y) - 1) / static_cast<int>(gridDim.y);
-  const int r0 = static_cast<int>(blockIdx.y) * per;
-  const int r1 = min(C, r0 + per);
-  float acc[8];
-#pragma unroll
-  for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-  auto add_row = [&](const uint4& v, int i) {
-    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-    float g[8];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      if (is_bf16) {
-        g[2 * h] = __uint_as_float(wv[h] << 16);
-        g[2 * h + 1] = __uint_as_float(wv[h] & 0xFFFF0000u);
-      } else {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wv[h]));
-        g[2 * h] = f.x;
-        g[2 * h + 1] = f.y;
-      }
-    }
-    const int yc = __ldg(y_c + i) - vp - j0;  // the row's label among this lane's columns
-    if (static_cast<unsigned>(yc) < 8u) {
-      const float e = __ldg(tgt_resid + i);
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-        if (t == yc) g[t] += e;
-    }
-#pragma unroll
-    for (int t = 0; t < 8; ++t) acc[t] += g[t];
-  };
-  if (j0 < w) {
-    int i = r0 + grp;
-    for (; i + 24 < r1; i += 32) {  // four rows per step, loads first
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = __ldg(reinterpret_cast<const uint4*>(Gp + static_cast<int64_t>(i + 8 * u) * ldg + j0));
-#pragma unroll
-      for (int u = 0; u < 4; ++u) add_row(v[u], i + 8 * u);
-    }
-    for (; i < r1; i += 8)
-      add_row(__ldg(reinterpret_cast<const uint4*>(Gp + static_cast<int64_t>(i) * ldg + j0)), i);
-  }
-#pragma unroll
-  for (int t = 0; t < 8; ++t) part[grp][lane * 8 + t] = acc[t];
-  __syncthreads();
-  const int j = blockIdx.x * 256 + threadIdx.x;
-  if (j < w) {
-    float t = part[0][threadIdx.x];
-#pragma unroll
-    for (int k = 1; k < 8; ++k) t += part[k][threadIdx.x];
-    bpart[static_cast<int64_t>(blockIdx.y) * w + j] = t;
-  }
-}
-
-// Pass 2: db[vp + j] = (S / sigma) * sum_s bpart[s][j], splits in order.
-__global__ void bias_finish_kernel(const float* __restrict__ bpart, int splits, int w,
+// db[j] = S * acc[j] * 2^-32: the bias gradient from the fixed-point column
+// sums that the gradient units added (acc[j] = 2^32 sum_i r_i (p_ij -
+// 1[j = y_i]), exact integer additions, so the result does not depend on
+// their order); 0 when C = 0.
+__global__ void bias_finish_kernel(const unsigned long long* __restrict__ acc, int V,
                                    const int* __restrict__ C_dev, const float* __restrict__ scal,
-                                   float inv_sigma, int vp, float* __restrict__ db) {
+                                   float* __restrict__ db) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= w) return;
-  float t = 0.f;
-  for (int sp = 0; sp < splits; ++sp) t += bpart[static_cast<int64_t>(sp) * w + j];
-  const float scale = (*C_dev > 0) ? *scal * inv_sigma : 0.f;
-  db[vp + j] = t * scale;
+  if (j >= V) return;
+  const double q = static_cast<double>(static_cast<long long>(acc[j]));
+  db[j] = (*C_dev > 0) ? static_cast<float>(q * 0x1p-32 * static_cast<double>(*scal)) : 0.f;
 }
 
 // dH[i] = dH_c[pos[i]] + (S / sigma) e_k W[y_k] for supervised rows (k =
@@ -485,6 +437,89 @@ __global__ void label_sort_prep_kernel(const int* __restrict__ C_dev, const int*
     const int y = k < C ? y_c[k] : -1;
     keys[k] = (y >= 0 && y < V_slice) ? static_cast<uint32_t>(y) : static_cast<uint32_t>(V_slice);
     vals[k] = static_cast<int>(k);
+  }
+}
+
+// Stable least-significant-digit radix sort of (key, row) pairs by key, used to
+// group the supervised rows by label: 8-bit digits, one pass per digit, each
+// pass three kernels -- per-tile digit counts, one exclusive scan over the
+// counts (digit-major, so that tiles keep their order inside a digit), and a
+// scatter in which every element's rank among the equal digits of its tile
+// comes from warp match masks and per-warp counts.  All ranks are fixed by the
+// input order, so the result is the stable sort whatever the schedule.
+constexpr int RS_BITS = 8;
+constexpr int RS_DIGITS = 1 << RS_BITS;
+constexpr int RS_TILE = 1024;  // one element per thread
+
+__global__ void __launch_bounds__(RS_TILE)
+    radix_count_kernel(const uint32_t* __restrict__ keys, int64_t n, int shift,
+                       int* __restrict__ counts) {
+  __shared__ int h[RS_DIGITS];
+  for (int d = threadIdx.x; d < RS_DIGITS; d += blockDim.x) h[d] = 0;
+  __syncthreads();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * RS_TILE + threadIdx.x;
+  if (i < n) atomicAdd(&h[(keys[i] >> shift) & (RS_DIGITS - 1)], 1);
+  __syncthreads();
+  for (int d = threadIdx.x; d < RS_DIGITS; d += blockDim.x)
+    counts[static_cast<int64_t>(d) * gridDim.x + blockIdx.x] = h[d];
+}
+
+// In-place exclusive scan of `total` ints with one block: each thread scans a
+// contiguous run, then the runs' sums are scanned across the block.
+__global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ a, int64_t total) {
+  __shared__ int sums[1024];
+  const int t = threadIdx.x;
+  const int64_t per = (total + blockDim.x - 1) / blockDim.x;
+  const int64_t b0 = t * per, b1 = min(total, b0 + per);
+  int run = 0;
+  for (int64_t i = b0; i < b1; ++i) run += a[i];
+  sums[t] = run;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan of the run sums
+    const int v = t >= off ? sums[t - off] : 0;
+    __syncthreads();
+    sums[t] += v;
+    __syncthreads();
+  }
+  int acc = sums[t] - run;
+  for (int64_t i = b0; i < b1; ++i) {
+    const int v = a[i];
+    a[i] = acc;
+    acc += v;
+  }
+}
+
+__global__ void __launch_bounds__(RS_TILE)
+    radix_scatter_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ vals,
+                         int64_t n, int shift, const int* __restrict__ offsets,
+                         uint32_t* __restrict__ keys_out, int* __restrict__ vals_out) {
+  constexpr int NW = RS_TILE / 32;
+  __shared__ int cnt[NW][RS_DIGITS];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j = threadIdx.x; j < NW * RS_DIGITS; j += blockDim.x) (&cnt[0][0])[j] = 0;
+  __syncthreads();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * RS_TILE + threadIdx.x;
+  const bool live = i < n;
+  const uint32_t k = live ? keys[i] : 0u;
+  const int d = live ? static_cast<int>((k >> shift) & (RS_DIGITS - 1)) : RS_DIGITS;
+  const unsigned peers = __match_any_sync(0xffffffffu, d);
+  const int below = __popc(peers & ((1u << lane) - 1u));
+  if (live && below == 0) cnt[warp][d] = __popc(peers);
+  __syncthreads();
+  if (threadIdx.x < RS_DIGITS) {  // per digit: counts of the earlier warps
+    int run = 0;
+    for (int w = 0; w < NW; ++w) {
+      const int c = cnt[w][threadIdx.x];
+      cnt[w][threadIdx.x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (live) {
+    const int64_t dst = offsets[static_cast<int64_t>(d) * gridDim.x + blockIdx.x] +
+                        cnt[warp][d] + below;
+    keys_out[dst] = k;
+    vals_out[dst] = vals[i];
   }
 }
 
@@ -577,6 +612,16 @@ __global__ void dw_target_resid_kernel(const uint32_t* __restrict__ keys,
                          fmaf(scale, a3, o.w));
     }
   }
+}
+
+// Accuracy check of the two exponentials the epilogues use: y_poly = ex2_poly(x),
+// y_sfu = ex2.approx(x), element-wise.
+__global__ void exp2_probe_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                  float* __restrict__ y_sfu, int64_t n) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  y_poly[i] = ex2_poly(x[i]);
+  y_sfu[i] = ex2_approx(x[i]);
 }
 
 // Failure-path check: waits on a barrier nothing completes, with a short

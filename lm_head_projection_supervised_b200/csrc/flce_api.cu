@@ -4,21 +4,24 @@
 // Forward  (one stream, no host synchronisation):
 //   compact -> gather H_c -> gemm<fwd> (Z tiles + online (m, s) + target)
 //   -> merge partials per row -> fixed-order loss reduction
-// Backward, with P vocabulary panels of Vc columns and two panel buffers:
-//   compact -> gather H_c ->
+// Backward, with P vocabulary panels of Vc columns and three panel buffers:
+//   compact -> gather H_c (skipped when reusing the forward's) ->
 //   for L = 0 .. P:   gemm<bwd> with
-//                       grad units of panel L     (if L < P) -> buffer L % 2
-//                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 2
-//                     db of panel L in two passes (bias only, if L < P)
-//   -> rows grouped by label (stable radix sort) -> dW target terms in fp32
+//                       grad units of panel L     (if L < P) -> buffer L % 3
+//                         (+ the bias gradient's fixed-point column sums)
+//                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 3
+//                     launches L >= 1 may start while launch L-1 runs
+//                     (programmatic dependent launch): their gradient units
+//                     overlap its tail, their dW / dH units wait for it
+//   -> db from the column sums (bias only)
+//   -> rows grouped by label (stable radix sort, own kernels) -> dW target
+//      terms in fp32
 //   -> scatter dH_c to dH with its target terms (zero rows for unsupervised
 //      positions)
 //   with row scales s_k = S r_k computed first (row_scale_kernel); the panels
 //   hold r_k (p - onehot) sigma and the dW / dH epilogues multiply by S / sigma.
 #include <mutex>
 #include <vector>
-
-#include <cub/device/device_radix_sort.cuh>
 
 #include "../../include/flce.h"
 #include "../../include/flce_diag.h"
@@ -38,15 +41,24 @@ constexpr int kMaxShards = 4096;  // vocabulary slices merged by one combine
 #endif
 constexpr int64_t kPanelCols = FLCE_PANEL_COLS;  // vocabulary columns per gradient panel
 constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
+#ifndef FLCE_POLY_EXP_MAX_D
+#define FLCE_POLY_EXP_MAX_D 256
+#endif
+// Up to this hidden size the epilogues' exponentials, not the tensor core,
+// bound the score tiles: one in four then goes to the FMA pipe (ex2_poly).
+constexpr int64_t kPolyExpMaxD = FLCE_POLY_EXP_MAX_D;
 constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
 int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t roundup64(int64_t a, int64_t b) { return cdiv64(a, b) * b; }
 
+constexpr int kPanelBufs = 3;  // panel buffers: written, read, and one of slack for the overlap
+
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, rs, resid, skeys[2], svals[2], cubtmp, cub_bytes, bpart, dhc, gpanel[2], total;
-  int64_t Np, nvt, nparts, vc, gld, panels;
+  size_t pos, rs, resid, skeys[2], svals[2], rscount, dbacc, keep, keep_bytes, dhc;
+  size_t gpanel[kPanelBufs], total;
+  int64_t Np, nvt, vc, gld, panels;
 };
 
 // Workspace carve-up.  The control block (error word, then one work counter
@@ -55,8 +67,7 @@ struct Layout {
 Layout make_layout(int64_t N, int64_t D, int64_t V) {
   Layout L{};
   L.Np = roundup64(N > 0 ? N : 1, PAIR_M);  // every half-tile of a CTA pair starts inside
-  L.nvt = cdiv64(V, BN);
-  L.nparts = L.nvt * NUM_EPI_WG;  // forward (m, s) partials per row: one per half tile
+  L.nvt = cdiv64(V, BN);  // forward (m, s) partials per row: one per vocabulary tile
   L.vc = roundup64(V, BN) < kPanelCols ? roundup64(V, BN) : kPanelCols;
   L.panels = cdiv64(V, L.vc);
   L.gld = L.vc;  // gradient-panel row pitch in elements
@@ -72,24 +83,25 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.idx = take(static_cast<size_t>(L.Np) * 4);
   L.yc = take(static_cast<size_t>(L.Np) * 4);
   L.hc = take(static_cast<size_t>(L.Np) * D * 2);
-  L.part = take(static_cast<size_t>(L.Np) * L.nparts * 8);
+  L.part = take(static_cast<size_t>(L.Np) * L.nvt * 8);  // tile-major [nvt][Np]
   L.tgt = take(static_cast<size_t>(L.Np) * 4);
   L.loss_rows = take(static_cast<size_t>(L.Np) * 4);
   L.pos = take(static_cast<size_t>(L.Np) * 4);
   L.fwd_total = off;
   L.rs = take(static_cast<size_t>(L.Np) * 4);
   L.resid = take(static_cast<size_t>(L.Np) * 4);
-  // rows grouped by label (stable radix sort, ping-pong buffers + CUB's scratch)
+  // rows grouped by label (stable radix sort: ping-pong buffers, digit counts per tile)
   for (int i = 0; i < 2; ++i) {
     L.skeys[i] = take(static_cast<size_t>(L.Np) * 4);
     L.svals[i] = take(static_cast<size_t>(L.Np) * 4);
   }
-  L.cub_bytes = static_cast<size_t>(L.Np) * 4 + (size_t(4) << 20);
-  L.cubtmp = take(L.cub_bytes);
-  L.bpart = take(static_cast<size_t>(BIAS_SPLITS) * L.vc * 4);  // db partials of one panel
+  L.rscount = take(static_cast<size_t>(RS_DIGITS) * cdiv64(L.Np, RS_TILE) * 4);
+  L.dbacc = take(static_cast<size_t>(V) * 8);  // bias gradient, fixed point per vocabulary id
+  // gradient filtering: one keep flag per 128-row x 64-column box of each panel buffer
+  L.keep_bytes = static_cast<size_t>(L.Np / BM) * static_cast<size_t>(L.gld / 64);
+  L.keep = take(L.keep_bytes * kPanelBufs);
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
-  L.gpanel[0] = take(static_cast<size_t>(L.Np) * L.gld * 2);
-  L.gpanel[1] = take(static_cast<size_t>(L.Np) * L.gld * 2);
+  for (int i = 0; i < kPanelBufs; ++i) L.gpanel[i] = take(static_cast<size_t>(L.Np) * L.gld * 2);
   L.total = off;
   return L;
 }
@@ -232,6 +244,7 @@ flce_status device_setup(DevInfo* out) {
 // ---- optional per-launch timing (diagnostic; off unless profile_begin)
 struct ProfRec {
   int kind;
+  int launches;  // kernels between the two events
   cudaEvent_t start, stop;
 };
 std::mutex g_prof_mu;
@@ -253,7 +266,7 @@ cudaError_t timed_launch(int kind, cudaStream_t s, F&& launch) {
     launch();
     return cudaGetLastError();
   }
-  ProfRec r{kind, nullptr, nullptr};
+  ProfRec r{kind, 1, nullptr, nullptr};
   if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess)
     return cudaErrorUnknown;
   cudaEventRecord(r.start, s);
@@ -265,27 +278,59 @@ cudaError_t timed_launch(int kind, cudaStream_t s, F&& launch) {
   return e;
 }
 
+// A timed span of several launches that overlap one another (the backward's
+// chain of GEMM launches): one event before the first and one after the last,
+// none in between.  begin returns false when profiling is off.
+bool prof_span_begin(ProfRec* r, int kind, cudaStream_t s) {
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_on) return false;
+  }
+  *r = ProfRec{kind, 0, nullptr, nullptr};
+  if (cudaEventCreate(&r->start) != cudaSuccess || cudaEventCreate(&r->stop) != cudaSuccess)
+    return false;
+  cudaEventRecord(r->start, s);
+  return true;
+}
+void prof_span_end(ProfRec* r, int launches, cudaStream_t s) {
+  r->launches = launches;
+  cudaEventRecord(r->stop, s);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof.push_back(*r);
+}
+
 // Persistent launch of CTA pairs: min(work units, resident pairs) clusters of 2.
+// pdl: the launch may start before the previous kernel of the stream ends
+// (programmatic stream serialisation; the kernel waits where it must).
+// timed: wrap the launch in profiling events (off inside a timed span).
 template <int MODE>
-cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaStream_t s) {
+cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaStream_t s,
+                        bool pdl = false, bool timed = true) {
   if (units_upper <= 0) return cudaSuccess;
   const int npairs = static_cast<int>(units_upper < pairs ? units_upper : pairs);
   const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeBwd ? kProfBwd : kProfPlain;
-  return timed_launch(kind, s, [&] {
+  auto launch = [&] {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
     cfg.blockDim = dim3(NUM_THREADS);
     cfg.dynamicSmemBytes = ModeCfg<MODE>::SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     cudaLaunchKernelEx(&cfg, flce_gemm_kernel<MODE>, a);
-  });
+  };
+  if (!timed) {
+    launch();
+    return cudaGetLastError();
+  }
+  return timed_launch(kind, s, launch);
 }
 
 struct WsPtrs {
@@ -304,10 +349,11 @@ struct WsPtrs {
   float* resid;
   uint32_t* skeys[2];
   int* svals[2];
-  void* cubtmp;
-  float* bpart;
+  int* rscount;
+  unsigned long long* dbacc;
+  uint8_t* keep;
   float* dhc;
-  uint16_t* gpanel[2];
+  uint16_t* gpanel[kPanelBufs];
 };
 
 WsPtrs carve(void* ws, const Layout& L) {
@@ -330,20 +376,26 @@ WsPtrs carve(void* ws, const Layout& L) {
     p.skeys[i] = reinterpret_cast<uint32_t*>(w + L.skeys[i]);
     p.svals[i] = reinterpret_cast<int*>(w + L.svals[i]);
   }
-  p.cubtmp = w + L.cubtmp;
-  p.bpart = reinterpret_cast<float*>(w + L.bpart);
+  p.rscount = reinterpret_cast<int*>(w + L.rscount);
+  p.dbacc = reinterpret_cast<unsigned long long*>(w + L.dbacc);
+  p.keep = w + L.keep;
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
-  p.gpanel[0] = reinterpret_cast<uint16_t*>(w + L.gpanel[0]);
-  p.gpanel[1] = reinterpret_cast<uint16_t*>(w + L.gpanel[1]);
+  for (int i = 0; i < kPanelBufs; ++i) p.gpanel[i] = reinterpret_cast<uint16_t*>(w + L.gpanel[i]);
   return p;
 }
 
-// control block reset + compaction + gather of the supervised rows
+// control block reset + compaction + gather of the supervised rows.  With
+// `reuse` (a forward on this workspace already did both) only the work
+// counters are reset; the error word keeps what the forward recorded.
 flce_status prologue(const void* H, const int64_t* labels, const uint8_t* mask, int64_t ignore,
                      int64_t N, int64_t D, int64_t V, int64_t v0, int64_t V_slice,
                      const Layout& L, const WsPtrs& p,
                      float* m_out, float* logs_out, int* pos, float* lossvec,
-                     cudaStream_t s) {
+                     cudaStream_t s, bool reuse = false) {
+  if (reuse) {
+    FLCE_CK(cudaMemsetAsync(p.counters, 0, L.ctrl_bytes - kCounterOffset, s));
+    return FLCE_OK;
+  }
   FLCE_CK(cudaMemsetAsync(p.err, 0, L.ctrl_bytes, s));
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     compact_kernel<<<1, COMPACT_THREADS, 0, s>>>(labels, mask, ignore, N, V, v0, V_slice, p.idx,
@@ -398,8 +450,9 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   const MapType mt = bf16 ? kMapBF16 : kMapFP16;
 
   float* lossvec = none ? loss_rows : nullptr;
+  // the row map (pos) is kept for a backward that reuses this compaction
   st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, V, L, p, shard ? nullptr : m,
-                shard ? nullptr : logs, shard ? p.pos : nullptr, lossvec, s);
+                shard ? nullptr : logs, p.pos, lossvec, s);
   if (st != FLCE_OK) return st;
 
   GemmArgs a{};
@@ -417,28 +470,31 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   a.idx = p.idx;
   a.bias = static_cast<const uint16_t*>(b);
   a.part = p.part;
-  a.part_ld = static_cast<int>(L.nparts);
+  a.part_ld = static_cast<int>(L.Np);
   a.tgt = p.tgt;
   a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
+  a.poly_exp = D <= kPolyExpMaxD ? 1 : 0;
   a.err = p.err;
   FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
-  const int64_t blocks = cdiv64(N, 8) < 8LL * di.sms ? cdiv64(N, 8) : 8LL * di.sms;
+  // 32 rows per block pass, at most 8 blocks per SM
+  const int64_t blocks =
+      cdiv64(N, MERGE_ROWS) < 8LL * di.sms ? cdiv64(N, MERGE_ROWS) : 8LL * di.sms;
   if (shard) {
     if (N > 0) {
       FLCE_CK(timed_launch(kProfAux, s, [&] {
-        shard_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            p.part, static_cast<int>(L.nparts), static_cast<int>(L.nparts), p.tgt, p.yc, p.pos, N,
-            static_cast<int>(V), stats, p.err);
+        shard_stats_kernel<<<static_cast<unsigned>(blocks), MERGE_ROWS * MERGE_SPLIT, 0, s>>>(
+            p.part, L.Np, static_cast<int>(L.nvt), p.tgt, p.yc, p.pos, N, static_cast<int>(V),
+            stats, p.err);
       }));
     }
     return FLCE_OK;
   }
   if (N > 0) {
     FLCE_CK(timed_launch(kProfAux, s, [&] {
-      merge_stats_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-          p.part, static_cast<int>(L.nparts), static_cast<int>(L.nparts), p.tgt, p.C, p.idx, m, logs,
-          p.loss_rows, weight, lossvec, p.err);
+      merge_stats_kernel<<<static_cast<unsigned>(blocks), MERGE_ROWS * MERGE_SPLIT, 0, s>>>(
+          p.part, L.Np, static_cast<int>(L.nvt), p.tgt, p.C, p.idx, m, logs, p.loss_rows, weight,
+          lossvec, p.err);
     }));
   }
   if (!none) {
@@ -458,11 +514,13 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
                           int64_t V, int64_t v0, int64_t V_total, int dtype, const float* m,
                           const float* logs, const float* weight, int reduction, float denom,
                           unsigned flags, float lambda, const float* lambda_dev,
-                          const float* grad_rows, float* dH, float* dW, float* db, void* ws,
-                          size_t ws_bytes, cudaStream_t s) {
+                          const float* grad_rows, float filter_eps, float* dH, float* dW,
+                          float* db, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (!(filter_eps >= 0.f) || !isfinite(filter_eps)) return FLCE_ERR_ARG;
   if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
        reduction != FLCE_REDUCE_NONE) ||
-      (flags & ~(FLCE_FLAG_ROUND_LOGITS | FLCE_FLAG_ACCUMULATE_DH)) != 0)
+      (flags & ~(FLCE_FLAG_ROUND_LOGITS | FLCE_FLAG_ACCUMULATE_DH | FLCE_FLAG_REUSE_FORWARD)) !=
+          0)
     return FLCE_ERR_ARG;
   const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
@@ -488,19 +546,10 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
   const float log2_sigma = bf16 ? 0.f : kFp16Log2Sigma;
   const float sigma = exp2f(log2_sigma);
 
-  // the label sort's scratch (checked before any work is enqueued)
   int end_bit = 1;
   while ((int64_t(1) << end_bit) <= V) ++end_bit;  // sort keys are 0 .. V
-  size_t need = 0;
-  {
-    cub::DoubleBuffer<uint32_t> k0(p.skeys[0], p.skeys[1]);
-    cub::DoubleBuffer<int> v0buf(p.svals[0], p.svals[1]);
-    FLCE_CK(cub::DeviceRadixSort::SortPairs(nullptr, need, k0, v0buf, static_cast<int>(L.Np), 0,
-                                            end_bit, s));
-    if (need > L.cub_bytes) return FLCE_ERR_WORKSPACE;
-  }
   st = prologue(H, labels, mask, ignore_index, N, D, V_total, v0, V, L, p, nullptr, nullptr,
-                p.pos, nullptr, s);
+                p.pos, nullptr, s, (flags & FLCE_FLAG_REUSE_FORWARD) != 0);
   if (st != FLCE_OK) return st;
   FLCE_CK(timed_launch(kProfAux, s, [&] {
     row_scale_kernel<<<1, 1024, 0, s>>>(p.C, p.idx, weight, none ? grad_rows : nullptr,
@@ -521,6 +570,13 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
 
   const int64_t nT_max = cdiv64(N, PAIR_M);
   const int64_t nD = cdiv64(D, BN);
+  if (b != nullptr) FLCE_CK(cudaMemsetAsync(p.dbacc, 0, static_cast<size_t>(V) * 8, s));
+  // The GEMM launches form one timed span: with programmatic dependent launch
+  // they overlap, so events between them would measure nothing useful (and
+  // would hold the next launch back).
+  ProfRec span;
+  const bool timed = prof_span_begin(&span, kProfBwd, s);
+  int launched = 0;
   for (int64_t Lp = 0; Lp <= L.panels; ++Lp) {
     const bool has_g = Lp < L.panels;
     const bool has_wh = Lp > 0;
@@ -536,10 +592,11 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.tmB[kClsDH] = wMN;
     a.tmDW = dwMap;
     a.tmDH = dhMap;
-    if (has_g && !make_map(&a.tmG, p.gpanel[Lp & 1], mt, w_g, L.Np, L.gld * 2, 64, BM))
+    if (has_g &&
+        !make_map(&a.tmG, p.gpanel[Lp % kPanelBufs], mt, w_g, L.Np, L.gld * 2, 64, BM))
       return FLCE_ERR_CUDA;
     if (has_wh) {
-      const uint16_t* gp = p.gpanel[(Lp - 1) & 1];
+      const uint16_t* gp = p.gpanel[(Lp - 1) % kPanelBufs];
       if (!make_map(&a.tmA[kClsDW], gp, mt, w_wh, L.Np, L.gld * 2, 64, BK) ||
           !make_map(&a.tmA[kClsDH], gp, mt, w_wh, L.Np, L.gld * 2, BK, BM))
         return FLCE_ERR_CUDA;
@@ -567,25 +624,32 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.tgt_resid = p.resid;
     a.scal = p.scal;
     a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
+    a.poly_exp = D <= kPolyExpMaxD ? 1 : 0;
     a.inv_sigma = 1.f / sigma;
+    a.db_acc = b != nullptr ? p.dbacc : nullptr;
+    a.db_fx_scale = 0x1p32f / sigma;
+    if (filter_eps > 0.f) {
+      a.filter_eps_sigma = filter_eps * sigma;
+      a.keep_ld = static_cast<int>(L.gld / 64);
+      a.keep_g = has_g ? p.keep + L.keep_bytes * (Lp % kPanelBufs) : nullptr;
+      a.keep_wh = has_wh ? p.keep + L.keep_bytes * ((Lp - 1) % kPanelBufs) : nullptr;
+      // a launch without gradient units still reads flags: keep_g stays null
+      // there, so the kernel tests keep_wh for the consumers
+    }
     a.err = p.err;
     const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +
                           (has_g ? nT_max * cdiv64(w_g, BN) : 0);
-    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.pairs, s));
-
-    if (b != nullptr && has_g) {
-      const uint16_t* gp = p.gpanel[Lp & 1];
-      FLCE_CK(timed_launch(kProfAux, s, [&] {
-        bias_partial_kernel<<<dim3(static_cast<unsigned>(cdiv64(w_g, 256)), BIAS_SPLITS), 256, 0,
-                              s>>>(gp, L.gld, static_cast<int>(w_g), p.C, bf16 ? 1 : 0,
-                                   static_cast<int>(vp_g), p.yc, p.resid, p.bpart);
-      }));
-      FLCE_CK(timed_launch(kProfAux, s, [&] {
-        bias_finish_kernel<<<static_cast<unsigned>(cdiv64(w_g, 256)), 256, 0, s>>>(
-            p.bpart, BIAS_SPLITS, static_cast<int>(w_g), p.C, p.scal, 1.f / sigma,
-            static_cast<int>(vp_g), db);
-      }));
-    }
+    // every launch after the first may overlap its predecessor
+    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.pairs, s, /*pdl=*/launched > 0,
+                                  /*timed=*/false));
+    launched += units > 0 ? 1 : 0;
+  }
+  if (timed) prof_span_end(&span, launched, s);
+  if (b != nullptr) {
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      bias_finish_kernel<<<static_cast<unsigned>(cdiv64(V, 256)), 256, 0, s>>>(
+          p.dbacc, static_cast<int>(V), p.C, p.scal, db);
+    }));
   }
   if (N > 0) {
     // dW's target terms in fp32: group the rows by label (stable sort), then
@@ -595,17 +659,27 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       label_sort_prep_kernel<<<static_cast<unsigned>(pblocks), 256, 0, s>>>(
           p.C, p.yc, L.Np, static_cast<int>(V), p.skeys[0], p.svals[0]);
     }));
-    cub::DoubleBuffer<uint32_t> dkeys(p.skeys[0], p.skeys[1]);
-    cub::DoubleBuffer<int> dvals(p.svals[0], p.svals[1]);
-    FLCE_CK(timed_launch(kProfAux, s, [&] {
-      cub::DeviceRadixSort::SortPairs(p.cubtmp, need, dkeys, dvals, static_cast<int>(L.Np), 0,
-                                      end_bit, s);
-    }));
+    int cur = 0;
+    const unsigned tiles = static_cast<unsigned>(cdiv64(L.Np, RS_TILE));
+    for (int shift = 0; shift < end_bit; shift += RS_BITS) {
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+        radix_count_kernel<<<tiles, RS_TILE, 0, s>>>(p.skeys[cur], L.Np, shift, p.rscount);
+      }));
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+        radix_scan_kernel<<<1, 1024, 0, s>>>(p.rscount, static_cast<int64_t>(RS_DIGITS) * tiles);
+      }));
+      FLCE_CK(timed_launch(kProfAux, s, [&] {
+        radix_scatter_kernel<<<tiles, RS_TILE, 0, s>>>(p.skeys[cur], p.svals[cur], L.Np, shift,
+                                                       p.rscount, p.skeys[cur ^ 1],
+                                                       p.svals[cur ^ 1]);
+      }));
+      cur ^= 1;
+    }
     const int64_t rwarps = L.Np * cdiv64(D / 4, 32);
     const int64_t rblocks = cdiv64(rwarps, 8) < 16LL * di.sms ? cdiv64(rwarps, 8) : 16LL * di.sms;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       dw_target_resid_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
-          dkeys.Current(), dvals.Current(), L.Np, static_cast<int>(V),
+          p.skeys[cur], p.svals[cur], L.Np, static_cast<int>(V),
           reinterpret_cast<const uint2*>(p.hc), D / 4, bf16 ? 1 : 0, p.resid, p.scal,
           1.f / sigma, reinterpret_cast<float4*>(dW));
     }));
@@ -777,8 +851,21 @@ flce_status flce_backward_ex(const void* H, const void* W, const void* b, const 
                              float* dW, float* db, void* ws, size_t ws_bytes,
                              flce_stream stream) {
   return backward_impl(H, W, b, labels, mask, ignore_index, N, D, V, 0, V, dtype, m, logs, weight,
-                       reduction, denom, flags, lambda, lambda_dev, grad_rows, dH, dW, db, ws,
-                       ws_bytes, static_cast<cudaStream_t>(stream));
+                       reduction, denom, flags, lambda, lambda_dev, grad_rows, 0.f, dH, dW, db,
+                       ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+flce_status flce_backward_filtered(const void* H, const void* W, const void* b,
+                                   const int64_t* labels, const uint8_t* mask,
+                                   int64_t ignore_index, int64_t N, int64_t D, int64_t V,
+                                   int dtype, const float* m, const float* logs,
+                                   const float* weight, int reduction, float denom,
+                                   unsigned flags, float lambda, const float* lambda_dev,
+                                   const float* grad_rows, float filter_eps, float* dH, float* dW,
+                                   float* db, void* ws, size_t ws_bytes, flce_stream stream) {
+  return backward_impl(H, W, b, labels, mask, ignore_index, N, D, V, 0, V, dtype, m, logs, weight,
+                       reduction, denom, flags, lambda, lambda_dev, grad_rows, filter_eps, dH,
+                       dW, db, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 flce_status flce_shard_backward(const void* H, const void* W_slice, const void* b_slice,
@@ -791,7 +878,7 @@ flce_status flce_shard_backward(const void* H, const void* W_slice, const void* 
                                 size_t ws_bytes, flce_stream stream) {
   return backward_impl(H, W_slice, b_slice, labels, mask, ignore_index, N, D, V_slice, v0,
                        V_total, dtype, m, logs, weight, reduction, denom, flags, lambda,
-                       lambda_dev, grad_rows, dH, dW_slice, db_slice, ws, ws_bytes,
+                       lambda_dev, grad_rows, 0.f, dH, dW_slice, db_slice, ws, ws_bytes,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -845,6 +932,21 @@ flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, 
   return FLCE_OK;
 }
 
+flce_status flce_diag_exp2(const float* x, float* y_poly, float* y_sfu, int64_t n,
+                           flce_stream stream) {
+  if (n > 0 && (x == nullptr || y_poly == nullptr || y_sfu == nullptr)) return FLCE_ERR_NULL;
+  if (n < 0 || n > (int64_t(1) << 31)) return FLCE_ERR_SHAPE;
+  if (n == 0) return FLCE_OK;
+  DevInfo di;
+  const flce_status st = device_setup(&di);
+  if (st != FLCE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FLCE_CK(timed_launch(kProfAux, s, [&] {
+    exp2_probe_kernel<<<static_cast<unsigned>(cdiv64(n, 256)), 256, 0, s>>>(x, y_poly, y_sfu, n);
+  }));
+  return FLCE_OK;
+}
+
 flce_status flce_diag_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, flce_stream stream) {
   if (ws == nullptr) return FLCE_ERR_NULL;
   if (!aligned(ws, 256)) return FLCE_ERR_ALIGN;
@@ -887,7 +989,7 @@ flce_status flce_diag_profile_end(double* ms, int64_t* launches, int nkinds) {
       st = FLCE_ERR_CUDA;
     if (r.kind < nkinds) {
       ms[r.kind] += t;
-      launches[r.kind] += 1;
+      launches[r.kind] += r.launches;
     }
     cudaEventDestroy(r.start);
     cudaEventDestroy(r.stop);
@@ -904,23 +1006,17 @@ flce_status flce_diag_profile_end(double* ms, int64_t* launches, int nkinds) {
 // ---------------------------------------------------------------------------
 namespace {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (host code cannot use the symbol itself as a device pointer).
+// Device address of g_noalloc_scratch on the current device (host code cannot
+// use the symbol itself as a device pointer).  Looked up on every call, with
+// the device current: the lookup allocates nothing, and an address kept from
+// an earlier call could be stale after a reset of the device's primary context
+// (the module, and with it the array, is loaded again).
 flce_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return FLCE_ERR_DEVICE;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return FLCE_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return FLCE_ERR_CUDA;
+  *out = p;
   return FLCE_OK;
 }
 }  // namespace

@@ -20,17 +20,24 @@
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
 //              running max / rescaled exp-sum over the tile's columns and
 //              captures the target logit from the tile that holds it
-//              ("分块交叉熵" page, §02), writing one (m, s) partial per row
-//              and half tile (one per epilogue warpgroup).
+//              ("分块交叉熵" page, §02); the two warpgroups' halves of a row
+//              are merged in shared memory and one (m, s) partial per row and
+//              tile is stored, tile-major (a warp's 32 rows are contiguous).
 //   kModeBwd   three unit classes in one launch, with no dependency between
-//              them:
+//              them (the gradient units first: they need nothing from the
+//              previous launch, which may still be running -- programmatic
+//              dependent launch -- and the producers wait for it before
+//              their first dW / dH unit):
 //              class 2 (grad): the tile of vocabulary panel p recomputed; the
 //                 epilogue rebuilds p = exp((Z - m) - log s) from the saved
 //                 statistics, subtracts the one-hot target (§04), rounds to
 //                 the 16-bit input type, stages 128 x 64 boxes in shared
 //                 memory and stores them with TMA into gradient buffer p % 2,
 //                 and records what the rounding took off each row's target
-//                 entry (added back in fp32 to dH, dW and db later);
+//                 entry (added back in fp32 to dH and dW later); with a bias,
+//                 the fp32 column sums of its rows go to the bias gradient
+//                 as 64-bit fixed-point integer additions (order-free, so
+//                 deterministic);
 //              The panel holds r_k (p - onehot) sigma with the row scale
 //              s_k = S r_k (S = max |s_k|), the contractions multiply by S / sigma.
 //              class 0 (dW): dW[panel p-1 rows] = G^T H_c  (K = C), stored by TMA;
@@ -73,7 +80,7 @@ constexpr int EPI_CHUNKS = BN / 32 / NUM_EPI_WG;  // 32-column chunks per epilog
 // Registers per thread after the split: the first warpgroup gives up what the
 // epilogue takes.  The block is launched with at least kRegsAtLaunch per
 // thread (checked on the host before any launch), which covers the split.
-constexpr uint32_t kRegsLow = 56;
+constexpr uint32_t kRegsLow = 72;
 constexpr uint32_t kRegsHigh = 216;
 constexpr uint32_t kRegsAtLaunch =
     (128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh + NUM_THREADS - 1) / NUM_THREADS;
@@ -89,8 +96,12 @@ template <int MODE>
 struct ModeCfg {
   static constexpr int STAGES = (MODE == kModeBwd) ? 6 : 7;
   static constexpr uint32_t STAGING = (MODE == kModeBwd) ? NUM_EPI_WG * STG_BYTES : 0;
+  // forward: one (m, s) pair per row of the CTA's half tile, to merge the two
+  // epilogue warpgroups' column halves
+  static constexpr uint32_t MERGE = (MODE == kModeFwd) ? BM * 8 : 0;
   static constexpr size_t SMEM_BYTES =
-      1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + STAGING + 512;
+      1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + STAGING + 512 + MERGE;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 constexpr size_t GEMM_SMEM_BYTES = ModeCfg<kModeBwd>::SMEM_BYTES;  // the largest
 enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
@@ -120,7 +131,9 @@ struct GemmArgs {
   const int* idx;          // compact row -> original row
   const uint16_t* bias;    // 16-bit bias [V] or null
   int round_logits;        // round each logit to the 16-bit input type first
-  float2* part;            // fwd: (m, s) partials [rows][part_ld]
+  int poly_exp;            // one exponential in four on the FMA pipe (ex2_poly): for small
+                           // D, where the epilogue's exponentials outrun the tensor core
+  float2* part;            // fwd: (m, s) partials [tiles][part_ld], part_ld >= rows
   int part_ld;
   float* tgt;              // fwd: target logits [rows]
   const float* m_saved;    // bwd: saved statistics [N]
@@ -132,6 +145,17 @@ struct GemmArgs {
                            //      panel value (written by the tile that holds the label)
   const float* scal;       // bwd: S (device scalar); G = S r_k (p - onehot)
   float inv_sigma;
+  unsigned long long* db_acc;  // bwd, bias only (else null): per vocabulary id, the sum of
+                               //      the column's r_k (p - onehot) in 2^-32 fixed point
+  float db_fx_scale;           // bwd: 2^32 / sigma (panel units -> fixed point)
+  // bwd, gradient filtering (keep_g / keep_wh null when off): a 128-row x
+  // 64-column box of the panel whose every |p - onehot| sigma is below
+  // filter_eps_sigma is dropped: stored as zeros and flagged 0, and the dW /
+  // dH units skip the k-blocks whose boxes are all dropped.
+  float filter_eps_sigma;
+  uint8_t* keep_g;             // flags of the panel being produced [Np / 128][keep_ld]
+  const uint8_t* keep_wh;      // flags of the panel being read
+  int keep_ld;                 // boxes per 128-row half (panel pitch / 64)
   float* out;              // plain
   float scale;             // plain
   uint32_t* err;
@@ -170,15 +194,12 @@ __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
     s.k0 = cdiv_i(C, BK);
     s.k1 = cdiv_i(g.w_wh, BK);
     s.k2 = cdiv_i(g.D, BK);
-    // order the three classes by K-blocks per unit, longest first (stable)
-    int a = 0, b = 1, c = 2;
-    int ka = s.k0, kb = s.k1, kc = s.k2;
-    if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
-    if (kb < kc) { int t = b; b = c; c = t; t = kb; kb = kc; kc = t; }
-    if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
-    s.o0 = a;
-    s.o1 = b;
-    s.o2 = c;
+    // The gradient units first: they depend on nothing the previous launch
+    // produces, so they fill the SMs while its last units finish.  Then dW
+    // and dH, longer units first.
+    s.o0 = kClsGrad;
+    s.o1 = (s.k0 >= s.k1) ? kClsDW : kClsDH;
+    s.o2 = (s.k0 >= s.k1) ? kClsDH : kClsDW;
     s.total = s.n0 + s.n1 + s.n2;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
@@ -240,6 +261,22 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
   if (MODE == kModeBwd) return un.cls != kClsGrad;
   if (MODE == kModePlain) return g.b_mn != 0;
   return false;
+}
+
+// Gradient filtering: whether k-block kb of a dW / dH unit reads any kept box
+// of the panel (always true without filtering).  dH: rows [m0, m0 + 256) are
+// row halves m0 / 128 and the next; k-block kb is column box kb.  dW:
+// vocabulary ids [m0, m0 + 256) of the panel are boxes m0 / 64 .. + 3; k-block
+// kb covers rows [64 kb, 64 kb + 64) of row half kb / 2.
+template <int MODE>
+__device__ __forceinline__ bool kb_active(const GemmArgs& g, const Unit& un, int kb) {
+  if (MODE != kModeBwd || g.keep_wh == nullptr || un.cls == kClsGrad) return true;
+  if (un.cls == kClsDH) {
+    const uint8_t* k = g.keep_wh + static_cast<size_t>(un.m0 / BM) * g.keep_ld + kb;
+    return (k[0] | k[g.keep_ld]) != 0;
+  }
+  const uint8_t* k = g.keep_wh + static_cast<size_t>(kb >> 1) * g.keep_ld + (un.m0 >> 6);
+  return (k[0] | k[1] | k[2] | k[3]) != 0;
 }
 
 // TMA loads of k-block kb of unit `un` into this CTA's ring stage: its 128
@@ -342,6 +379,13 @@ struct FwdRowState {
   bool have_tgt;
 };
 
+// 2^x for element j of a chunk: with POLY every fourth on the FMA pipe.
+template <bool POLY>
+__device__ __forceinline__ float ex2_elem(float x, int j) {
+  return (POLY && (j & 3) == 3) ? ex2_poly(x) : ex2_approx(x);
+}
+
+template <bool POLY>
 __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb, int vglob0,
                                           int vlim, int yl, FwdRowState& st) {
   float x[32];
@@ -379,7 +423,7 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
     a0 += ex2_approx(fmaf(x[j], kLog2e, nb));
     a1 += ex2_approx(fmaf(x[j + 1], kLog2e, nb));
     a2 += ex2_approx(fmaf(x[j + 2], kLog2e, nb));
-    a3 += ex2_approx(fmaf(x[j + 3], kLog2e, nb));
+    a3 += ex2_elem<POLY>(fmaf(x[j + 3], kLog2e, nb), j + 3);
   }
   // first chunk: st.m = -inf, the old sum is scaled by exp(-inf) = 0
   st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + ((a0 + a1) + (a2 + a3));
@@ -393,13 +437,33 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
   }
 }
 
+// Column sums over a warp's 32 rows of a 32-column chunk: a butterfly that
+// halves the columns a lane holds at each step, so that lane j ends with
+// column j's sum.  The order of the additions is fixed.
+__device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = upper ? v[i] : v[i + s];
+      const float keep = upper ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
 // ---------------------------------------------------------------------------
 // Epilogue: gradient-panel values of one 32-column chunk, packed to 16 bits.
 // ---------------------------------------------------------------------------
+// krow is log2(sigma) - (log s) log2(e) - m log2(e) for the row, so that
+// sigma p = 2^(z log2(e) + krow) takes one FMA per entry.
+template <bool POLY>
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
-                                           int vglob0, int vlim, int yl, bool valid, float mrow,
-                                           float krow, float rrow, int row,
-                                           uint32_t (&packed)[16]) {
+                                           int vglob0, int vlim, int yl, bool valid,
+                                           float krow, float rrow, int row, int lane,
+                                           uint32_t (&packed)[16], bool& big) {
   float x[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(z[j]);
@@ -413,7 +477,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   float gv[32];
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
 #pragma unroll
-  for (int j = 0; j < 32; ++j) gv[j] = ex2_approx(fmaf(x[j] - mrow, kLog2e, krow));
+  for (int j = 0; j < 32; ++j) gv[j] = ex2_elem<POLY>(fmaf(x[j], kLog2e, krow), j);
   if (!valid) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) gv[j] = 0.f;
@@ -428,6 +492,11 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       if (j == jt) gv[j] -= g.sigma;
+  }
+  if (g.keep_g != nullptr) {
+    // gradient filtering: does this row hold an entry that is not negligible?
+#pragma unroll
+    for (int j = 0; j < 32; ++j) big |= fabsf(gv[j]) >= g.filter_eps_sigma;
   }
 #pragma unroll
   for (int j = 0; j < 32; ++j) gv[j] *= rrow;  // the row's scale relative to S
@@ -453,6 +522,15 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
     for (int j = 0; j < 16; ++j) {
       const __half2 h = __floats2half2_rn(gv[2 * j], gv[2 * j + 1]);
       packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  if (g.db_acc != nullptr) {
+    // bias gradient: this warp's 32 rows of the chunk, in fp32 (target
+    // entries included exactly), added as 2^-32 fixed-point integers
+    const float cs = warp_column_sums(gv, lane);
+    if (cb + lane < vlim) {
+      const long long q = __float2ll_rn(cs * g.db_fx_scale);
+      atomicAdd(g.db_acc + vglob0 + cb + lane, static_cast<unsigned long long>(q));
     }
   }
 }
@@ -484,7 +562,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_STAGE_BYTES;
   uint8_t* sStg = sB + STAGES * B_STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + ModeCfg<MODE>::STAGING);
+  float2* sMerge = reinterpret_cast<float2*>(sStg + ModeCfg<MODE>::STAGING);  // forward only
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + ModeCfg<MODE>::STAGING + ModeCfg<MODE>::MERGE);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -495,6 +574,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* decision = abort_flag + 1;  // [2]
   volatile int* s_unit = decision + 2;      // [UQ]
+  volatile int* s_keep = s_unit + UQ;       // [NUM_EPI_THREADS / 32]: filtering votes per warp
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -569,6 +649,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       if (lane == 0) {
         uint32_t n_issued = 0;
         bool ok = true;
+        // backward: whether this thread has waited for the previous launch
+        // (which may still run) and let the next one start
+        bool dep_done = MODE != kModeBwd;
         const uint32_t full_c0 = leader_addr(&full[0]);
         for (int it = 0; ok; ++it) {
           const int slot = it % UQ;
@@ -592,7 +675,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           }
           if (u < 0) break;
           const Unit un = decode_unit<MODE>(g, us, C, u);
+          if (MODE == kModeBwd && !dep_done && un.cls != kClsGrad) {
+            // dW / dH read the panel the previous launch wrote and add to the
+            // dH tiles it added to: wait for it to complete.  Only then may
+            // the next launch start (its gradient units overwrite the panel
+            // buffer that the launch before the previous one read).
+            griddep_wait();
+            griddep_launch_dependents();
+            dep_done = true;
+          }
           for (int kb = 0; kb < un.nk; ++kb) {
+            if (!kb_active<MODE>(g, un, kb)) continue;
             const uint32_t stage = n_issued % STAGES;
             const uint32_t phase = (n_issued / STAGES) & 1u;
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, g.err)) {
@@ -607,6 +700,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
                                     part);
             ++n_issued;
           }
+        }
+        if (!dep_done) {
+          griddep_wait();
+          griddep_launch_dependents();
         }
         // The even CTA lets every copy still in flight (its own and its peer's,
         // both producers') land before the pair can exit.
@@ -629,6 +726,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           mbar_arrive(&uq_empty[slot]);
           if (u < 0) break;
           const Unit un = decode_unit<MODE>(g, us, C, u);
+          // the filtering flags of the panel being read come from the previous launch
+          if (MODE == kModeBwd && g.keep_wh != nullptr && un.cls != kClsGrad) griddep_wait();
           if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, g.err)) break;
           tc_fence_after();
           const bool a_mn = unit_a_mn<MODE>(g, un);
@@ -640,7 +739,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           const uint32_t a_step = a_mn ? 16u * 128u : 32u;  // bytes per K=16 slice
           const uint32_t b_step = b_mn ? 16u * 128u : 32u;
           bool ok = true;
+          bool first = true;  // the first k-block issued overwrites the accumulator
           for (int kb = 0; kb < un.nk; ++kb) {
+            if (!kb_active<MODE>(g, un, kb)) continue;
             const uint32_t stage = n_used % STAGES;
             const uint32_t phase = (n_used / STAGES) & 1u;
             if (!mbar_wait(&full[stage], phase, abort_flag, g.err)) {
@@ -654,8 +755,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             for (int kk = 0; kk < BK / 16; ++kk) {
               const uint64_t ad = smem_desc_sw128(sa + kk * a_step, a_lbo, 1024u);
               const uint64_t bd = smem_desc_sw128(sb + kk * b_step, b_lbo, 1024u);
-              umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              umma_f16_pair(d_tmem, ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
             }
+            first = false;
             umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
             ++n_used;
           }
@@ -742,7 +844,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         if (MODE == kModeBwd && valid) {
           const int o = __ldg(g.idx + row);
           mrow = __ldg(g.m_saved + o);
-          krow = g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e;
+          krow = fmaf(-mrow, kLog2e, g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e);
           rrow = __ldg(g.row_scale + row);
         }
       } else if (MODE == kModePlain) {
@@ -763,19 +865,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 #pragma unroll 1
         for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
           tmem_ld32(t_acc + (c + 1) * 32, zb);
-          fwd_chunk(g, za, c * 32, vglob0, vlim, yl, st);
+          if (g.poly_exp)
+            fwd_chunk<true>(g, za, c * 32, vglob0, vlim, yl, st);
+          else
+            fwd_chunk<false>(g, za, c * 32, vglob0, vlim, yl, st);
           tmem_wait_ld(zb);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          fwd_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          if (g.poly_exp)
+            fwd_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          else
+            fwd_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_on_leader(&tempty[acc]);
-        if (valid) {
-          g.part[static_cast<size_t>(row) * g.part_ld + (un.n0 / BN) * NUM_EPI_WG + wg] =
-              make_float2(st.m, st.s);
-          if (st.have_tgt) g.tgt[row] = st.tgt;
+        if (valid && st.have_tgt) g.tgt[row] = st.tgt;
+        // the second warpgroup's half of the row joins the first's: one
+        // partial per row and tile, stored tile-major (coalesced per warp).
+        // The buffer is reused only after the next unit's decide_abort, which
+        // both warpgroups pass together.
+        if (wg == 1) sMerge[r] = make_float2(st.m, st.s);
+        named_bar_sync(4, NUM_EPI_THREADS);
+        if (wg == 0) {
+          const float2 o = sMerge[r];
+          const float mn = fmaxf(st.m, o.x);
+          if (mn != -INFINITY) {
+            st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + o.y * ex2_approx((o.x - mn) * kLog2e);
+            st.m = mn;
+          }
+          if (valid)
+            g.part[static_cast<size_t>(un.n0 / BN) * g.part_ld + row] = make_float2(st.m, st.s);
         }
       } else if (MODE == kModeBwd && un.cls == kClsGrad) {
         uint32_t za[32], zb[32];
@@ -788,16 +908,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           named_bar_sync(wg_bar, EPI_WG_THREADS);
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
-          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row, pk);
+          bool big = false;
+          if (g.poly_exp)
+            grad_chunk<true>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
+                             big);
+          else
+            grad_chunk<false>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
+                              big);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, mrow, krow, rrow, row,
-                     pk);
+          if (g.poly_exp)
+            grad_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row,
+                             lane, pk, big);
+          else
+            grad_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row,
+                              lane, pk, big);
           stage_row128(stg, r, 4, pk);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
           fence_proxy_async_smem();
+          if (g.keep_g != nullptr) {
+            const bool any = __any_sync(0xffffffffu, big);
+            if (lane == 0) s_keep[wg * 4 + q] = any ? 1 : 0;
+          }
           named_bar_sync(wg_bar, EPI_WG_THREADS);
+          if (g.keep_g != nullptr) {
+            // gradient filtering: the box (this warpgroup's 128 rows x 64
+            // columns) is kept when any of its entries is not negligible;
+            // a dropped box is stored as zeros, and the target entries it
+            // holds lose their fp32 residual as well
+            const int* sk = const_cast<const int*>(s_keep) + wg * 4;
+            const bool keep = (sk[0] | sk[1] | sk[2] | sk[3]) != 0;
+            if (!keep) {
+              const uint32_t zw[32] = {};
+              stage_row128(stg, r, 0, zw);
+              if (valid && static_cast<unsigned>(yl - c * 32) < 64u) g.tgt_resid[row] = 0.f;
+              fence_proxy_async_smem();
+              named_bar_sync(wg_bar, EPI_WG_THREADS);
+            }
+            if (wtid == 0)
+              g.keep_g[static_cast<size_t>(tm0 / BM) * g.keep_ld + (un.n0 + c * 32) / 64] =
+                  keep ? 1 : 0;
+          }
           if (wtid == 0) {
             // a box that starts past the panel's last column holds only padding
             if (un.n0 + c * 32 < g.w_g) tma_store_2d(&g.tmG, smem_addr(stg), un.n0 + c * 32, tm0);
@@ -813,9 +965,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         const CUtensorMap* map = is_dw ? &g.tmDW : &g.tmDH;
         const int y = is_dw ? g.vp_wh + tm0 : tm0;
         const bool reduce = !is_dw && g.dh_accumulate;
-        const bool zero = (un.nk == 0);
-        // a dW half that starts past the panel's last row has nothing to store
-        const bool issue = !is_dw || tm0 < g.w_wh;
+        bool zero = (un.nk == 0);
+        if (g.keep_wh != nullptr && !zero) {
+          // with filtering, no MMA ran when every k-block was skipped: the
+          // warp scans the unit's flags (from the previous launch)
+          griddep_wait();
+          bool any = false;
+          for (int kb = lane; kb < un.nk && !any; kb += 32) any = kb_active<MODE>(g, un, kb);
+          zero = !__any_sync(0xffffffffu, any);
+        }
+        // a dW half that starts past the panel's last row has nothing to store;
+        // adding a zero tile to dH changes nothing
+        const bool issue = (!is_dw || tm0 < g.w_wh) && !(zero && reduce);
         // this warpgroup's chunks [c0, ce) of the ones inside D
         const int ce = min(c0 + EPI_CHUNKS, cdiv_i(g.D - un.n0, 32));
         const int nch = ce;

@@ -83,6 +83,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a launch made with programmatic stream
+// serialisation may start while the previous kernel of the stream still
+// runs, once every CTA of that kernel has signalled (or exited).
+// ---------------------------------------------------------------------------
+// Waits until the previous kernel of the stream has completed and its memory
+// operations are visible (returns at once when there is no such dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Signals, for this CTA, that the next kernel of the stream may start.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters (CTA pairs)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -357,6 +370,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for epilogues whose exponentials outrun the special-
+// function unit.  x = n + f with n the nearest integer (adding 1.5 * 2^23
+// leaves n in the low bits of the sum) and f in [-1/2, 1/2]; 2^f from the
+// degree-5 polynomial of best relative approximation on [-1/2, 1/2] (Remez
+// exchange; exp2_poly_fit.py derives the coefficients: relative error
+// 1.55e-7 once rounded to float32); 2^n by adding n to the exponent field.
+// Arguments below -125 are clamped there (a result below 2^-125 instead of a
+// flush to zero); the callers' arguments never exceed 16.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23
+  const float n = t - 12582912.f;
+  const float f = x - n;
+  float p = fmaf(0x1.5c08e6p-10f, f, 0x1.3d0c52p-7f);
+  p = fmaf(p, f, 0x1.c6b6e4p-5f);
+  p = fmaf(p, f, 0x1.ebf918p-3f);
+  p = fmaf(p, f, 0x1.62e428p-1f);
+  p = fmaf(p, f, 0x1.000002p+0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 }  // namespace flce

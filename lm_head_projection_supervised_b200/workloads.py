@@ -48,6 +48,13 @@ class WorkloadSpec:
     big_row_frac: float = 0.0   # rows scaled by big_row_scale before rounding
     big_row_scale: float = 1.0
     lam: float = 1.0
+    # peaked logits (0 = off): each hidden row gets the direction of its label's
+    # weight row scaled so that the label's logit is about `peak_logit`, and of
+    # `n_comp` competitor ids (Zipf-distributed, frequent ids first) with logits
+    # drawn uniformly from `comp_logits`; h_scale then sets the noise level
+    peak_logit: float = 0.0
+    n_comp: int = 0
+    comp_logits: tuple = (0.0, 0.0)
 
 
 SPECS = {
@@ -66,6 +73,16 @@ SPECS = {
     "packed_d512": WorkloadSpec("packed_d512", 6, N=16384, D=512, V=248320, dtype="bf16",
                                 w_std=0.02 * 2 ** 0.5, label_dist="zipf", segments=8,
                                 prefix_frac=0.3),
+    "packed_d128": WorkloadSpec("packed_d128", 8, N=16384, D=128, V=248320, dtype="bf16",
+                                w_std=0.02 * 8 ** 0.5, label_dist="zipf", segments=8,
+                                prefix_frac=0.3),
+    "packed_d64": WorkloadSpec("packed_d64", 9, N=16384, D=64, V=248320, dtype="bf16",
+                               w_std=0.08, label_dist="zipf", segments=8, prefix_frac=0.3),
+    # the packed recipe with a few dominant logits per row (a trained model's
+    # shape of softmax), for the opt-in gradient filtering
+    "peaked": WorkloadSpec("peaked", 7, N=16384, D=1024, V=248320, dtype="bf16", w_std=0.02,
+                           h_scale=0.5, label_dist="zipf", segments=8, prefix_frac=0.3,
+                           peak_logit=16.0, n_comp=8, comp_logits=(6.0, 12.0)),
     "stress": WorkloadSpec("stress", 4, N=32768, D=4096, V=248320, dtype="bf16", w_std=0.02,
                            h_scale=4.0, big_row_frac=0.01, big_row_scale=50.0,
                            ignore_frac=0.5),
@@ -84,9 +101,14 @@ def round_half_up(x: float) -> int:
 # ---------------------------------------------------------------------------
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    u = u + 0x7FFF + ((u >> 16) & 1)
-    return (u >> 16).astype(np.uint16)
+    """Round to nearest even.  In 32-bit arithmetic: for finite inputs the
+    sum stays below 2^32 (the draws here are always finite)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -123,6 +145,7 @@ class Inputs:
     labels: np.ndarray            # int64 [N]
     mask: np.ndarray              # uint8 [N] (1 = supervised position)
     ignore_index: int = IGNORE_INDEX
+    big_rows: Optional[np.ndarray] = None  # rows scaled by big_row_scale (ascending), if any
 
     @property
     def N(self):
@@ -181,6 +204,30 @@ def _zipf_labels(rng: np.random.Generator, n: int, V: int, s: float) -> np.ndarr
     return np.minimum(np.searchsorted(cdf, u, side="right"), V - 1).astype(np.int64)
 
 
+def _peaked_hidden(rng: np.random.Generator, H_bits: np.ndarray, W_bits: np.ndarray,
+                   labels: np.ndarray, spec: "WorkloadSpec", chunk_rows: int = 2048):
+    """Adds to each (noise) hidden row a / |w|^2 times the weight row w of its
+    label (a = peak_logit) and of n_comp Zipf-drawn competitor ids (a drawn
+    from comp_logits), so that those logits sit near a; re-rounded to 16 bits."""
+    N, D = H_bits.shape
+    V = W_bits.shape[0]
+    comp = _zipf_labels(rng, N * spec.n_comp, V, spec.zipf_s).reshape(N, spec.n_comp)
+    lo, hi = spec.comp_logits
+    amp = rng.uniform(lo, hi, size=(N, spec.n_comp))
+    out = np.empty_like(H_bits)
+    for r0 in range(0, N, chunk_rows):
+        r1 = min(N, r0 + chunk_rows)
+        h = decode_f64(H_bits[r0:r1], spec.dtype).astype(np.float32)
+        ids = np.concatenate([labels[r0:r1, None], comp[r0:r1]], axis=1)
+        a = np.concatenate([np.full((r1 - r0, 1), spec.peak_logit), amp[r0:r1]], axis=1)
+        w = decode_f64(W_bits[ids.reshape(-1)], spec.dtype).astype(np.float32)
+        w = w.reshape(r1 - r0, ids.shape[1], D)
+        coef = (a / np.maximum((w.astype(np.float64) ** 2).sum(axis=2), 1e-30)).astype(np.float32)
+        h += np.einsum("rk,rkd->rd", coef, w)
+        out[r0:r1] = encode(h, spec.dtype)
+    return out
+
+
 def make_inputs(name_or_spec, seed: Optional[int] = None, **overrides) -> Inputs:
     """Build the seeded inputs of a named workload (or of a spec).
 
@@ -194,6 +241,7 @@ def make_inputs(name_or_spec, seed: Optional[int] = None, **overrides) -> Inputs
     N, D, V = spec.N, spec.D, spec.V
 
     row_scale = np.full(N, spec.h_scale, dtype=np.float64)
+    big = None
     if spec.big_row_frac > 0:
         nb = round_half_up(spec.big_row_frac * N)
         big = rng.permutation(N)[:nb]
@@ -208,6 +256,8 @@ def make_inputs(name_or_spec, seed: Optional[int] = None, **overrides) -> Inputs
         labels = _zipf_labels(rng, N, V, spec.zipf_s)
     else:
         labels = rng.integers(0, V, size=N, dtype=np.int64)
+    if spec.peak_logit > 0:
+        H = _peaked_hidden(rng, H, W, labels, spec)
 
     if spec.all_ignored:
         labels[:] = IGNORE_INDEX
@@ -225,7 +275,8 @@ def make_inputs(name_or_spec, seed: Optional[int] = None, **overrides) -> Inputs
         nm = round_half_up(spec.mask_false_frac * N)
         mask[rng.permutation(N)[:nm]] = 0
 
-    return Inputs(spec=spec, H=H, W=W, b=b, labels=labels, mask=mask)
+    return Inputs(spec=spec, H=H, W=W, b=b, labels=labels, mask=mask,
+                  big_rows=None if big is None else np.sort(big))
 
 
 def random_case(seed: int, N: int, D: int, V: int, dtype: str = "bf16", bias: bool = True,

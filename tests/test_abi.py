@@ -162,6 +162,7 @@ def bwd_ex(L, **kw):
     (dict(red=3), "FLCE_ERR_ARG"),
     (dict(red=-1), "FLCE_ERR_ARG"),
     (dict(fl=2), "FLCE_ERR_ARG"),                    # dH accumulation: backward-only bit
+    (dict(fl=4), "FLCE_ERR_ARG"),                    # reuse of a forward: backward-only bit
     (dict(red=2, rows=None), "FLCE_ERR_NULL"),       # 'none' needs the per-row output
     (dict(red=1, loss=None), "FLCE_ERR_NULL"),       # 'sum' needs the scalar
     (dict(red=0, w=FAKE + 2), "FLCE_ERR_ALIGN"),
@@ -248,7 +249,7 @@ def test_shard_combine_argument_errors(L, kw, want):
     (dict(b=FAKE, db=None), "FLCE_ERR_NULL"),
     (dict(v0=4, Vt=1004, wsb=4096), "FLCE_ERR_WORKSPACE"),
     (dict(v0=10, Vt=1004), "FLCE_ERR_SHAPE"),
-    (dict(fl=4), "FLCE_ERR_ARG"),
+    (dict(fl=8), "FLCE_ERR_ARG"),
 ])
 def test_shard_backward_argument_errors(L, kw, want):
     assert sbwd(L, **kw) == S[want]

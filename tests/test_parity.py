@@ -40,8 +40,9 @@ def full_check(inp, got):
     check_loss(got["loss"], ref["loss"])
     idx = ref["idx"]
     unsup = np.setdiff1d(np.arange(inp.N), idx)
-    check_stats(got["m"], ref["m"], idx)
-    check_stats(got["logs"], ref["logs"], idx, floor=logs_floor(ref["m"][idx], inp.D))
+    check_stats(got["m"], ref["m"], idx, quantity="m")
+    check_stats(got["logs"], ref["logs"], idx, floor=logs_floor(ref["m"][idx], inp.D),
+                quantity="logs")
     assert np.all(np.isneginf(got["m"][unsup])) and np.all(np.isneginf(got["logs"][unsup]))
     assert not got["dH"][unsup].any()
     check_grad("dH", got["dH"], ref["dH"])
@@ -97,6 +98,9 @@ CASES = [
     ("no_bias_wide_d", dict(seed=5, N=160, D=520, V=3000, bias=False)),
     ("single_class", dict(seed=6, N=5, D=8, V=1)),
     ("one_row", dict(seed=7, N=1, D=16, V=700, ignore_frac=0.0, mask_false_frac=0.0)),
+    # small hidden sizes: one exponential in four on the FMA pipe
+    ("small_d64", dict(seed=15, N=700, D=64, V=9000)),
+    ("small_d128_fp16", dict(seed=16, N=600, D=128, V=8300, dtype="fp16")),
 ]
 
 
@@ -158,6 +162,22 @@ def test_backward_is_deterministic():
     assert torch.equal(loss, l2)
 
 
+def test_backward_reuses_forward_compaction():
+    """FLCE_FLAG_REUSE_FORWARD: the backward on the forward's workspace skips
+    the compaction and gather and gives bit-identical gradients."""
+    inp = wl.random_case(seed=14, N=900, D=96, V=5000, dtype="fp16")
+    H, W, b, y, mk = to_device(inp)
+    ws = binding.Workspace(inp.N, inp.D, inp.V, H.dtype)
+    _, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
+    fresh = binding.backward(H, W, b, y, mk, -100, m, logs, lam=0.7, ws=ws)
+    _, m2, logs2 = binding.forward(H, W, b, y, mk, -100, ws=ws)
+    reused = binding.backward(H, W, b, y, mk, -100, m2, logs2, lam=0.7, ws=ws,
+                              reuse_forward=True)
+    assert binding.device_status(ws) == 0
+    for a, c in zip(fresh, reused):
+        assert torch.equal(a, c)
+
+
 def test_lambda_on_device_and_sign():
     inp = wl.random_case(seed=12, N=150, D=48, V=1200)
     H, W, b, y, mk = to_device(inp)
@@ -186,7 +206,8 @@ def test_autograd_wrapper_matches_abi():
 # --------------------------------------------------------------------------
 # full-size workloads, as the benchmark launches them
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("name", ["page2", "packed", "packed_d256", "packed_d512"])
+@pytest.mark.parametrize("name", ["page2", "packed", "packed_d64", "packed_d128", "packed_d256",
+                                  "packed_d512"])
 def test_full_size_sampled(name):
     inp = wl.make_inputs(name)
     got = run_gpu(inp)
@@ -194,11 +215,18 @@ def test_full_size_sampled(name):
     sampled_check(inp, got, full_stats=True)
 
 
-def test_stress_sampled():
+def test_stress_full():
+    """Stress (N=32768, D=4096, V=248320, 1 % of rows x50): the loss and m, log s
+    of every supervised row from the oracle's full forward, dW of the hottest,
+    tail and random ids, dH of sampled rows, and every x50 row on its own
+    (the large common shifts of the "分块交叉熵" page, §02 and §06)."""
     inp = wl.make_inputs("stress")
     got = run_gpu(inp)
     assert got["status"] == 0
-    sampled_check(inp, got, n_rows=48, full_stats=False)
+    idx, _ = orc.supervised_rows(inp.labels, inp.mask)
+    big = np.intersect1d(inp.big_rows, idx)
+    assert big.size > 100
+    sampled_check(inp, got, n_rows=48, full_stats=True, extra_rows=big)
 
 
 def test_stress_all_ignored():

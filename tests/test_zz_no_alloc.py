@@ -6,7 +6,7 @@ path where cudaMalloc's device-wide synchronisation is not acceptable.  Its
 scratch is a fixed buffer compiled into the library.  These tests call it
 through the C ABI and compare it with flce_forward() run on a caller-owned
 workspace, on two calls in a row (the second call finds the first call's
-leftovers in the shared buffer).  This file is collected last so that a run
+leftovers in the shared buffer), and both with the binary64 oracle.  This file is collected last so that a run
 stopping at the first failure has already run every other test.
 """
 import ctypes
@@ -44,6 +44,7 @@ def test_oversized_problem_is_rejected_before_any_gpu_work():
 def test_noalloc_forward_matches_workspace_forward(cuda_device, name):
     import torch
     from _gpu_helpers import check_loss, check_stats, logs_floor, to_device
+    from oracle import flce_oracle as orc
 
     f = _noalloc_fn()
     if name == "fp16_bias":
@@ -54,6 +55,7 @@ def test_noalloc_forward_matches_workspace_forward(cuda_device, name):
     ref_loss, ref_m, ref_logs = binding.forward(H, W, b, y, mk, -100)
     ref_m, ref_logs = ref_m.cpu().numpy(), ref_logs.cpu().numpy()
     sup = (inp.labels != -100) & (inp.mask != 0)
+    exact = orc.forward(inp.H64(), inp.W64(), inp.b64(), inp.labels, inp.mask)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for _ in range(2):
         loss = torch.full((), float("nan"), dtype=torch.float32, device=cuda_device)
@@ -67,8 +69,14 @@ def test_noalloc_forward_matches_workspace_forward(cuda_device, name):
                ctypes.c_void_p(logs.data_ptr()), stream)
         assert st == 0, binding.status_string(st)
         torch.cuda.synchronize()
-        check_loss(loss.item(), ref_loss.item())
+        check_loss(loss.item(), ref_loss.item(), quantity="loss vs flce_forward")
         gm, gl = m.cpu().numpy(), logs.cpu().numpy()
-        check_stats(gm[sup], ref_m[sup])
-        check_stats(gl[sup], ref_logs[sup], floor=logs_floor(ref_m[sup], inp.D))
+        check_stats(gm[sup], ref_m[sup], quantity="m vs flce_forward")
+        check_stats(gl[sup], ref_logs[sup], floor=logs_floor(ref_m[sup], inp.D),
+                    quantity="logs vs flce_forward")
         assert np.all(np.isneginf(gm[~sup])) and np.all(np.isneginf(gl[~sup]))
+        # and both against the oracle
+        check_loss(loss.item(), exact["loss"], quantity="loss vs oracle")
+        check_stats(gm[sup], exact["m"][sup], quantity="m vs oracle")
+        check_stats(gl[sup], exact["logs"][sup], floor=logs_floor(exact["m"][sup], inp.D),
+                    quantity="logs vs oracle")
