@@ -541,6 +541,36 @@ def main():
                        "the loss is read back every step, the gradients dH, dW (db) stay on "
                        "the device for an on-device optimizer step"}
 
+        # The same through the nn.Module a training loop calls
+        # (binding.LinearCrossEntropyLoss + loss.backward(): autograd, one
+        # workspace for both passes, gradients cast to the parameters' dtype).
+        crit = binding.LinearCrossEntropyLoss(ignore_index=-100)
+        barrier()
+        torch.cuda.synchronize(dev)
+        s0.record(stream)
+        copy_stream.wait_event(s0)
+        copy_in(0)
+        for k in range(args.steps):
+            if k + 1 < args.steps:
+                copy_in(k + 1)
+            stream.wait_event(copied[k % 2])
+            Hb, Wb, bb, yb, mb = bufs[k % 2]
+            Hp = Hb.detach().requires_grad_(True)
+            Wp = Wb.detach().requires_grad_(True)
+            bp = None if bb is None else bb.detach().requires_grad_(True)
+            loss = crit(Hp, yb, Wp, bias=bp, mask=mb)
+            (loss * inp.lam).backward()
+            freed[k % 2].record(stream)
+            loss_host.copy_(loss.detach(), non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        mod_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+        e2e["module"] = {"value": weak_scaling_tflops(flop_step, args.steps, mod_ms, world),
+                         "unit": UNIT, "loss": float(loss_host.item()),
+                         "note": "LinearCrossEntropyLoss forward + loss.backward(), the same "
+                                 "host-to-device copies; includes autograd and the casts of "
+                                 "dH, dW to the parameters' dtype (torch kernels)"}
+
     # roofline of the dominant kernel (largest share of device time)
     peaks, peak_src = load_peaks()
     flop_per_step = {"fwd_gemm": 2.0 * C * inp.D * inp.V,   # algorithmic FLOP per step

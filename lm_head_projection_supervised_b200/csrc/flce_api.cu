@@ -11,8 +11,10 @@
 //                         (+ the bias gradient's fixed-point column sums)
 //                       dW, dH units of panel L-1 (if L > 0) <- buffer (L-1) % 3
 //                     launches L >= 1 may start while launch L-1 runs
-//                     (programmatic dependent launch): their gradient units
-//                     overlap its tail, their dW / dH units wait for it
+//                     (programmatic dependent launch): their set-up overlaps
+//                     its tail, their dW / dH units wait for it; the third
+//                     panel buffer keeps a gradient unit from overwriting a
+//                     panel the previous launch may still read
 //   -> db from the column sums (bias only)
 //   -> rows grouped by label (stable radix sort, own kernels) -> dW target
 //      terms in fp32
@@ -44,8 +46,10 @@ constexpr float kFp16Log2Sigma = 15.f;  // fp16 panels hold (p - onehot) * 2^15
 #ifndef FLCE_POLY_EXP_MAX_D
 #define FLCE_POLY_EXP_MAX_D 256
 #endif
-// Up to this hidden size the epilogues' exponentials, not the tensor core,
-// bound the score tiles: one in four then goes to the FMA pipe (ex2_poly).
+// Up to this hidden size the forward epilogue, not the tensor core, bounds
+// the score tiles: one exponential in four then goes to the FMA pipe
+// (ex2_poly).  Measured: 6 % off the forward at D = 64 .. 256, nothing in the
+// gradient epilogue (which is not bound by the exponentials), a loss at 512.
 constexpr int64_t kPolyExpMaxD = FLCE_POLY_EXP_MAX_D;
 constexpr size_t kCounterOffset = 64;   // work counters follow the error word
 
@@ -624,7 +628,6 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.tgt_resid = p.resid;
     a.scal = p.scal;
     a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
-    a.poly_exp = D <= kPolyExpMaxD ? 1 : 0;
     a.inv_sigma = 1.f / sigma;
     a.db_acc = b != nullptr ? p.dbacc : nullptr;
     a.db_fx_scale = 0x1p32f / sigma;

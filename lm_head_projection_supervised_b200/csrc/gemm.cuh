@@ -24,10 +24,9 @@
 //              are merged in shared memory and one (m, s) partial per row and
 //              tile is stored, tile-major (a warp's 32 rows are contiguous).
 //   kModeBwd   three unit classes in one launch, with no dependency between
-//              them (the gradient units first: they need nothing from the
-//              previous launch, which may still be running -- programmatic
-//              dependent launch -- and the producers wait for it before
-//              their first dW / dH unit):
+//              them, longest first.  The launch may start while the previous
+//              one still runs (programmatic dependent launch): its producers
+//              wait for it before their first dW / dH unit.
 //              class 2 (grad): the tile of vocabulary panel p recomputed; the
 //                 epilogue rebuilds p = exp((Z - m) - log s) from the saved
 //                 statistics, subtracts the one-hot target (§04), rounds to
@@ -131,8 +130,8 @@ struct GemmArgs {
   const int* idx;          // compact row -> original row
   const uint16_t* bias;    // 16-bit bias [V] or null
   int round_logits;        // round each logit to the 16-bit input type first
-  int poly_exp;            // one exponential in four on the FMA pipe (ex2_poly): for small
-                           // D, where the epilogue's exponentials outrun the tensor core
+  int poly_exp;            // fwd: one exponential in four on the FMA pipe (ex2_poly), for
+                           // small D
   float2* part;            // fwd: (m, s) partials [tiles][part_ld], part_ld >= rows
   int part_ld;
   float* tgt;              // fwd: target logits [rows]
@@ -194,12 +193,22 @@ __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
     s.k0 = cdiv_i(C, BK);
     s.k1 = cdiv_i(g.w_wh, BK);
     s.k2 = cdiv_i(g.D, BK);
-    // The gradient units first: they depend on nothing the previous launch
-    // produces, so they fill the SMs while its last units finish.  Then dW
-    // and dH, longer units first.
-    s.o0 = kClsGrad;
-    s.o1 = (s.k0 >= s.k1) ? kClsDW : kClsDH;
-    s.o2 = (s.k0 >= s.k1) ? kClsDH : kClsDW;
+    // Longest units first (dW, dH, then the short gradient units), so that a
+    // launch ends on short units (a short tail), and the panel the gradient
+    // units write at the end of a launch is still in L2 when the next
+    // launch's dW / dH units read it at its start.  Measured against
+    // gradient-units-first (which lets them overlap the previous launch's
+    // tail): about 1 % faster.
+    {
+      int a = 0, b = 1, c = 2;
+      int ka = s.k0, kb = s.k1, kc = s.k2;
+      if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
+      if (kb < kc) { int t = b; b = c; c = t; t = kb; kb = kc; kc = t; }
+      if (ka < kb) { int t = a; a = b; b = t; t = ka; ka = kb; kb = t; }
+      s.o0 = a;
+      s.o1 = b;
+      s.o2 = c;
+    }
     s.total = s.n0 + s.n1 + s.n2;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
@@ -263,20 +272,46 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
   return false;
 }
 
-// Gradient filtering: whether k-block kb of a dW / dH unit reads any kept box
-// of the panel (always true without filtering).  dH: rows [m0, m0 + 256) are
-// row halves m0 / 128 and the next; k-block kb is column box kb.  dW:
-// vocabulary ids [m0, m0 + 256) of the panel are boxes m0 / 64 .. + 3; k-block
-// kb covers rows [64 kb, 64 kb + 64) of row half kb / 2.
+// Gradient filtering: which k-blocks of a dW / dH unit read any kept box of
+// the panel (all of them without filtering).  dH: rows [m0, m0 + 256) are row
+// halves m0 / 128 and the next; k-block kb is column box kb.  dW: vocabulary
+// ids [m0, m0 + 256) of the panel are boxes m0 / 64 .. + 3; k-block kb covers
+// rows [64 kb, 64 kb + 64) of row half kb / 2.  Computed for k-blocks
+// kb0 .. kb0 + 31 at once, as a bit mask (bit j: k-block kb0 + j; bits past nk
+// are 0): the flags are read with independent loads issued back to back.
 template <int MODE>
-__device__ __forceinline__ bool kb_active(const GemmArgs& g, const Unit& un, int kb) {
-  if (MODE != kModeBwd || g.keep_wh == nullptr || un.cls == kClsGrad) return true;
+__device__ __forceinline__ uint32_t active_mask32(const GemmArgs& g, const Unit& un, int kb0) {
+  if (MODE != kModeBwd || g.keep_wh == nullptr || un.cls == kClsGrad) return 0xffffffffu;
+  uint32_t m = 0;
   if (un.cls == kClsDH) {
-    const uint8_t* k = g.keep_wh + static_cast<size_t>(un.m0 / BM) * g.keep_ld + kb;
-    return (k[0] | k[g.keep_ld]) != 0;
+    // 32 flag bytes of each of the two row halves, read as 32-bit words (a row
+    // holds a multiple of 4 flags, and a word that starts before nk ends
+    // inside the row); flag byte k of a word becomes bit k
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(
+        g.keep_wh + static_cast<size_t>(un.m0 / BM) * g.keep_ld + kb0);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(
+        reinterpret_cast<const uint8_t*>(r0) + g.keep_ld);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t w = (kb0 + 4 * i < un.nk) ? (r0[i] | r1[i]) : 0u;
+      const uint32_t b4 = (w & 1u) | ((w >> 7) & 2u) | ((w >> 14) & 4u) | ((w >> 21) & 8u);
+      m |= b4 << (4 * i);
+    }
+    if (un.nk - kb0 < 32) m &= (1u << (un.nk - kb0)) - 1u;
+  } else {
+    // two k-blocks per row half; four flag bytes (one 32-bit word) per row half
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      w[i] = (kb0 + 2 * i < un.nk)
+                 ? *reinterpret_cast<const uint32_t*>(
+                       g.keep_wh + static_cast<size_t>((kb0 >> 1) + i) * g.keep_ld + (un.m0 >> 6))
+                 : 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m |= (w[i] != 0 ? 3u : 0u) << (2 * i);
+    if (un.nk - kb0 < 32) m &= (1u << (un.nk - kb0)) - 1u;
   }
-  const uint8_t* k = g.keep_wh + static_cast<size_t>(kb >> 1) * g.keep_ld + (un.m0 >> 6);
-  return (k[0] | k[1] | k[2] | k[3]) != 0;
+  return m;
 }
 
 // TMA loads of k-block kb of unit `un` into this CTA's ring stage: its 128
@@ -459,7 +494,6 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
 // ---------------------------------------------------------------------------
 // krow is log2(sigma) - (log s) log2(e) - m log2(e) for the row, so that
 // sigma p = 2^(z log2(e) + krow) takes one FMA per entry.
-template <bool POLY>
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
                                            int vglob0, int vlim, int yl, bool valid,
                                            float krow, float rrow, int row, int lane,
@@ -477,7 +511,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   float gv[32];
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
 #pragma unroll
-  for (int j = 0; j < 32; ++j) gv[j] = ex2_elem<POLY>(fmaf(x[j], kLog2e, krow), j);
+  for (int j = 0; j < 32; ++j) gv[j] = ex2_approx(fmaf(x[j], kLog2e, krow));
   if (!valid) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) gv[j] = 0.f;
@@ -684,8 +718,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             griddep_launch_dependents();
             dep_done = true;
           }
+          uint32_t act = 0;
           for (int kb = 0; kb < un.nk; ++kb) {
-            if (!kb_active<MODE>(g, un, kb)) continue;
+            if ((kb & 31) == 0) act = active_mask32<MODE>(g, un, kb);
+            if (!((act >> (kb & 31)) & 1u)) continue;
             const uint32_t stage = n_issued % STAGES;
             const uint32_t phase = (n_issued / STAGES) & 1u;
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, g.err)) {
@@ -740,8 +776,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           const uint32_t b_step = b_mn ? 16u * 128u : 32u;
           bool ok = true;
           bool first = true;  // the first k-block issued overwrites the accumulator
+          uint32_t act = 0;
           for (int kb = 0; kb < un.nk; ++kb) {
-            if (!kb_active<MODE>(g, un, kb)) continue;
+            if ((kb & 31) == 0) act = active_mask32<MODE>(g, un, kb);
+            if (!((act >> (kb & 31)) & 1u)) continue;
             const uint32_t stage = n_used % STAGES;
             const uint32_t phase = (n_used / STAGES) & 1u;
             if (!mbar_wait(&full[stage], phase, abort_flag, g.err)) {
@@ -857,29 +895,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       const uint32_t t_acc = lane_base + static_cast<uint32_t>(acc * BN);
 
       if (MODE == kModeFwd) {
-        // (m, s) of this warpgroup's 128 columns: one partial per half tile
+        // (m, s) of this warpgroup's 128 columns.  All four 32-column chunks
+        // are read from TMEM first and the accumulator is handed back to the
+        // MMA issuer before the arithmetic, so the next unit's MMAs into it
+        // overlap this epilogue.
         FwdRowState st{-INFINITY, 0.f, 0.f, false};
-        uint32_t za[32], zb[32];
-        tmem_ld32(t_acc + c0 * 32, za);
-        tmem_wait_ld(za);
-#pragma unroll 1
-        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
-          tmem_ld32(t_acc + (c + 1) * 32, zb);
-          if (g.poly_exp)
-            fwd_chunk<true>(g, za, c * 32, vglob0, vlim, yl, st);
-          else
-            fwd_chunk<false>(g, za, c * 32, vglob0, vlim, yl, st);
-          tmem_wait_ld(zb);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          if (g.poly_exp)
-            fwd_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          else
-            fwd_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
-        }
+        uint32_t zz[EPI_CHUNKS][32];
+#pragma unroll
+        for (int k = 0; k < EPI_CHUNKS; ++k) tmem_ld32(t_acc + (c0 + k) * 32, zz[k]);
+#pragma unroll
+        for (int k = 0; k < EPI_CHUNKS; ++k) tmem_wait_ld(zz[k]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_on_leader(&tempty[acc]);
+        if (g.poly_exp) {
+#pragma unroll
+          for (int k = 0; k < EPI_CHUNKS; ++k)
+            fwd_chunk<true>(g, zz[k], (c0 + k) * 32, vglob0, vlim, yl, st);
+        } else {
+#pragma unroll
+          for (int k = 0; k < EPI_CHUNKS; ++k)
+            fwd_chunk<false>(g, zz[k], (c0 + k) * 32, vglob0, vlim, yl, st);
+        }
         if (valid && st.have_tgt) g.tgt[row] = st.tgt;
         // the second warpgroup's half of the row joins the first's: one
         // partial per row and tile, stored tile-major (coalesced per warp).
@@ -898,6 +935,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             g.part[static_cast<size_t>(un.n0 / BN) * g.part_ld + row] = make_float2(st.m, st.s);
         }
       } else if (MODE == kModeBwd && un.cls == kClsGrad) {
+        // Chunks stream out of TMEM two at a time (registers allow no more);
+        // the accumulator is handed back to the MMA issuer as soon as the last
+        // chunk has been read, before its arithmetic.
         uint32_t za[32], zb[32];
         tmem_ld32(t_acc + c0 * 32, za);
         tmem_wait_ld(za);
@@ -909,21 +949,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
           bool big = false;
-          if (g.poly_exp)
-            grad_chunk<true>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
-                             big);
-          else
-            grad_chunk<false>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
-                              big);
+          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk, big);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          if (g.poly_exp)
-            grad_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row,
-                             lane, pk, big);
-          else
-            grad_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row,
-                              lane, pk, big);
+          if (c + 2 < c0 + EPI_CHUNKS) {
+            tmem_ld32(t_acc + (c + 2) * 32, za);
+          } else {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_on_leader(&tempty[acc]);
+          }
+          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
+                     big);
           stage_row128(stg, r, 4, pk);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
           fence_proxy_async_smem();
@@ -956,9 +993,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             bulk_commit_group();
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else if (MODE == kModeBwd) {
         // dW (class 0) or dH (class 1): fp32, scaled by lambda / (C sigma)
         const bool is_dw = un.cls == kClsDW;
@@ -971,7 +1005,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           // warp scans the unit's flags (from the previous launch)
           griddep_wait();
           bool any = false;
-          for (int kb = lane; kb < un.nk && !any; kb += 32) any = kb_active<MODE>(g, un, kb);
+          for (int kb0 = 32 * lane; kb0 < un.nk && !any; kb0 += 32 * 32)
+            any = active_mask32<MODE>(g, un, kb0) != 0;
           zero = !__any_sync(0xffffffffu, any);
         }
         // a dW half that starts past the panel's last row has nothing to store;

@@ -91,3 +91,17 @@ def test_filter_eps_rejected_when_negative():
     _, m, logs = binding.forward(H, W, b, y, mk)
     with pytest.raises(binding.FlceError):
         binding.backward(H, W, b, y, mk, -100, m, logs, filter_eps=-1e-3)
+
+
+def test_exact_backward_on_peaked_logits():
+    """The exact path on the same peaked inputs: its dH error against the exact
+    oracle shows what the 16-bit staging of large non-target probabilities
+    costs without any filtering."""
+    inp = _peaked(**CASES[0][1])
+    H, W, b, y, mk = to_device(inp)
+    ws = binding.Workspace(inp.N, inp.D, inp.V, H.dtype)
+    _, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws)
+    dH, dW, _ = binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws)
+    ex = orc.forward_backward(inp.H64(), inp.W64(), inp.b64(), inp.labels, inp.mask, lam=inp.lam)
+    check_grad("dH exact, peaked", dH.cpu().numpy(), ex["dH"])
+    check_grad("dW exact, peaked", dW.cpu().numpy(), ex["dW"])
