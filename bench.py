@@ -545,6 +545,18 @@ def main():
         # (binding.LinearCrossEntropyLoss + loss.backward(): autograd, one
         # workspace for both passes, gradients cast to the parameters' dtype).
         crit = binding.LinearCrossEntropyLoss(ignore_index=-100)
+
+        def module_step(x):
+            Hb, Wb, bb, yb, mb = x
+            Hp = Hb.detach().requires_grad_(True)
+            Wp = Wb.detach().requires_grad_(True)
+            bp = None if bb is None else bb.detach().requires_grad_(True)
+            loss = crit(Hp, yb, Wp, bias=bp, mask=mb)
+            (loss * inp.lam).backward()
+            return loss.detach()
+
+        for _ in range(2):  # untimed: the allocator's first blocks for this path
+            module_step(inputs)
         barrier()
         torch.cuda.synchronize(dev)
         s0.record(stream)
@@ -554,14 +566,9 @@ def main():
             if k + 1 < args.steps:
                 copy_in(k + 1)
             stream.wait_event(copied[k % 2])
-            Hb, Wb, bb, yb, mb = bufs[k % 2]
-            Hp = Hb.detach().requires_grad_(True)
-            Wp = Wb.detach().requires_grad_(True)
-            bp = None if bb is None else bb.detach().requires_grad_(True)
-            loss = crit(Hp, yb, Wp, bias=bp, mask=mb)
-            (loss * inp.lam).backward()
+            loss = module_step(bufs[k % 2])
             freed[k % 2].record(stream)
-            loss_host.copy_(loss.detach(), non_blocking=True)
+            loss_host.copy_(loss, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize(dev)
         mod_ms = max_over_ranks(s0.elapsed_time(s1), dev)

@@ -573,7 +573,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     return FLCE_ERR_CUDA;
 
   const int64_t nT_max = cdiv64(N, PAIR_M);
-  const int64_t nD = cdiv64(D, BN);
+  const int bn_wh = D <= 128 ? 128 : BN;  // dW / dH tile width along D
+  const int64_t nD = cdiv64(D, bn_wh);
   if (b != nullptr) FLCE_CK(cudaMemsetAsync(p.dbacc, 0, static_cast<size_t>(V) * 8, s));
   // The GEMM launches form one timed span: with programmatic dependent launch
   // they overlap, so events between them would measure nothing useful (and
@@ -614,6 +615,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.vp_wh = static_cast<int>(vp_wh);
     a.w_wh = static_cast<int>(w_wh);
     a.dh_accumulate = Lp > 1;
+    a.bn_wh = bn_wh;
     a.has_g = has_g;
     a.vp_g = static_cast<int>(vp_g);
     a.w_g = static_cast<int>(w_g);

@@ -63,7 +63,10 @@ constexpr int BK = 64;
 constexpr int UQ = 4;                            // depth of the unit-id ring
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;       // 16 KiB
 constexpr uint32_t B_STAGE_BYTES = BN_HALF * BK * 2;  // 16 KiB
-constexpr uint32_t PAIR_TX_BYTES = 2 * (A_STAGE_BYTES + B_STAGE_BYTES);  // both CTAs' loads
+// bytes both CTAs' loads bring per k-block for a tile of bn columns
+__host__ __device__ constexpr uint32_t pair_tx_bytes(int bn) {
+  return 2 * (A_STAGE_BYTES + static_cast<uint32_t>(bn / 2) * BK * 2);
+}
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;   // 8 KiB: 64 MN-elements x 64 K rows
 constexpr uint32_t STG_BYTES = BM * 128;         // 16 KiB: 128 rows x 128 bytes
 // Warps 0-3 form the first warpgroup: scheduler + producer (warp 0), MMA
@@ -79,7 +82,7 @@ constexpr int EPI_CHUNKS = BN / 32 / NUM_EPI_WG;  // 32-column chunks per epilog
 // Registers per thread after the split: the first warpgroup gives up what the
 // epilogue takes.  The block is launched with at least kRegsAtLaunch per
 // thread (checked on the host before any launch), which covers the split.
-constexpr uint32_t kRegsLow = 72;
+constexpr uint32_t kRegsLow = 72;  // 56 spilled in the producers (backward 4 % slower)
 constexpr uint32_t kRegsHigh = 216;
 constexpr uint32_t kRegsAtLaunch =
     (128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh + NUM_THREADS - 1) / NUM_THREADS;
@@ -124,6 +127,8 @@ struct GemmArgs {
   // bwd: the dW/dH part works on panel [vp_wh, vp_wh + w_wh), the gradient
   // part produces panel [vp_g, vp_g + w_g)
   int has_wh, vp_wh, w_wh, dh_accumulate;
+  int bn_wh;               // bwd: columns (hidden dimension) of a dW / dH tile: BN, or 128
+                           //      when D <= 128, so that small D does not pay for padding
   int has_g, vp_g, w_g;
   // epilogue data
   const int* y_c;          // compact labels
@@ -165,6 +170,7 @@ struct Unit {
   int m0;
   int n0;
   int nk;
+  int bn;  // columns of the unit's tile: BN, or GemmArgs::bn_wh for dW / dH units
 };
 
 __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
@@ -186,7 +192,7 @@ template <int MODE>
 __device__ __forceinline__ UnitSpace make_unit_space(const GemmArgs& g, int C) {
   UnitSpace s;
   if (MODE == kModeBwd) {
-    const int nT = cdiv_i(C, PAIR_M), nD = cdiv_i(g.D, BN);
+    const int nT = cdiv_i(C, PAIR_M), nD = cdiv_i(g.D, g.bn_wh);
     s.n0 = g.has_wh ? cdiv_i(g.w_wh, PAIR_M) * nD : 0;   // dW
     s.n1 = g.has_wh ? nT * nD : 0;                       // dH
     s.n2 = g.has_g ? nT * cdiv_i(g.w_g, BN) : 0;         // grad
@@ -247,14 +253,16 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& g, const UnitSpace& 
     // dW / dH: the hidden-dimension block varies fastest, so the units that
     // read the same block of the gradient panel (a column strip for dW, a
     // row block for dH) run side by side and share it through L2
-    const int nD = cdiv_i(g.D, BN);
+    const int nD = cdiv_i(g.D, g.bn_wh);
     un.m0 = (u / nD) * PAIR_M;
-    un.n0 = (u % nD) * BN;
+    un.n0 = (u % nD) * g.bn_wh;
+    un.bn = g.bn_wh;
   } else {
     const int rows = (MODE == kModePlain) ? g.M : C;
     const int nT = cdiv_i(rows, PAIR_M);
     un.m0 = (u % nT) * PAIR_M;
     un.n0 = (u / nT) * BN;
+    un.bn = BN;
   }
   return un;
 }
@@ -335,7 +343,7 @@ __device__ __forceinline__ void issue_stage_loads(const GemmArgs& g, const Unit&
   const CUtensorMap* tB = &g.tmB[mapi];
   const int k0 = kb * BK;
   const int am0 = un.m0 + static_cast<int>(rank) * BM;       // this CTA's A rows
-  const int bn0 = un.n0 + static_cast<int>(rank) * BN_HALF;  // this CTA's B rows
+  const int bn0 = un.n0 + static_cast<int>(rank) * (un.bn / 2);  // this CTA's B rows
   if (part != kLoadB) {
     if (unit_a_mn<MODE>(g, un)) {
       tma_load_2d_pair(sa, tA, bar_cluster, am0, k0);
@@ -349,7 +357,7 @@ __device__ __forceinline__ void issue_stage_loads(const GemmArgs& g, const Unit&
     // dH: the k index is a vocabulary id of the panel
     const int kB = (MODE == kModeBwd && un.cls == kClsDH) ? g.vp_wh + k0 : k0;
     tma_load_2d_pair(sb, tB, bar_cluster, bn0, kB);
-    tma_load_2d_pair(sb + MN_BOX_BYTES, tB, bar_cluster, bn0 + 64, kB);
+    if (un.bn / 2 > 64) tma_load_2d_pair(sb + MN_BOX_BYTES, tB, bar_cluster, bn0 + 64, kB);
   } else {
     // fwd / grad: the row index is a vocabulary id
     const int nrow = (MODE == kModeBwd) ? g.vp_g + bn0 : bn0;
@@ -729,7 +737,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
               break;
             }
             // one arrival (with both CTAs' bytes) per stage, from the scheduler
-            if (scheduler) mbar_arrive_expect_tx(&full[stage], PAIR_TX_BYTES);
+            if (scheduler) mbar_arrive_expect_tx(&full[stage], pair_tx_bytes(un.bn));
             issue_stage_loads<MODE>(g, un, kb, rank, smem_addr(sA + stage * A_STAGE_BYTES),
                                     smem_addr(sB + stage * B_STAGE_BYTES),
                                     full_c0 + stage * static_cast<uint32_t>(sizeof(uint64_t)),
@@ -768,7 +776,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           tc_fence_after();
           const bool a_mn = unit_a_mn<MODE>(g, un);
           const bool b_mn = unit_b_mn<MODE>(g, un);
-          const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, PAIR_M, BN);
+          const uint32_t idesc = make_idesc_f16(g.is_bf16 != 0, a_mn, b_mn, PAIR_M, un.bn);
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
           const uint32_t a_lbo = a_mn ? MN_BOX_BYTES : 16u;
           const uint32_t b_lbo = b_mn ? MN_BOX_BYTES : 16u;
@@ -895,27 +903,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       const uint32_t t_acc = lane_base + static_cast<uint32_t>(acc * BN);
 
       if (MODE == kModeFwd) {
-        // (m, s) of this warpgroup's 128 columns.  All four 32-column chunks
-        // are read from TMEM first and the accumulator is handed back to the
-        // MMA issuer before the arithmetic, so the next unit's MMAs into it
-        // overlap this epilogue.
+        // (m, s) of this warpgroup's 128 columns.  Chunks stream out of TMEM
+        // two at a time (one loading while the other is reduced), and the
+        // accumulator goes back to the MMA issuer as soon as the last chunk
+        // has been read.  (Reading all four first and releasing before any
+        // arithmetic measured slower: 8 % on the forward at D = 64 and 128.)
         FwdRowState st{-INFINITY, 0.f, 0.f, false};
-        uint32_t zz[EPI_CHUNKS][32];
-#pragma unroll
-        for (int k = 0; k < EPI_CHUNKS; ++k) tmem_ld32(t_acc + (c0 + k) * 32, zz[k]);
-#pragma unroll
-        for (int k = 0; k < EPI_CHUNKS; ++k) tmem_wait_ld(zz[k]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_on_leader(&tempty[acc]);
-        if (g.poly_exp) {
-#pragma unroll
-          for (int k = 0; k < EPI_CHUNKS; ++k)
-            fwd_chunk<true>(g, zz[k], (c0 + k) * 32, vglob0, vlim, yl, st);
-        } else {
-#pragma unroll
-          for (int k = 0; k < EPI_CHUNKS; ++k)
-            fwd_chunk<false>(g, zz[k], (c0 + k) * 32, vglob0, vlim, yl, st);
+        uint32_t za[32], zb[32];
+        tmem_ld32(t_acc + c0 * 32, za);
+        tmem_wait_ld(za);
+#pragma unroll 1
+        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
+          tmem_ld32(t_acc + (c + 1) * 32, zb);
+          if (g.poly_exp)
+            fwd_chunk<true>(g, za, c * 32, vglob0, vlim, yl, st);
+          else
+            fwd_chunk<false>(g, za, c * 32, vglob0, vlim, yl, st);
+          tmem_wait_ld(zb);
+          const bool last = c + 2 >= c0 + EPI_CHUNKS;
+          if (!last) {
+            tmem_ld32(t_acc + (c + 2) * 32, za);
+          } else {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_on_leader(&tempty[acc]);
+          }
+          if (g.poly_exp)
+            fwd_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          else
+            fwd_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          if (!last) tmem_wait_ld(za);
         }
         if (valid && st.have_tgt) g.tgt[row] = st.tgt;
         // the second warpgroup's half of the row joins the first's: one
