@@ -193,23 +193,29 @@ flce_status device_setup(DevInfo* out) {
       return FLCE_ERR_CUDA;
     d.ok = (major == 10 && minor == 0) && encode_fn() != nullptr;
     if (d.ok) {
-      if (cudaFuncSetAttribute(flce_gemm_kernel<kModeFwd>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(ModeCfg<kModeFwd>::SMEM_BYTES)) != cudaSuccess ||
-          cudaFuncSetAttribute(flce_gemm_kernel<kModeBwd>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(ModeCfg<kModeBwd>::SMEM_BYTES)) != cudaSuccess ||
-          cudaFuncSetAttribute(flce_gemm_kernel<kModePlain>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(ModeCfg<kModePlain>::SMEM_BYTES)) != cudaSuccess)
-        return FLCE_ERR_CUDA;
-      // The GEMM kernels split registers between warpgroups with setmaxnreg;
-      // the split only fits if the block was launched with enough of them.
-      for (const void* fn : {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd>),
-                             reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd>),
-                             reinterpret_cast<const void*>(flce_gemm_kernel<kModePlain>)}) {
+      const struct {
+        const void* fn;
+        size_t smem;
+      } kernels[] = {
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd>), ModeCfg<kModeFwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, 0>),
+           ModeCfg<kModeBwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatBias>),
+           ModeCfg<kModeBwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatFilter>),
+           ModeCfg<kModeBwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatBias | kFeatFilter>),
+           ModeCfg<kModeBwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModePlain>),
+           ModeCfg<kModePlain>::SMEM_BYTES}};
+      for (const auto& k : kernels) {
+        if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(k.smem)) != cudaSuccess)
+          return FLCE_ERR_CUDA;
+        // The GEMM kernels split registers between warpgroups with setmaxnreg;
+        // the split only fits if the block was launched with enough of them.
         cudaFuncAttributes fa{};
-        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return FLCE_ERR_CUDA;
+        if (cudaFuncGetAttributes(&fa, k.fn) != cudaSuccess) return FLCE_ERR_CUDA;
         if (fa.numRegs < static_cast<int>(kRegsAtLaunch)) d.ok = false;
       }
     }
@@ -307,7 +313,7 @@ void prof_span_end(ProfRec* r, int launches, cudaStream_t s) {
 // pdl: the launch may start before the previous kernel of the stream ends
 // (programmatic stream serialisation; the kernel waits where it must).
 // timed: wrap the launch in profiling events (off inside a timed span).
-template <int MODE>
+template <int MODE, int FEAT = 0>
 cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaStream_t s,
                         bool pdl = false, bool timed = true) {
   if (units_upper <= 0) return cudaSuccess;
@@ -328,7 +334,7 @@ cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaS
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    cudaLaunchKernelEx(&cfg, flce_gemm_kernel<MODE>, a);
+    cudaLaunchKernelEx(&cfg, flce_gemm_kernel<MODE, FEAT>, a);
   };
   if (!timed) {
     launch();
@@ -645,8 +651,22 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +
                           (has_g ? nT_max * cdiv64(w_g, BN) : 0);
     // every launch after the first may overlap its predecessor
-    FLCE_CK(launch_gemm<kModeBwd>(a, units, di.pairs, s, /*pdl=*/launched > 0,
-                                  /*timed=*/false));
+    const bool pdl = launched > 0;
+    cudaError_t e;
+    switch ((b != nullptr ? kFeatBias : 0) | (filter_eps > 0.f ? kFeatFilter : 0)) {
+      case kFeatBias:
+        e = launch_gemm<kModeBwd, kFeatBias>(a, units, di.pairs, s, pdl, false);
+        break;
+      case kFeatFilter:
+        e = launch_gemm<kModeBwd, kFeatFilter>(a, units, di.pairs, s, pdl, false);
+        break;
+      case kFeatBias | kFeatFilter:
+        e = launch_gemm<kModeBwd, kFeatBias | kFeatFilter>(a, units, di.pairs, s, pdl, false);
+        break;
+      default:
+        e = launch_gemm<kModeBwd, 0>(a, units, di.pairs, s, pdl, false);
+    }
+    FLCE_CK(e);
     launched += units > 0 ? 1 : 0;
   }
   if (timed) prof_span_end(&span, launched, s);

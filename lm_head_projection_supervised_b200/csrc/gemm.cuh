@@ -16,7 +16,8 @@
 // lane = tile row) and run the epilogue while the next unit accumulates in
 // the other.
 //
-// Modes (one launch = one mode):
+// Modes (one launch = one mode; the backward is instantiated once per
+// combination of its optional features, FEAT = kFeatBias | kFeatFilter):
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
 //              running max / rescaled exp-sum over the tile's columns and
 //              captures the target logit from the tile that holds it
@@ -107,6 +108,10 @@ struct ModeCfg {
 };
 constexpr size_t GEMM_SMEM_BYTES = ModeCfg<kModeBwd>::SMEM_BYTES;  // the largest
 enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
+// Optional work of the backward, chosen when the kernel is compiled (one
+// instantiation per combination), so that the common path carries none of
+// its code: measured, the runtime-switched form cost the backward 3-4 %.
+enum BwdFeature : int { kFeatBias = 1, kFeatFilter = 2 };
 
 struct GemmArgs {
   CUtensorMap tmA[3];  // A operand map per unit class (fwd / plain use [0])
@@ -287,9 +292,9 @@ __device__ __forceinline__ bool unit_b_mn(const GemmArgs& g, const Unit& un) {
 // rows [64 kb, 64 kb + 64) of row half kb / 2.  Computed for k-blocks
 // kb0 .. kb0 + 31 at once, as a bit mask (bit j: k-block kb0 + j; bits past nk
 // are 0): the flags are read with independent loads issued back to back.
-template <int MODE>
+template <int MODE, int FEAT>
 __device__ __forceinline__ uint32_t active_mask32(const GemmArgs& g, const Unit& un, int kb0) {
-  if (MODE != kModeBwd || g.keep_wh == nullptr || un.cls == kClsGrad) return 0xffffffffu;
+  if (MODE != kModeBwd || !(FEAT & kFeatFilter) || un.cls == kClsGrad) return 0xffffffffu;
   uint32_t m = 0;
   if (un.cls == kClsDH) {
     // 32 flag bytes of each of the two row halves, read as 32-bit words (a row
@@ -502,6 +507,7 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
 // ---------------------------------------------------------------------------
 // krow is log2(sigma) - (log s) log2(e) - m log2(e) for the row, so that
 // sigma p = 2^(z log2(e) + krow) takes one FMA per entry.
+template <int FEAT>
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
                                            int vglob0, int vlim, int yl, bool valid,
                                            float krow, float rrow, int row, int lane,
@@ -535,7 +541,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
     for (int j = 0; j < 32; ++j)
       if (j == jt) gv[j] -= g.sigma;
   }
-  if (g.keep_g != nullptr) {
+  if (FEAT & kFeatFilter) {
     // gradient filtering: does this row hold an entry that is not negligible?
 #pragma unroll
     for (int j = 0; j < 32; ++j) big |= fabsf(gv[j]) >= g.filter_eps_sigma;
@@ -566,7 +572,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
       packed[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
   }
-  if (g.db_acc != nullptr) {
+  if (FEAT & kFeatBias) {
     // bias gradient: this warp's 32 rows of the chunk, in fp32 (target
     // entries included exactly), added as 2^-32 fixed-point integers
     const float cs = warp_column_sums(gv, lane);
@@ -595,7 +601,7 @@ __device__ __forceinline__ void stage_row128(uint8_t* stg, int r, int chunk0,
 // ---------------------------------------------------------------------------
 // The kernel (launched as clusters of 2 CTAs)
 // ---------------------------------------------------------------------------
-template <int MODE>
+template <int MODE, int FEAT = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_constant__ GemmArgs g) {
   constexpr int STAGES = ModeCfg<MODE>::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -728,8 +734,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           }
           uint32_t act = 0;
           for (int kb = 0; kb < un.nk; ++kb) {
-            if ((kb & 31) == 0) act = active_mask32<MODE>(g, un, kb);
-            if (!((act >> (kb & 31)) & 1u)) continue;
+            if (FEAT & kFeatFilter) {
+              if ((kb & 31) == 0) act = active_mask32<MODE, FEAT>(g, un, kb);
+              if (!((act >> (kb & 31)) & 1u)) continue;
+            }
             const uint32_t stage = n_issued % STAGES;
             const uint32_t phase = (n_issued / STAGES) & 1u;
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, g.err)) {
@@ -771,7 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           if (u < 0) break;
           const Unit un = decode_unit<MODE>(g, us, C, u);
           // the filtering flags of the panel being read come from the previous launch
-          if (MODE == kModeBwd && g.keep_wh != nullptr && un.cls != kClsGrad) griddep_wait();
+          if (MODE == kModeBwd && (FEAT & kFeatFilter) && un.cls != kClsGrad) griddep_wait();
           if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, g.err)) break;
           tc_fence_after();
           const bool a_mn = unit_a_mn<MODE>(g, un);
@@ -786,8 +794,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           bool first = true;  // the first k-block issued overwrites the accumulator
           uint32_t act = 0;
           for (int kb = 0; kb < un.nk; ++kb) {
-            if ((kb & 31) == 0) act = active_mask32<MODE>(g, un, kb);
-            if (!((act >> (kb & 31)) & 1u)) continue;
+            if (FEAT & kFeatFilter) {
+              if ((kb & 31) == 0) act = active_mask32<MODE, FEAT>(g, un, kb);
+              if (!((act >> (kb & 31)) & 1u)) continue;
+            }
             const uint32_t stage = n_used % STAGES;
             const uint32_t phase = (n_used / STAGES) & 1u;
             if (!mbar_wait(&full[stage], phase, abort_flag, g.err)) {
@@ -904,10 +914,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 
       if (MODE == kModeFwd) {
         // (m, s) of this warpgroup's 128 columns.  Chunks stream out of TMEM
-        // two at a time (one loading while the other is reduced), and the
-        // accumulator goes back to the MMA issuer as soon as the last chunk
-        // has been read.  (Reading all four first and releasing before any
-        // arithmetic measured slower: 8 % on the forward at D = 64 and 128.)
+        // two at a time (one loading while the other is reduced); the
+        // accumulator goes back to the MMA issuer after the last chunk's
+        // arithmetic.  (Measured slower: reading all four chunks first, 8 %
+        // on the forward at D = 64 and 128; releasing the accumulator right
+        // after its last read, 2 % here and 2 % on the backward.)
         FwdRowState st{-INFINITY, 0.f, 0.f, false};
         uint32_t za[32], zb[32];
         tmem_ld32(t_acc + c0 * 32, za);
@@ -920,20 +931,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           else
             fwd_chunk<false>(g, za, c * 32, vglob0, vlim, yl, st);
           tmem_wait_ld(zb);
-          const bool last = c + 2 >= c0 + EPI_CHUNKS;
-          if (!last) {
-            tmem_ld32(t_acc + (c + 2) * 32, za);
-          } else {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_on_leader(&tempty[acc]);
-          }
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
           if (g.poly_exp)
             fwd_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
           else
             fwd_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          if (!last) tmem_wait_ld(za);
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
         if (valid && st.have_tgt) g.tgt[row] = st.tgt;
         // the second warpgroup's half of the row joins the first's: one
         // partial per row and tile, stored tile-major (coalesced per warp).
@@ -953,8 +960,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         }
       } else if (MODE == kModeBwd && un.cls == kClsGrad) {
         // Chunks stream out of TMEM two at a time (registers allow no more);
-        // the accumulator is handed back to the MMA issuer as soon as the last
-        // chunk has been read, before its arithmetic.
+        // the accumulator is handed back after the last box.
         uint32_t za[32], zb[32];
         tmem_ld32(t_acc + c0 * 32, za);
         tmem_wait_ld(za);
@@ -966,27 +972,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           tmem_ld32(t_acc + (c + 1) * 32, zb);
           uint32_t pk[16];
           bool big = false;
-          grad_chunk(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk, big);
+          grad_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk, big);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
-          if (c + 2 < c0 + EPI_CHUNKS) {
-            tmem_ld32(t_acc + (c + 2) * 32, za);
-          } else {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_on_leader(&tempty[acc]);
-          }
-          grad_chunk(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
+          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
+          grad_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
                      big);
           stage_row128(stg, r, 4, pk);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
           fence_proxy_async_smem();
-          if (g.keep_g != nullptr) {
+          if (FEAT & kFeatFilter) {
             const bool any = __any_sync(0xffffffffu, big);
             if (lane == 0) s_keep[wg * 4 + q] = any ? 1 : 0;
           }
           named_bar_sync(wg_bar, EPI_WG_THREADS);
-          if (g.keep_g != nullptr) {
+          if (FEAT & kFeatFilter) {
             // gradient filtering: the box (this warpgroup's 128 rows x 64
             // columns) is kept when any of its entries is not negligible;
             // a dropped box is stored as zeros, and the target entries it
@@ -1010,6 +1010,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
             bulk_commit_group();
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else if (MODE == kModeBwd) {
         // dW (class 0) or dH (class 1): fp32, scaled by lambda / (C sigma)
         const bool is_dw = un.cls == kClsDW;
@@ -1017,13 +1020,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         const int y = is_dw ? g.vp_wh + tm0 : tm0;
         const bool reduce = !is_dw && g.dh_accumulate;
         bool zero = (un.nk == 0);
-        if (g.keep_wh != nullptr && !zero) {
+        if ((FEAT & kFeatFilter) && !zero) {
           // with filtering, no MMA ran when every k-block was skipped: the
           // warp scans the unit's flags (from the previous launch)
           griddep_wait();
           bool any = false;
           for (int kb0 = 32 * lane; kb0 < un.nk && !any; kb0 += 32 * 32)
-            any = active_mask32<MODE>(g, un, kb0) != 0;
+            any = active_mask32<MODE, FEAT>(g, un, kb0) != 0;
           zero = !__any_sync(0xffffffffu, any);
         }
         // a dW half that starts past the panel's last row has nothing to store;
