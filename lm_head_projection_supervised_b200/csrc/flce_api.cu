@@ -198,6 +198,8 @@ flce_status device_setup(DevInfo* out) {
         size_t smem;
       } kernels[] = {
           {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd>), ModeCfg<kModeFwd>::SMEM_BYTES},
+          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd, kFeatPolyExp>),
+           ModeCfg<kModeFwd>::SMEM_BYTES},
           {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, 0>),
            ModeCfg<kModeBwd>::SMEM_BYTES},
           {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatBias>),
@@ -483,9 +485,12 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   a.part_ld = static_cast<int>(L.Np);
   a.tgt = p.tgt;
   a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
-  a.poly_exp = D <= kPolyExpMaxD ? 1 : 0;
   a.err = p.err;
-  FLCE_CK(launch_gemm<kModeFwd>(a, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
+  const int64_t fwd_units = cdiv64(N, PAIR_M) * L.nvt;
+  if (D <= kPolyExpMaxD)
+    FLCE_CK((launch_gemm<kModeFwd, kFeatPolyExp>(a, fwd_units, di.pairs, s)));
+  else
+    FLCE_CK(launch_gemm<kModeFwd>(a, fwd_units, di.pairs, s));
 
   // 32 rows per block pass, at most 8 blocks per SM
   const int64_t blocks =

@@ -16,8 +16,8 @@
 // lane = tile row) and run the epilogue while the next unit accumulates in
 // the other.
 //
-// Modes (one launch = one mode; the backward is instantiated once per
-// combination of its optional features, FEAT = kFeatBias | kFeatFilter):
+// Modes (one launch = one mode; each mode is instantiated once per
+// combination of its optional features FEAT, see Feature):
 //   kModeFwd   Z = H_c W^T (+ b) per 128 x 256 tile; the epilogue keeps the
 //              running max / rescaled exp-sum over the tile's columns and
 //              captures the target logit from the tile that holds it
@@ -108,10 +108,11 @@ struct ModeCfg {
 };
 constexpr size_t GEMM_SMEM_BYTES = ModeCfg<kModeBwd>::SMEM_BYTES;  // the largest
 enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
-// Optional work of the backward, chosen when the kernel is compiled (one
-// instantiation per combination), so that the common path carries none of
-// its code: measured, the runtime-switched form cost the backward 3-4 %.
-enum BwdFeature : int { kFeatBias = 1, kFeatFilter = 2 };
+// Optional work, chosen when the kernel is compiled (one instantiation per
+// combination), so that the common path carries none of its code: measured,
+// the runtime-switched form cost the backward 3-4 %.  Backward: bias column
+// sums, gradient filtering.  Forward: one exponential in four on the FMA pipe.
+enum Feature : int { kFeatBias = 1, kFeatFilter = 2, kFeatPolyExp = 4 };
 
 struct GemmArgs {
   CUtensorMap tmA[3];  // A operand map per unit class (fwd / plain use [0])
@@ -140,8 +141,6 @@ struct GemmArgs {
   const int* idx;          // compact row -> original row
   const uint16_t* bias;    // 16-bit bias [V] or null
   int round_logits;        // round each logit to the 16-bit input type first
-  int poly_exp;            // fwd: one exponential in four on the FMA pipe (ex2_poly), for
-                           // small D
   float2* part;            // fwd: (m, s) partials [tiles][part_ld], part_ld >= rows
   int part_ld;
   float* tgt;              // fwd: target logits [rows]
@@ -926,16 +925,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 #pragma unroll 1
         for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
           tmem_ld32(t_acc + (c + 1) * 32, zb);
-          if (g.poly_exp)
-            fwd_chunk<true>(g, za, c * 32, vglob0, vlim, yl, st);
-          else
-            fwd_chunk<false>(g, za, c * 32, vglob0, vlim, yl, st);
+          fwd_chunk<(FEAT & kFeatPolyExp) != 0>(g, za, c * 32, vglob0, vlim, yl, st);
           tmem_wait_ld(zb);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          if (g.poly_exp)
-            fwd_chunk<true>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          else
-            fwd_chunk<false>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          fwd_chunk<(FEAT & kFeatPolyExp) != 0>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
         }
         tc_fence_before();
