@@ -23,6 +23,7 @@
 //   with row scales s_k = S r_k computed first (row_scale_kernel); the panels
 //   hold r_k (p - onehot) sigma and the dW / dH epilogues multiply by S / sigma.
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/flce.h"
@@ -169,6 +170,37 @@ bool make_map(CUtensorMap* m, const void* base, MapType t, uint64_t inner, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---- the GEMM kernel's instantiations: one per mode and combination of the
+// optional features that mode can use (bias, rounding of the logits, and the
+// forward's polynomial exponentials or the backward's gradient filtering)
+using GemmKernel = void (*)(GemmArgs);
+using FwdFeats = std::integer_sequence<int, 0, kFeatBias, kFeatPolyExp, kFeatBias | kFeatPolyExp,
+                                       kFeatRound, kFeatRound | kFeatBias,
+                                       kFeatRound | kFeatPolyExp,
+                                       kFeatRound | kFeatBias | kFeatPolyExp>;
+using BwdFeats = std::integer_sequence<int, 0, kFeatBias, kFeatFilter, kFeatBias | kFeatFilter,
+                                       kFeatRound, kFeatRound | kFeatBias,
+                                       kFeatRound | kFeatFilter,
+                                       kFeatRound | kFeatBias | kFeatFilter>;
+using PlainFeats = std::integer_sequence<int, 0>;
+
+template <int MODE, int... F>
+GemmKernel pick_kernel(int feat, std::integer_sequence<int, F...>) {
+  GemmKernel k = nullptr;
+  ((feat == F ? (k = flce_gemm_kernel<MODE, F>, 0) : 0), ...);
+  return k;
+}
+template <int MODE>
+GemmKernel gemm_kernel(int feat) {
+  if constexpr (MODE == kModeFwd) return pick_kernel<MODE>(feat, FwdFeats{});
+  else if constexpr (MODE == kModeBwd) return pick_kernel<MODE>(feat, BwdFeats{});
+  else return pick_kernel<MODE>(feat, PlainFeats{});
+}
+template <int MODE, int... F, class Fn>
+void each_kernel(std::integer_sequence<int, F...>, Fn&& fn) {
+  (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>), ModeCfg<MODE>::SMEM_BYTES), ...);
+}
+
 // ---- per-device set-up
 struct DevInfo {
   bool init = false;
@@ -193,33 +225,23 @@ flce_status device_setup(DevInfo* out) {
       return FLCE_ERR_CUDA;
     d.ok = (major == 10 && minor == 0) && encode_fn() != nullptr;
     if (d.ok) {
-      const struct {
-        const void* fn;
-        size_t smem;
-      } kernels[] = {
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd>), ModeCfg<kModeFwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeFwd, kFeatPolyExp>),
-           ModeCfg<kModeFwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, 0>),
-           ModeCfg<kModeBwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatBias>),
-           ModeCfg<kModeBwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatFilter>),
-           ModeCfg<kModeBwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModeBwd, kFeatBias | kFeatFilter>),
-           ModeCfg<kModeBwd>::SMEM_BYTES},
-          {reinterpret_cast<const void*>(flce_gemm_kernel<kModePlain>),
-           ModeCfg<kModePlain>::SMEM_BYTES}};
-      for (const auto& k : kernels) {
-        if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(k.smem)) != cudaSuccess)
-          return FLCE_ERR_CUDA;
+      bool fail = false;
+      auto setup = [&](const void* fn, size_t smem) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess) {
+          fail = true;
+          return;
+        }
         // The GEMM kernels split registers between warpgroups with setmaxnreg;
         // the split only fits if the block was launched with enough of them.
         cudaFuncAttributes fa{};
-        if (cudaFuncGetAttributes(&fa, k.fn) != cudaSuccess) return FLCE_ERR_CUDA;
-        if (fa.numRegs < static_cast<int>(kRegsAtLaunch)) d.ok = false;
-      }
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) fail = true;
+        else if (fa.numRegs < static_cast<int>(kRegsAtLaunch)) d.ok = false;
+      };
+      each_kernel<kModeFwd>(FwdFeats{}, setup);
+      each_kernel<kModeBwd>(BwdFeats{}, setup);
+      each_kernel<kModePlain>(PlainFeats{}, setup);
+      if (fail) return FLCE_ERR_CUDA;
     }
     if (d.ok) {
       // how many CTA pairs can be resident together (one CTA per SM)
@@ -315,9 +337,11 @@ void prof_span_end(ProfRec* r, int launches, cudaStream_t s) {
 // pdl: the launch may start before the previous kernel of the stream ends
 // (programmatic stream serialisation; the kernel waits where it must).
 // timed: wrap the launch in profiling events (off inside a timed span).
-template <int MODE, int FEAT = 0>
-cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaStream_t s,
-                        bool pdl = false, bool timed = true) {
+template <int MODE>
+cudaError_t launch_gemm(const GemmArgs& a, int feat, int64_t units_upper, int pairs,
+                        cudaStream_t s, bool pdl = false, bool timed = true) {
+  const GemmKernel kernel = gemm_kernel<MODE>(feat);
+  if (kernel == nullptr) return cudaErrorInvalidValue;
   if (units_upper <= 0) return cudaSuccess;
   const int npairs = static_cast<int>(units_upper < pairs ? units_upper : pairs);
   const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeBwd ? kProfBwd : kProfPlain;
@@ -336,7 +360,7 @@ cudaError_t launch_gemm(const GemmArgs& a, int64_t units_upper, int pairs, cudaS
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    cudaLaunchKernelEx(&cfg, flce_gemm_kernel<MODE, FEAT>, a);
+    cudaLaunchKernelEx(&cfg, kernel, a);
   };
   if (!timed) {
     launch();
@@ -484,13 +508,11 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   a.part = p.part;
   a.part_ld = static_cast<int>(L.Np);
   a.tgt = p.tgt;
-  a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
   a.err = p.err;
-  const int64_t fwd_units = cdiv64(N, PAIR_M) * L.nvt;
-  if (D <= kPolyExpMaxD)
-    FLCE_CK((launch_gemm<kModeFwd, kFeatPolyExp>(a, fwd_units, di.pairs, s)));
-  else
-    FLCE_CK(launch_gemm<kModeFwd>(a, fwd_units, di.pairs, s));
+  const int feat = (b != nullptr ? kFeatBias : 0) |
+                   ((flags & FLCE_FLAG_ROUND_LOGITS) ? kFeatRound : 0) |
+                   (D <= kPolyExpMaxD ? kFeatPolyExp : 0);
+  FLCE_CK(launch_gemm<kModeFwd>(a, feat, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
   // 32 rows per block pass, at most 8 blocks per SM
   const int64_t blocks =
@@ -640,7 +662,6 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     a.row_scale = p.rs;
     a.tgt_resid = p.resid;
     a.scal = p.scal;
-    a.round_logits = (flags & FLCE_FLAG_ROUND_LOGITS) ? 1 : 0;
     a.inv_sigma = 1.f / sigma;
     a.db_acc = b != nullptr ? p.dbacc : nullptr;
     a.db_fx_scale = 0x1p32f / sigma;
@@ -656,22 +677,10 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     const int64_t units = (has_wh ? cdiv64(w_wh, PAIR_M) * nD + nT_max * nD : 0) +
                           (has_g ? nT_max * cdiv64(w_g, BN) : 0);
     // every launch after the first may overlap its predecessor
-    const bool pdl = launched > 0;
-    cudaError_t e;
-    switch ((b != nullptr ? kFeatBias : 0) | (filter_eps > 0.f ? kFeatFilter : 0)) {
-      case kFeatBias:
-        e = launch_gemm<kModeBwd, kFeatBias>(a, units, di.pairs, s, pdl, false);
-        break;
-      case kFeatFilter:
-        e = launch_gemm<kModeBwd, kFeatFilter>(a, units, di.pairs, s, pdl, false);
-        break;
-      case kFeatBias | kFeatFilter:
-        e = launch_gemm<kModeBwd, kFeatBias | kFeatFilter>(a, units, di.pairs, s, pdl, false);
-        break;
-      default:
-        e = launch_gemm<kModeBwd, 0>(a, units, di.pairs, s, pdl, false);
-    }
-    FLCE_CK(e);
+    const int feat = (b != nullptr ? kFeatBias : 0) | (filter_eps > 0.f ? kFeatFilter : 0) |
+                     ((flags & FLCE_FLAG_ROUND_LOGITS) ? kFeatRound : 0);
+    FLCE_CK(launch_gemm<kModeBwd>(a, feat, units, di.pairs, s, /*pdl=*/launched > 0,
+                                  /*timed=*/false));
     launched += units > 0 ? 1 : 0;
   }
   if (timed) prof_span_end(&span, launched, s);
@@ -958,7 +967,7 @@ flce_status flce_diag_gemm(const void* A, const void* B, float* out, int64_t M, 
   a.err = static_cast<uint32_t*>(ws);
   a.counter = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + kCounterOffset);
   FLCE_CK(cudaMemsetAsync(ws, 0, 256, s));
-  FLCE_CK(launch_gemm<kModePlain>(a, cdiv64(M, PAIR_M) * cdiv64(N, BN), di.pairs, s));
+  FLCE_CK(launch_gemm<kModePlain>(a, 0, cdiv64(M, PAIR_M) * cdiv64(N, BN), di.pairs, s));
   return FLCE_OK;
 }
 

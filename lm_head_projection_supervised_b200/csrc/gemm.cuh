@@ -83,8 +83,10 @@ constexpr int EPI_CHUNKS = BN / 32 / NUM_EPI_WG;  // 32-column chunks per epilog
 // Registers per thread after the split: the first warpgroup gives up what the
 // epilogue takes.  The block is launched with at least kRegsAtLaunch per
 // thread (checked on the host before any launch), which covers the split.
-constexpr uint32_t kRegsLow = 72;  // 56 spilled in the producers (backward 4 % slower)
-constexpr uint32_t kRegsHigh = 216;
+// 80 / 208 is the split at which no instantiation spills: 72 / 216 spilled
+// in the plain forward and backward variants, 56 in the producers.
+constexpr uint32_t kRegsLow = 80;
+constexpr uint32_t kRegsHigh = 208;
 constexpr uint32_t kRegsAtLaunch =
     (128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh + NUM_THREADS - 1) / NUM_THREADS;
 static_assert(128 * kRegsLow + NUM_EPI_THREADS * kRegsHigh <= 65536, "register split");
@@ -110,9 +112,11 @@ constexpr size_t GEMM_SMEM_BYTES = ModeCfg<kModeBwd>::SMEM_BYTES;  // the larges
 enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
 // Optional work, chosen when the kernel is compiled (one instantiation per
 // combination), so that the common path carries none of its code: measured,
-// the runtime-switched form cost the backward 3-4 %.  Backward: bias column
-// sums, gradient filtering.  Forward: one exponential in four on the FMA pipe.
-enum Feature : int { kFeatBias = 1, kFeatFilter = 2, kFeatPolyExp = 4 };
+// the runtime-switched form cost the backward 3-4 %.  Both passes: the bias
+// (its add to the logits, and in the backward its column sums) and the
+// rounding of the logits to the input type.  Backward: gradient filtering.
+// Forward: one exponential in four on the FMA pipe.
+enum Feature : int { kFeatBias = 1, kFeatFilter = 2, kFeatPolyExp = 4, kFeatRound = 8 };
 
 struct GemmArgs {
   CUtensorMap tmA[3];  // A operand map per unit class (fwd / plain use [0])
@@ -140,7 +144,6 @@ struct GemmArgs {
   const int* y_c;          // compact labels
   const int* idx;          // compact row -> original row
   const uint16_t* bias;    // 16-bit bias [V] or null
-  int round_logits;        // round each logit to the 16-bit input type first
   float2* part;            // fwd: (m, s) partials [tiles][part_ld], part_ld >= rows
   int part_ld;
   float* tgt;              // fwd: target logits [rows]
@@ -432,19 +435,20 @@ __device__ __forceinline__ float ex2_elem(float x, int j) {
   return (POLY && (j & 3) == 3) ? ex2_poly(x) : ex2_approx(x);
 }
 
-template <bool POLY>
+template <int FEAT>
 __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb, int vglob0,
                                           int vlim, int yl, FwdRowState& st) {
+  constexpr bool POLY = (FEAT & kFeatPolyExp) != 0;
   float x[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(z[j]);
-  if (g.bias != nullptr) {
+  if (FEAT & kFeatBias) {
     float bv[32];
     load_bias32(g.bias, vglob0 + cb, g.V, g.is_bf16 != 0, bv);
 #pragma unroll
     for (int j = 0; j < 32; ++j) x[j] += bv[j];
   }
-  if (g.round_logits) round_to_input_type(g, x);
+  if (FEAT & kFeatRound) round_to_input_type(g, x);
   if (cb + 32 > vlim) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -514,13 +518,13 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   float x[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(z[j]);
-  if (g.bias != nullptr) {
+  if (FEAT & kFeatBias) {
     float bv[32];
     load_bias32(g.bias, vglob0 + cb, g.V, g.is_bf16 != 0, bv);
 #pragma unroll
     for (int j = 0; j < 32; ++j) x[j] += bv[j];
   }
-  if (g.round_logits) round_to_input_type(g, x);
+  if (FEAT & kFeatRound) round_to_input_type(g, x);
   float gv[32];
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
 #pragma unroll
@@ -925,10 +929,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
 #pragma unroll 1
         for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
           tmem_ld32(t_acc + (c + 1) * 32, zb);
-          fwd_chunk<(FEAT & kFeatPolyExp) != 0>(g, za, c * 32, vglob0, vlim, yl, st);
+          fwd_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, st);
           tmem_wait_ld(zb);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          fwd_chunk<(FEAT & kFeatPolyExp) != 0>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+          fwd_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
           if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
         }
         tc_fence_before();
