@@ -57,6 +57,9 @@ def parse():
                    help="one vocabulary slice per rank (P = number of ranks, a one-rank NCCL "
                         "group without torchrun), statistics all-gathered and dH all-reduced "
                         "with NCCL; strong scaling (the whole vocabulary is split)")
+    p.add_argument("--panel-backward", action="store_true",
+                   help="the panel form of the backward where the single-kernel form applies "
+                        "(D <= 64)")
     p.add_argument("--filter-eps", type=float, default=0.0,
                    help="> 0: the backward with gradient filtering (an approximation; see "
                         "flce_backward_filtered)")
@@ -86,16 +89,18 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_kind):
+def ncu_traffic(kernel_kind, workload):
     """DRAM bytes per launch of `kernel_kind` from the committed ncu summary,
-    or None when absent or taken on a different version of the kernel."""
+    or None when absent, taken on another workload or on a different version
+    of the kernel."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel_kind)
-    if not e or e.get("source_hash") != source_hash(GEMM_SOURCES):
+    if not e or e.get("source_hash") != source_hash(GEMM_SOURCES) or \
+            e.get("workload", "packed") != workload:
         return None
     return e.get("bytes_per_launch")
 
@@ -376,6 +381,8 @@ def main():
 
     inp = wl.make_inputs(spec, seed=wl.SEED_BASE + spec.k + 1000 * rank)
     cfg = workload_config(spec, inp, world)
+    cfg["backward"] = ("single-kernel" if inp.D <= 64 and not args.panel_backward and
+                       args.filter_eps <= 0 else "panel")
     if args.filter_eps > 0:
         cfg["filter_eps"] = args.filter_eps
         cfg["note"] = "backward with gradient filtering: an approximation, not the exact path"
@@ -428,6 +435,7 @@ def main():
                 binding.shard_backward(H, W[v0:v0 + n], None if b is None else b[v0:v0 + n], y,
                                        mk, -100, m, logs, v0=v0, V_total=inp.V, lam=inp.lam,
                                        ws=ws, accumulate_dh=r > 0,
+                                       panel_backward=args.panel_backward,
                                        out=(dH, dW[v0:v0 + n],
                                             None if db is None else db[v0:v0 + n]))
     else:
@@ -439,7 +447,8 @@ def main():
             H, W, b, y, mk = x
             # the forward's compaction and gathered rows are still in ws
             binding.backward(H, W, b, y, mk, -100, m, logs, lam=inp.lam, ws=ws,
-                             out=(dH, dW, db), reuse_forward=True, filter_eps=args.filter_eps)
+                             out=(dH, dW, db), reuse_forward=True, filter_eps=args.filter_eps,
+                             panel_backward=args.panel_backward)
 
     inputs = (H, W, b, y, mk)
 
@@ -600,7 +609,7 @@ def main():
     # fp16 and bf16 share the dense tensor-core rate on this part.
     peak = peaks.get("bf16_tflops")
     peak_sus = peaks.get("bf16_tflops_sustained")
-    tb = ncu_traffic(dom)
+    tb = ncu_traffic(dom, spec.name) if not cfg.get("backward", "").startswith("single") else None
     alg_launch = bytes_per_step[dom] * args.steps / max(n_l, 1)
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak,

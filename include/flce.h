@@ -82,7 +82,9 @@ typedef enum { FLCE_BF16 = 0, FLCE_FP16 = 1 } flce_dtype;
 typedef void* flce_stream;
 
 /* Bytes of device workspace needed for problem size (N, D, V).  Returns 0
- * when the sizes are out of range (same limits as FLCE_ERR_SHAPE). */
+ * when the sizes are out of range (same limits as FLCE_ERR_SHAPE).  For
+ * D <= 64 it includes the single-kernel backward's partial sums (see
+ * flce_backward), about ceil(N / 256) * V * D * 4 bytes. */
 FLCE_API size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype);
 
 /*
@@ -126,6 +128,14 @@ FLCE_API flce_status flce_forward(const void* H, const void* W, const void* b,
  *
  * dH, dW and db are deterministic: every output element is reduced in a
  * fixed order independent of scheduling.
+ *
+ * Two forms of the same computation.  D > 64 (or FLCE_FLAG_PANEL_BACKWARD):
+ * the gradient of the logits is staged in 16 bits, one vocabulary panel of
+ * 8192 ids at a time, and read by the dW and dH contractions.  D <= 64: one
+ * kernel per call does the score tile, the gradient and both contractions
+ * per 256-row x 128-id tile (§04's single fused pass: dH of the row block
+ * accumulates across the vocabulary on chip, dW is summed from one partial
+ * per 256-row block in a fixed order by a second kernel).
  */
 FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
                           const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
@@ -208,6 +218,11 @@ typedef enum { FLCE_REDUCE_MEAN = 0, FLCE_REDUCE_SUM = 1, FLCE_REDUCE_NONE = 2 }
  *   H, labels and mask did not change in between; the result is undefined
  *   otherwise.  A device error recorded by that forward stays recorded. */
 #define FLCE_FLAG_REUSE_FORWARD 4u
+/* FLCE_FLAG_PANEL_BACKWARD (backward calls only): use the panel form of the
+ *   backward where the single-kernel form would apply (D <= 64); the results
+ *   agree within rounding (see flce_backward).  Gradient filtering always
+ *   uses the panel form. */
+#define FLCE_FLAG_PANEL_BACKWARD 8u
 
 /*
  * Forward with a reduction.  weight: device float [N] or NULL.  loss: device

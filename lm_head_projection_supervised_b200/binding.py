@@ -25,6 +25,7 @@ REDUCTIONS = {"mean": 0, "sum": 1, "none": 2}
 FLAG_ROUND_LOGITS = 1
 FLAG_ACCUMULATE_DH = 2
 FLAG_REUSE_FORWARD = 4
+FLAG_PANEL_BACKWARD = 8
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
 _lib = None
@@ -181,10 +182,12 @@ def _mask_u8(mask):
     return mk.contiguous()
 
 
-def _flags(round_logits=False, accumulate_dh=False, reuse_forward=False) -> int:
+def _flags(round_logits=False, accumulate_dh=False, reuse_forward=False,
+           panel_backward=False) -> int:
     return (FLAG_ROUND_LOGITS if round_logits else 0) | \
         (FLAG_ACCUMULATE_DH if accumulate_dh else 0) | \
-        (FLAG_REUSE_FORWARD if reuse_forward else 0)
+        (FLAG_REUSE_FORWARD if reuse_forward else 0) | \
+        (FLAG_PANEL_BACKWARD if panel_backward else 0)
 
 
 def _vec(t, N, device):
@@ -230,7 +233,7 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
              ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
              reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
              round_logits: bool = False, accumulate_dh: bool = False,
-             reuse_forward: bool = False, filter_eps: float = 0.0):
+             reuse_forward: bool = False, filter_eps: float = 0.0, panel_backward: bool = False):
     """dH [N, D], dW [V, D], db [V] or None (float32) -- flce_backward_ex(), or
     flce_backward_filtered() when filter_eps > 0 (gradient filtering: 128-row x
     64-id blocks whose |p - onehot| are all below filter_eps are left out of
@@ -240,7 +243,9 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
     loss; otherwise lam (or the device scalar lam_dev) is dJ/dL.  With
     accumulate_dh the call adds its dH to out[0] instead of overwriting it.
     reuse_forward: `ws` holds the compaction of a forward() on the same
-    inputs, untouched since; the backward skips redoing it."""
+    inputs, untouched since; the backward skips redoing it.  panel_backward:
+    the panel form of the backward even where the single-kernel form applies
+    (D <= 64)."""
     H2, W2, b2, y, mk = _prep(H, W, b, labels, mask)
     N, D = H2.shape
     V = W2.shape[0]
@@ -259,7 +264,8 @@ def backward(H, W, b, labels, mask, ignore_index: int, m, logs, lam: float = 1.0
     gr = _vec(grad_rows, N, H2.device)
     common = (_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index, N, D, V,
               dtype_code(H2.dtype), _ptr(m), _ptr(logs), _ptr(wt), red, float(denom or 0.0),
-              _flags(round_logits, accumulate_dh, reuse_forward), float(lam), _ptr(lam_dev),
+              _flags(round_logits, accumulate_dh, reuse_forward, panel_backward), float(lam),
+              _ptr(lam_dev),
               _ptr(gr))
     tail = (_ptr(dH), _ptr(dW), _ptr(db), ws.ptr(), ws.nbytes, _stream(stream))
     if filter_eps:
@@ -343,7 +349,8 @@ def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index: int, m, logs
                    V_total: Optional[int] = None, lam: float = 1.0, lam_dev=None,
                    ws: Optional[Workspace] = None, out=None, stream=None, weight=None,
                    reduction: str = "mean", denom: Optional[float] = None, grad_rows=None,
-                   round_logits: bool = False, accumulate_dh: bool = False):
+                   round_logits: bool = False, accumulate_dh: bool = False,
+                   panel_backward: bool = False):
     """(dH_r [N, D], dW_slice [V_slice, D], db_slice [V_slice] or None),
     float32 -- flce_shard_backward().  dH_r is this slice's term of dH (added
     to out[0] with accumulate_dh)."""
@@ -366,7 +373,9 @@ def shard_backward(H, W_slice, b_slice, labels, mask, ignore_index: int, m, logs
     st = lib().flce_shard_backward(_ptr(H2), _ptr(W2), _ptr(b2), _ptr(y), _ptr(mk), ignore_index,
                                    N, D, Vs, int(v0), V_total, dtype_code(H2.dtype), _ptr(m),
                                    _ptr(logs), _ptr(wt), REDUCTIONS[reduction],
-                                   float(denom or 0.0), _flags(round_logits, accumulate_dh),
+                                   float(denom or 0.0),
+                                   _flags(round_logits, accumulate_dh,
+                                          panel_backward=panel_backward),
                                    float(lam), _ptr(lam_dev), _ptr(gr), _ptr(dH), _ptr(dW),
                                    _ptr(db), ws.ptr(), ws.nbytes, _stream(stream))
     _check(st, "flce_shard_backward")

@@ -30,6 +30,7 @@
 #include "../../include/flce_diag.h"
 #include "aux_kernels.cuh"
 #include "gemm.cuh"
+#include "fused_bwd.cuh"
 
 using namespace flce;
 
@@ -62,9 +63,12 @@ constexpr int kPanelBufs = 3;  // panel buffers: written, read, and one of slack
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
   size_t pos, rs, resid, skeys[2], svals[2], rscount, dbacc, keep, keep_bytes, dhc;
-  size_t gpanel[kPanelBufs], total;
+  size_t gpanel[kPanelBufs], dwp, dhp, total;
   int64_t Np, nvt, vc, gld, panels;
+  bool fused;   // the single-kernel backward applies (D <= 64)
+  int64_t Vp;   // its dW partials: FB_NG_MAX slabs of Vp rows
 };
+
 
 // Workspace carve-up.  The control block (error word, then one work counter
 // per GEMM launch) sits at offset 0 for every size.  The regions the forward
@@ -102,11 +106,25 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   }
   L.rscount = take(static_cast<size_t>(RS_DIGITS) * cdiv64(L.Np, RS_TILE) * 4);
   L.dbacc = take(static_cast<size_t>(V) * 8);  // bias gradient, fixed point per vocabulary id
+  L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
+  // What follows is used by one of the two backward forms only: the panel
+  // backward's flags and panels, or the single-kernel backward's partials.
+  const size_t shared_base = off;
   // gradient filtering: one keep flag per 128-row x 64-column box of each panel buffer
   L.keep_bytes = static_cast<size_t>(L.Np / BM) * static_cast<size_t>(L.gld / 64);
   L.keep = take(L.keep_bytes * kPanelBufs);
-  L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
   for (int i = 0; i < kPanelBufs; ++i) L.gpanel[i] = take(static_cast<size_t>(L.Np) * L.gld * 2);
+  const size_t panel_end = off;
+  L.Vp = roundup64(V, FB_COLS);
+  // (the partials' TMA coordinates are 32-bit)
+  L.fused = D <= FB_MAX_D && FB_NG_MAX * L.Vp < (int64_t(1) << 31) &&
+            FB_NCH_MAX * L.Np < (int64_t(1) << 31);
+  if (L.fused) {
+    off = shared_base;
+    L.dwp = take(static_cast<size_t>(FB_NG_MAX * L.Vp * D) * 4);
+    L.dhp = take(static_cast<size_t>(FB_NCH_MAX) * static_cast<size_t>(L.Np) * D * 4);
+    if (off < panel_end) off = panel_end;
+  }
   L.total = off;
   return L;
 }
@@ -200,6 +218,19 @@ template <int MODE, int... F, class Fn>
 void each_kernel(std::integer_sequence<int, F...>, Fn&& fn) {
   (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>), ModeCfg<MODE>::SMEM_BYTES), ...);
 }
+// the single-kernel backward: bias and rounding of the logits
+using FusedFeats = std::integer_sequence<int, 0, kFeatBias, kFeatRound, kFeatBias | kFeatRound>;
+using FusedKernel = void (*)(FusedArgs);
+template <int... F>
+FusedKernel pick_fused(int feat, std::integer_sequence<int, F...>) {
+  FusedKernel k = nullptr;
+  ((feat == F ? (k = flce_fused_bwd_kernel<F>, 0) : 0), ...);
+  return k;
+}
+template <int... F, class Fn>
+void each_fused(std::integer_sequence<int, F...>, Fn&& fn) {
+  (fn(reinterpret_cast<const void*>(flce_fused_bwd_kernel<F>), FB_SMEM_BYTES), ...);
+}
 
 // ---- per-device set-up
 struct DevInfo {
@@ -241,6 +272,7 @@ flce_status device_setup(DevInfo* out) {
       each_kernel<kModeFwd>(FwdFeats{}, setup);
       each_kernel<kModeBwd>(BwdFeats{}, setup);
       each_kernel<kModePlain>(PlainFeats{}, setup);
+      each_fused(FusedFeats{}, setup);
       if (fail) return FLCE_ERR_CUDA;
     }
     if (d.ok) {
@@ -390,6 +422,8 @@ struct WsPtrs {
   uint8_t* keep;
   float* dhc;
   uint16_t* gpanel[kPanelBufs];
+  float* dwp;  // single-kernel backward: dW partials [FB_NG_MAX][Vp][D]
+  float* dhp;  //   and dH partials [FB_NCH_MAX][Np][D]
 };
 
 WsPtrs carve(void* ws, const Layout& L) {
@@ -417,6 +451,8 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.keep = w + L.keep;
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
   for (int i = 0; i < kPanelBufs; ++i) p.gpanel[i] = reinterpret_cast<uint16_t*>(w + L.gpanel[i]);
+  p.dwp = L.fused ? reinterpret_cast<float*>(w + L.dwp) : nullptr;
+  p.dhp = L.fused ? reinterpret_cast<float*>(w + L.dhp) : nullptr;
   return p;
 }
 
@@ -556,8 +592,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
   if (!(filter_eps >= 0.f) || !isfinite(filter_eps)) return FLCE_ERR_ARG;
   if ((reduction != FLCE_REDUCE_MEAN && reduction != FLCE_REDUCE_SUM &&
        reduction != FLCE_REDUCE_NONE) ||
-      (flags & ~(FLCE_FLAG_ROUND_LOGITS | FLCE_FLAG_ACCUMULATE_DH | FLCE_FLAG_REUSE_FORWARD)) !=
-          0)
+      (flags & ~(FLCE_FLAG_ROUND_LOGITS | FLCE_FLAG_ACCUMULATE_DH | FLCE_FLAG_REUSE_FORWARD |
+                 FLCE_FLAG_PANEL_BACKWARD)) != 0)
     return FLCE_ERR_ARG;
   const bool none = reduction == FLCE_REDUCE_NONE;
   if ((N > 0 && (H == nullptr || labels == nullptr || m == nullptr || logs == nullptr ||
@@ -605,17 +641,74 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       !make_map(&dhMap, p.dhc, kMapF32, D, L.Np, D * 4, 32, BM))
     return FLCE_ERR_CUDA;
 
+  const bool fused =
+      L.fused && filter_eps == 0.f && (flags & FLCE_FLAG_PANEL_BACKWARD) == 0;
+  if (b != nullptr) FLCE_CK(cudaMemsetAsync(p.dbacc, 0, static_cast<size_t>(V) * 8, s));
+  if (fused) {
+    // single kernel: scores, gradient and both contractions per tile, then
+    // the fixed-order sums of the dW and dH slabs
+    FusedArgs fa{};
+    GemmArgs& a = fa.g;
+    a.tmA[0] = hcK;
+    a.tmB[0] = wK;
+    if (!make_map(&a.tmDW, p.dwp, kMapF32, D, FB_NG_MAX * L.Vp, D * 4, 32, BM) ||
+        !make_map(&a.tmDH, p.dhp, kMapF32, D, FB_NCH_MAX * L.Np, D * 4, 32, BM))
+      return FLCE_ERR_CUDA;
+    a.is_bf16 = bf16;
+    a.C_dev = p.C;
+    a.counter = p.counters + 1;
+    a.D = static_cast<int>(D);
+    a.V = static_cast<int>(V);
+    a.y_c = p.yc;
+    a.idx = p.idx;
+    a.bias = static_cast<const uint16_t*>(b);
+    a.m_saved = m;
+    a.logs_saved = logs;
+    a.log2_sigma = log2_sigma;
+    a.sigma = sigma;
+    a.row_scale = p.rs;
+    a.tgt_resid = p.resid;
+    a.scal = p.scal;
+    a.inv_sigma = 1.f / sigma;
+    a.db_acc = b != nullptr ? p.dbacc : nullptr;
+    a.db_fx_scale = 0x1p32f / sigma;
+    a.err = p.err;
+    fa.Vp = static_cast<int>(L.Vp);
+    fa.Np = static_cast<int>(L.Np);
+    fa.nctas = di.sms;
+    const FusedKernel kern = pick_fused(
+        (b != nullptr ? kFeatBias : 0) | ((flags & FLCE_FLAG_ROUND_LOGITS) ? kFeatRound : 0),
+        FusedFeats{});
+    if (kern == nullptr) return FLCE_ERR_ARG;
+    FLCE_CK(timed_launch(kProfBwd, s, [&] {
+      kern<<<static_cast<unsigned>(di.sms), NUM_THREADS, FB_SMEM_BYTES, s>>>(fa);
+    }));
+    const int64_t D4 = D / 4;
+    const int64_t dw_blocks = cdiv64(V * D4, 256) < 8LL * di.sms ? cdiv64(V * D4, 256) : 8LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      fused_reduce_dw_kernel<<<static_cast<unsigned>(dw_blocks), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(p.dwp), L.Vp * D4, static_cast<int>(V),
+          static_cast<int>(D4), p.C, di.sms, p.scal, 1.f / sigma, reinterpret_cast<float4*>(dW));
+    }));
+    const int64_t dh_blocks =
+        cdiv64(L.Np * D4, 256) < 8LL * di.sms ? cdiv64(L.Np * D4, 256) : 8LL * di.sms;
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      fused_reduce_dh_kernel<<<static_cast<unsigned>(dh_blocks), 256, 0, s>>>(
+          reinterpret_cast<const float4*>(p.dhp), L.Np * D4, static_cast<int>(D4), p.C,
+          static_cast<int>(V), di.sms, p.scal, 1.f / sigma, reinterpret_cast<float4*>(p.dhc));
+    }));
+  }
+
   const int64_t nT_max = cdiv64(N, PAIR_M);
   const int bn_wh = D <= 128 ? 128 : BN;  // dW / dH tile width along D
   const int64_t nD = cdiv64(D, bn_wh);
-  if (b != nullptr) FLCE_CK(cudaMemsetAsync(p.dbacc, 0, static_cast<size_t>(V) * 8, s));
   // The GEMM launches form one timed span: with programmatic dependent launch
   // they overlap, so events between them would measure nothing useful (and
   // would hold the next launch back).
   ProfRec span;
-  const bool timed = prof_span_begin(&span, kProfBwd, s);
+  const bool timed = !fused && prof_span_begin(&span, kProfBwd, s);
   int launched = 0;
-  for (int64_t Lp = 0; Lp <= L.panels; ++Lp) {
+  for (int64_t Lp = 0; !fused && Lp <= L.panels; ++Lp) {
     const bool has_g = Lp < L.panels;
     const bool has_wh = Lp > 0;
     const int64_t vp_g = Lp * L.vc;

@@ -163,6 +163,7 @@ def bwd_ex(L, **kw):
     (dict(red=-1), "FLCE_ERR_ARG"),
     (dict(fl=2), "FLCE_ERR_ARG"),                    # dH accumulation: backward-only bit
     (dict(fl=4), "FLCE_ERR_ARG"),                    # reuse of a forward: backward-only bit
+    (dict(fl=8), "FLCE_ERR_ARG"),                    # panel backward: backward-only bit
     (dict(red=2, rows=None), "FLCE_ERR_NULL"),       # 'none' needs the per-row output
     (dict(red=1, loss=None), "FLCE_ERR_NULL"),       # 'sum' needs the scalar
     (dict(red=0, w=FAKE + 2), "FLCE_ERR_ALIGN"),
@@ -249,10 +250,26 @@ def test_shard_combine_argument_errors(L, kw, want):
     (dict(b=FAKE, db=None), "FLCE_ERR_NULL"),
     (dict(v0=4, Vt=1004, wsb=4096), "FLCE_ERR_WORKSPACE"),
     (dict(v0=10, Vt=1004), "FLCE_ERR_SHAPE"),
-    (dict(fl=8), "FLCE_ERR_ARG"),
+    (dict(fl=16), "FLCE_ERR_ARG"),
 ])
 def test_shard_backward_argument_errors(L, kw, want):
     assert sbwd(L, **kw) == S[want]
+
+
+def test_workspace_holds_the_fused_backward_partials(L):
+    """D <= 64: the workspace carries the single-kernel backward's partial
+    sums (8 dW slabs of V rows, 160 dH slabs of N rows), sharing space with the
+    panel buffers; at the packed shape that is about a sixth of one 16-bit
+    copy of the N x V logits."""
+    N, V = 16384, 248320
+    Vp, Np = (V + 127) // 128 * 128, (N + 255) // 256 * 256
+    for D in (8, 40, 64):
+        ws = L.flce_workspace_bytes(N, D, V, 0)
+        assert ws >= (8 * Vp + 160 * Np) * D * 4
+        assert ws < N * V * 2 / 5
+    # D > 64 has no partials
+    d72 = L.flce_workspace_bytes(N, 72, V, 0)
+    assert d72 < (8 * Vp + 160 * Np) * 72 * 4
 
 
 def test_shard_combine_workspace_bytes(L):
