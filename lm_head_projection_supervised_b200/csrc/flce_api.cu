@@ -651,8 +651,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
     GemmArgs& a = fa.g;
     a.tmA[0] = hcK;
     a.tmB[0] = wK;
-    if (!make_map(&a.tmDW, p.dwp, kMapF32, D, FB_NG_MAX * L.Vp, D * 4, 32, BM) ||
-        !make_map(&a.tmDH, p.dhp, kMapF32, D, FB_NCH_MAX * L.Np, D * 4, 32, BM))
+    if (!make_map(&a.tmDW, p.dwp, kMapF32, D, FB_NG_MAX * L.Vp, D * 4, 32, 32) ||
+        !make_map(&a.tmDH, p.dhp, kMapF32, D, FB_NCH_MAX * L.Np, D * 4, 32, 32))
       return FLCE_ERR_CUDA;
     a.is_bf16 = bf16;
     a.C_dev = p.C;

@@ -26,11 +26,13 @@
 // drains one while the next accumulates.  D > 64 does not fit: dH of 256 rows
 // and a dW tile need 2 D + D columns beside the 256 of the scores.
 //
-// Roles (384 threads): warp 0 schedules items and loads H (once per item) and
-// the W tiles (a ring); warp 1 issues the MMAs; warps 4..11 are two epilogue
-// warpgroups, warpgroup h on row half h (thread = TMEM lane = row), which
-// also drain the dW tiles (lane = vocabulary id, 32 columns each) and the dH
-// halves.  Every wait is bounded (see mbar_wait).
+// Roles (384 threads): warp 0 schedules items and loads H (once per row
+// block) and the W tiles (a ring); warp 1 issues the MMAs; warps 4..11 are two
+// epilogue warpgroups, warpgroup h on row half h (thread = TMEM lane = row),
+// which also drain the dW tiles (lane = vocabulary id, 32 columns each) and
+// the dH halves, each warp its 32 TMEM lanes through its own 4 KiB staging
+// box and TMA, so that the epilogue warps meet only once per row block.
+// Every wait is bounded (see mbar_wait).
 #pragma once
 
 #include "gemm.cuh"
@@ -79,7 +81,7 @@ __host__ __device__ inline FusedPlan fused_plan(int C, int V, int nctas) {
 struct FusedArgs {
   // tmA[0]: H_c, K-major 64 x 128 boxes; tmB[0]: W, K-major 64 x 128 boxes;
   // tmDW: dW partials [FB_NG_MAX * Vp][D] f32; tmDH: dH partials
-  // [FB_NCH_MAX * Np][D] f32 (32 x 128 boxes); the rest as for the backward's
+  // [FB_NCH_MAX * Np][D] f32 (32 x 32 boxes); the rest as for the backward's
   // gradient units
   GemmArgs g;
   int Vp;     // rows per dW slab (V rounded up to a tile)
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sH = smem;                              // [2 buffers][2 halves][16 KiB]
   uint8_t* sW = sH + 2 * FB_HB_BYTES;              // [FB_WSTAGES][16 KiB]
   uint8_t* sG = sW + FB_WSTAGES * FB_W_BYTES;      // [2 halves][2 boxes][16 KiB]
-  uint8_t* sStg = sG + 2 * FB_G_BYTES;             // [2 warpgroups][16 KiB]
+  uint8_t* sStg = sG + 2 * FB_G_BYTES;             // [8 epilogue warps][4 KiB]
   uint64_t* w_full = reinterpret_cast<uint64_t*>(sStg + NUM_EPI_WG * STG_BYTES);
   uint64_t* w_empty = w_full + FB_WSTAGES;
   uint64_t* h_full = w_empty + FB_WSTAGES;  // [2]
@@ -350,9 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int r = q * 32 + lane;  // TMEM lane: a row of the half, or a vocabulary id of a dW tile
     const int epi_tid = threadIdx.x - EPI_WARP0 * 32;
     const int wg = epi_tid / EPI_WG_THREADS;  // row half; 32-column slice of a dW tile
-    const int wtid = epi_tid % EPI_WG_THREADS;
-    const uint32_t wg_bar = 2 + static_cast<uint32_t>(wg);
-    uint8_t* stg = sStg + wg * STG_BYTES;
+    uint8_t* stg = sStg + (epi_tid / 32) * (STG_BYTES / 4);  // this warp's 32 x 128-byte box
     uint8_t* gbox = sG + wg * FB_G_BYTES;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int round = 0;
@@ -362,24 +362,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       named_bar_sync(1, NUM_EPI_THREADS);
       return decision[(round++) & 1] != 0;
     };
-    // one 128-row x 32-column f32 box through this warpgroup's staging
-    // buffer, stored or added (TMA reduction) to global memory.  The
-    // staging buffer is reused once the previous box has been read from it;
-    // with `order`, once everything this warpgroup sent before has been
-    // written.
+    // this warp's 32 rows x 32 f32 columns through its staging box, stored
+    // or added (TMA reduction) to global memory.  The box is reused once the
+    // previous one has been read from it; with `order`, once everything this
+    // warp sent before has been written.
     auto emit_box = [&](const uint32_t (&w)[32], const CUtensorMap* map, int x, int y,
                         bool issue, bool add, bool order) {
-      if (wtid == 0) {
+      if (lane == 0) {
         if (order)
           bulk_wait_group<0>();
         else
           bulk_wait_group_read<0>();
       }
-      named_bar_sync(wg_bar, EPI_WG_THREADS);
-      stage_row128(stg, r, 0, w);
+      __syncwarp();
+      stage_row128(stg, lane, 0, w);
       fence_proxy_async_smem();
-      named_bar_sync(wg_bar, EPI_WG_THREADS);
-      if (wtid == 0) {
+      __syncwarp();
+      if (lane == 0) {
         if (issue) {
           if (add)
             tma_reduce_add_2d(map, smem_addr(stg), x, y);
@@ -389,8 +388,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bulk_commit_group();
       }
     };
-    // dW of tile t (TMEM buffer buf) -> slab sg, stored or added; TMEM is
-    // handed back as soon as it has been read
+    // dW of tile t (TMEM buffer buf) -> slab sg, stored or added: this warp's
+    // 32 vocabulary ids x its warpgroup's 32 columns.  TMEM is handed back as
+    // soon as it has been read.
     auto drain_dw = [&](uint32_t buf, int sg, int t, bool add, bool order) {
       uint32_t w[32];
       tmem_ld32(lane_base + FB_TM_DW + 64 * buf + 32 * wg, w);
@@ -398,7 +398,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dw_empty[buf]);
-      emit_box(w, &g.tmDW, 32 * wg, sg * fa.Vp + t * FB_COLS, 32 * wg < g.D, add, order);
+      emit_box(w, &g.tmDW, 32 * wg, sg * fa.Vp + t * FB_COLS + 32 * q, 32 * wg < g.D, add,
+               order);
     };
 
     uint32_t n_t = 0;
@@ -429,14 +430,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e);
           rrow = __ldg(g.row_scale + row);
         }
+        // The epilogue warps decide together whether to stop once per row
+        // block (at its end): a wait that gives up raises the abort flag and
+        // returns, the later waits return at once, and the warps run on to
+        // the decision with whatever TMEM and shared memory hold.
         for (int t = t0; t < t1; ++t, ++n_t) {
-          // Z_t is in TMEM.  (A wait that gives up raises the abort flag,
-          // which the next decision reads; until then the epilogue runs on.)
+          // Z_t is in TMEM
           mbar_wait(z_full, n_t & 1, abort_flag, g.err);
-          if (decide_abort()) {
-            aborted = true;
-            break;
-          }
           tc_fence_after();
           const int vglob0 = t * FB_COLS;
           const int vlim = g.V - vglob0;
@@ -477,16 +477,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             drain_dw((n_t - 1) & 1, itm.g, t - 1, add, add && t == t0 + 1);
           }
         }
-        if (aborted) break;
         // the last dW tile, then the row block's dH halves -> the slab of chunk ch
         const uint32_t nl = n_t - 1;
-        bool okw = mbar_wait(&dw_full[nl & 1], (nl >> 1) & 1, abort_flag, g.err);
-        okw = okw && mbar_wait(dh_full, n_item & 1, abort_flag, g.err);
-        (void)okw;
-        if (decide_abort()) {
-          aborted = true;
-          break;
-        }
+        mbar_wait(&dw_full[nl & 1], (nl >> 1) & 1, abort_flag, g.err);
+        mbar_wait(dh_full, n_item & 1, abort_flag, g.err);
         tc_fence_after();
         drain_dw(nl & 1, itm.g, t1 - 1, add, add && t1 == t0 + 1);
         uint32_t w0[32], w1[32];
@@ -497,14 +491,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dh_empty);
-        const int ydh = itm.ch * fa.Np + rb * FB_ROWS + wg * BM;
+        const int ydh = itm.ch * fa.Np + rb * FB_ROWS + wg * BM + 32 * q;
         emit_box(w0, &g.tmDH, 0, ydh, true, false, false);
         emit_box(w1, &g.tmDH, 32, ydh, 32 < g.D, false, false);
         ++n_item;
+        if (decide_abort()) {
+          aborted = true;
+          break;
+        }
       }
       if (aborted) break;
     }
-    if (wtid == 0) bulk_wait_group<0>();
+    if (lane == 0) bulk_wait_group<0>();
   }
 
   tc_fence_before();
