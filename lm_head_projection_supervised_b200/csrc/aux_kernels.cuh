@@ -526,91 +526,173 @@ __global__ void __launch_bounds__(RS_TILE)
 // dW[v] += (S / sigma) sum_{k: y_k = v} e_k H_c[k], over the rows grouped by
 // label (keys sorted stably, so each group's rows are in ascending order):
 // the fp32 residuals of the 16-bit target entries (see scatter_dh_kernel),
-// added once per label after every panel's dW is written.  One warp per
-// (group start, 128-column chunk): a lane owns 4 columns; the group's row
-// ids and residuals are read 32 at a time (one step ahead) and broadcast by
-// shuffles, so the H loads of consecutive rows are independent.  Fixed
-// order: deterministic.
-__global__ void dw_target_resid_kernel(const uint32_t* __restrict__ keys,
-                                       const int* __restrict__ rows, int64_t Np, int V_slice,
-                                       const uint2* __restrict__ Hc, int64_t vec_per_row,
-                                       int is_bf16, const float* __restrict__ tgt_resid,
+// added once per label after every panel's dW is written.  A segmented sum
+// in two passes over windows of 32 sorted positions, so that no warp walks a
+// long group (the hottest label of a Zipf batch holds about a tenth of the
+// rows):
+//   pass 1 (dw_target_window_kernel), a warp per (window, 128-column chunk):
+//     the window's runs of equal labels, each summed in row order; a run
+//     that is a whole group is added to dW; otherwise its sum is kept in the
+//     window's slot 0 (the run that begins at the window's start) or slot 1
+//     (the run that begins inside the window and goes on past its end);
+//   pass 2 (dw_target_chain_kernel), a warp per (window, chunk) whose last
+//     run opens a group that goes on: the group's window sums in window
+//     order, added to dW.
+// Fixed order everywhere: deterministic.  A lane owns 4 columns.
+constexpr int TW = 32;  // sorted positions per window
+
+__device__ __forceinline__ void h4_to_f32(uint2 hv, bool bf16, float& h0, float& h1, float& h2,
+                                          float& h3) {
+  if (bf16) {
+    h0 = __uint_as_float(hv.x << 16);
+    h1 = __uint_as_float(hv.x & 0xFFFF0000u);
+    h2 = __uint_as_float(hv.y << 16);
+    h3 = __uint_as_float(hv.y & 0xFFFF0000u);
+  } else {
+    const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+    const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+    h0 = lo.x;
+    h1 = lo.y;
+    h2 = hi.x;
+    h3 = hi.y;
+  }
+}
+
+__global__ void dw_target_window_kernel(const uint32_t* __restrict__ keys,
+                                        const int* __restrict__ rows, int64_t Np, int V_slice,
+                                        const uint2* __restrict__ Hc, int64_t vec_per_row,
+                                        int is_bf16, const float* __restrict__ tgt_resid,
+                                        const float* __restrict__ scal, float inv_sigma,
+                                        float4* __restrict__ win_sums, float4* __restrict__ dW) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nchunk = (vec_per_row + 31) / 32;
+  const int64_t nwin = (Np + TW - 1) / TW;
+  const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
+  const float scale = (*scal) * inv_sigma;
+  for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < nwin * nchunk; w += warps) {
+    const int64_t win = w / nchunk;
+    const int64_t c = (w % nchunk) * 32 + lane;  // this lane's 4-column group
+    const int64_t base = win * TW;
+    const int n = static_cast<int>(Np - base < TW ? Np - base : TW);
+    const uint32_t none = 0xFFFFFFFFu;
+    const uint32_t key = lane < n ? keys[base + lane] : none;
+    const bool counted = key < static_cast<uint32_t>(V_slice);
+    const int k = counted ? rows[base + lane] : 0;
+    const float e = counted ? tgt_resid[k] : 0.f;
+    const uint32_t prev_key = base > 0 ? keys[base - 1] : none;
+    const uint32_t next_key = base + TW < Np ? keys[base + TW] : none;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int run0 = 0;  // first window position of the current run
+    // the current run [run0, j] ends at j: whole group or window slot
+    auto flush = [&](uint32_t kv, bool ends_group) {
+      if (kv < static_cast<uint32_t>(V_slice) && c < vec_per_row) {
+        const bool starts_group = !(run0 == 0 && prev_key == kv);
+        if (starts_group && ends_group) {
+          float4* dst = dW + static_cast<int64_t>(kv) * vec_per_row + c;
+          const float4 o = *dst;
+          *dst = make_float4(fmaf(scale, a0, o.x), fmaf(scale, a1, o.y), fmaf(scale, a2, o.z),
+                             fmaf(scale, a3, o.w));
+        } else {
+          win_sums[(win * 2 + (run0 == 0 ? 0 : 1)) * vec_per_row + c] =
+              make_float4(a0, a1, a2, a3);
+        }
+      }
+      a0 = a1 = a2 = a3 = 0.f;
+    };
+    for (int j0 = 0; j0 < n; j0 += 16) {
+      // sixteen rows' loads in flight, then their terms in row order
+      // (measured: all 32 at once needs more registers and ran slower)
+      uint2 hv[16];
+      float ej[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int kj = __shfl_sync(0xffffffffu, k, j0 + u);
+        ej[u] = __shfl_sync(0xffffffffu, e, j0 + u);
+        hv[u] = (j0 + u < n && c < vec_per_row && ej[u] != 0.f)
+                    ? __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c)
+                    : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int j = j0 + u;
+        const uint32_t kv = __shfl_sync(0xffffffffu, key, j);
+        const uint32_t nk = __shfl_sync(0xffffffffu, key, (j + 1) & 31);
+        if (j >= n) break;
+        float h0, h1, h2, h3;
+        h4_to_f32(hv[u], is_bf16 != 0, h0, h1, h2, h3);
+        a0 = fmaf(ej[u], h0, a0);
+        a1 = fmaf(ej[u], h1, a1);
+        a2 = fmaf(ej[u], h2, a2);
+        a3 = fmaf(ej[u], h3, a3);
+        const uint32_t after = j + 1 < n ? nk : next_key;  // label of the next sorted position
+        if (after != kv) {
+          flush(kv, true);
+          run0 = j + 1;
+        } else if (j + 1 == n) {
+          flush(kv, false);  // the group goes on in the next window
+        }
+      }
+    }
+  }
+}
+
+__global__ void dw_target_chain_kernel(const uint32_t* __restrict__ keys, int64_t Np,
+                                       int V_slice, int64_t vec_per_row,
+                                       const float4* __restrict__ win_sums,
                                        const float* __restrict__ scal, float inv_sigma,
                                        float4* __restrict__ dW) {
   const int lane = threadIdx.x & 31;
   const int64_t nchunk = (vec_per_row + 31) / 32;
+  const int64_t nwin = (Np + TW - 1) / TW;
   const int64_t warps = static_cast<int64_t>(blockDim.x >> 5) * gridDim.x;
   const float scale = (*scal) * inv_sigma;
   for (int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       w < Np * nchunk; w += warps) {
-    const int64_t p = w / nchunk;
-    const int64_t c = (w % nchunk) * 32 + lane;  // this lane's 4-column group
-    const uint32_t v = keys[p];
-    if (v >= static_cast<uint32_t>(V_slice) || (p > 0 && keys[p - 1] == v)) continue;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    // up to 32 rows of the group per step: row id and residual in lane order;
-    // the next step's are fetched while this step's H rows load
-    bool in = p + lane < Np && keys[p + lane] == v;
-    int k = in ? rows[p + lane] : 0;
-    float e = in ? tgt_resid[k] : 0.f;
-    for (int64_t q0 = p;; q0 += 32) {
-      const unsigned live = __ballot_sync(0xffffffffu, in);
-      const int n = __popc(live);  // the group's rows are contiguous from q0
-      bool in_next = false;
-      int k_next = 0;
-      float e_next = 0.f;
-      if (n == 32) {
-        const int64_t qn = q0 + 32 + lane;
-        in_next = qn < Np && keys[qn] == v;
-        k_next = in_next ? rows[qn] : 0;
-        e_next = in_next ? tgt_resid[k_next] : 0.f;
-      }
-      for (int j0 = 0; j0 < n; j0 += 16) {
-        // sixteen rows' loads in flight, then their terms in row order
-        uint2 hv[16];
-        float ej[16];
+       w < nwin * nchunk; w += warps) {
+    const int64_t win = w / nchunk;
+    const int64_t c = (w % nchunk) * 32 + lane;
+    const int64_t base = win * TW;
+    const int n = static_cast<int>(Np - base < TW ? Np - base : TW);
+    const uint32_t v = keys[base + n - 1];  // label of the window's last run
+    if (v >= static_cast<uint32_t>(V_slice)) continue;
+    if (!(base + TW < Np && keys[base + TW] == v)) continue;  // the run ends here: pass 1 had it
+    // where the last run begins: after the last position (below n) with another label
+    const uint32_t key = lane < n ? keys[base + lane] : v;
+    const unsigned other = __ballot_sync(0xffffffffu, key != v);
+    const int run0 = other ? 32 - __clz(other) : 0;
+    if (run0 == 0 && base > 0 && keys[base - 1] == v) continue;  // a window before opens it
+    if (c >= vec_per_row) continue;
+    float4 t = win_sums[(win * 2 + (run0 == 0 ? 0 : 1)) * vec_per_row + c];
+    // the following windows eight at a time (loads in flight together); a
+    // window's sum is added when the group reaches it, in window order
+    bool go = true;
+    for (int64_t w0 = win + 1; go && w0 < nwin; w0 += 8) {
+      float4 u[8];
+      bool cont[8];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int kj = __shfl_sync(0xffffffffu, k, j0 + u);
-          ej[u] = __shfl_sync(0xffffffffu, e, j0 + u);
-          hv[u] = (j0 + u < n && c < vec_per_row)
-                      ? __ldg(Hc + static_cast<int64_t>(kj) * vec_per_row + c)
-                      : make_uint2(0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (j0 + u >= n) break;
-          float h0, h1, h2, h3;
-          if (is_bf16) {
-            h0 = __uint_as_float(hv[u].x << 16);
-            h1 = __uint_as_float(hv[u].x & 0xFFFF0000u);
-            h2 = __uint_as_float(hv[u].y << 16);
-            h3 = __uint_as_float(hv[u].y & 0xFFFF0000u);
-          } else {
-            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].x));
-            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv[u].y));
-            h0 = lo.x;
-            h1 = lo.y;
-            h2 = hi.x;
-            h3 = hi.y;
-          }
-          a0 = fmaf(ej[u], h0, a0);
-          a1 = fmaf(ej[u], h1, a1);
-          a2 = fmaf(ej[u], h2, a2);
-          a3 = fmaf(ej[u], h3, a3);
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int64_t ww = w0 + i;
+        const int64_t nb = (ww + 1) * TW;
+        u[i] = ww < nwin ? win_sums[(ww * 2) * vec_per_row + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        cont[i] = nb < Np && keys[nb] == v;
       }
-      if (n < 32) break;
-      in = in_next;
-      k = k_next;
-      e = e_next;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (!go || w0 + i >= nwin) {
+          go = false;
+          break;
+        }
+        t.x += u[i].x;
+        t.y += u[i].y;
+        t.z += u[i].z;
+        t.w += u[i].w;
+        go = cont[i];
+      }
     }
-    if (c < vec_per_row) {
-      float4* dst = dW + static_cast<int64_t>(v) * vec_per_row + c;
-      const float4 o = *dst;
-      *dst = make_float4(fmaf(scale, a0, o.x), fmaf(scale, a1, o.y), fmaf(scale, a2, o.z),
-                         fmaf(scale, a3, o.w));
-    }
+    float4* dst = dW + static_cast<int64_t>(v) * vec_per_row + c;
+    const float4 o = *dst;
+    *dst = make_float4(fmaf(scale, t.x, o.x), fmaf(scale, t.y, o.y), fmaf(scale, t.z, o.z),
+                       fmaf(scale, t.w, o.w));
   }
 }
 

@@ -62,7 +62,7 @@ constexpr int kPanelBufs = 3;  // panel buffers: written, read, and one of slack
 
 struct Layout {
   size_t ctrl, ctrl_bytes, C, idx, yc, hc, part, tgt, loss_rows, fwd_total;
-  size_t pos, rs, resid, skeys[2], svals[2], rscount, dbacc, keep, keep_bytes, dhc;
+  size_t pos, rs, resid, skeys[2], svals[2], rscount, dbacc, keep, keep_bytes, dhc, twin;
   size_t gpanel[kPanelBufs], dwp, dhp, total;
   int64_t Np, nvt, vc, gld, panels;
   bool fused;   // the single-kernel backward applies (D <= 64)
@@ -107,6 +107,8 @@ Layout make_layout(int64_t N, int64_t D, int64_t V) {
   L.rscount = take(static_cast<size_t>(RS_DIGITS) * cdiv64(L.Np, RS_TILE) * 4);
   L.dbacc = take(static_cast<size_t>(V) * 8);  // bias gradient, fixed point per vocabulary id
   L.dhc = take(static_cast<size_t>(L.Np) * D * 4);
+  // dW target terms: two partial sums per window of TW label-sorted rows
+  L.twin = take(static_cast<size_t>(cdiv64(L.Np, TW)) * 2 * D * 4);
   // What follows is used by one of the two backward forms only: the panel
   // backward's flags and panels, or the single-kernel backward's partials.
   const size_t shared_base = off;
@@ -421,6 +423,7 @@ struct WsPtrs {
   unsigned long long* dbacc;
   uint8_t* keep;
   float* dhc;
+  float* twin;
   uint16_t* gpanel[kPanelBufs];
   float* dwp;  // single-kernel backward: dW partials [FB_NG_MAX][Vp][D]
   float* dhp;  //   and dH partials [FB_NCH_MAX][Np][D]
@@ -450,6 +453,7 @@ WsPtrs carve(void* ws, const Layout& L) {
   p.dbacc = reinterpret_cast<unsigned long long*>(w + L.dbacc);
   p.keep = w + L.keep;
   p.dhc = reinterpret_cast<float*>(w + L.dhc);
+  p.twin = reinterpret_cast<float*>(w + L.twin);
   for (int i = 0; i < kPanelBufs; ++i) p.gpanel[i] = reinterpret_cast<uint16_t*>(w + L.gpanel[i]);
   p.dwp = L.fused ? reinterpret_cast<float*>(w + L.dwp) : nullptr;
   p.dhp = L.fused ? reinterpret_cast<float*>(w + L.dhp) : nullptr;
@@ -807,13 +811,20 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       }));
       cur ^= 1;
     }
-    const int64_t rwarps = L.Np * cdiv64(D / 4, 32);
-    const int64_t rblocks = cdiv64(rwarps, 8) < 16LL * di.sms ? cdiv64(rwarps, 8) : 16LL * di.sms;
+    // one warp per (window of TW sorted rows, 128 columns), both passes
+    const int64_t rwarps = cdiv64(L.Np, TW) * cdiv64(D / 4, 32);
+    const int64_t rblocks = cdiv64(rwarps, 8);
     FLCE_CK(timed_launch(kProfAux, s, [&] {
-      dw_target_resid_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+      dw_target_window_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
           p.skeys[cur], p.svals[cur], L.Np, static_cast<int>(V),
           reinterpret_cast<const uint2*>(p.hc), D / 4, bf16 ? 1 : 0, p.resid, p.scal,
-          1.f / sigma, reinterpret_cast<float4*>(dW));
+          1.f / sigma, reinterpret_cast<float4*>(p.twin), reinterpret_cast<float4*>(dW));
+    }));
+    FLCE_CK(timed_launch(kProfAux, s, [&] {
+      dw_target_chain_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+          p.skeys[cur], L.Np, static_cast<int>(V), D / 4,
+          reinterpret_cast<const float4*>(p.twin), p.scal, 1.f / sigma,
+          reinterpret_cast<float4*>(dW));
     }));
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       scatter_dh_kernel<<<static_cast<unsigned>(cdiv64(N, 8)), 256, 0, s>>>(
