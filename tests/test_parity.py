@@ -102,7 +102,7 @@ CASES = [
     ("small_d64", dict(seed=15, N=700, D=64, V=9000)),
     ("small_d128_fp16", dict(seed=16, N=600, D=128, V=8300, dtype="fp16")),
     # few labels: each label's rows span many windows of the dW target-term sums
-    ("few_labels", dict(seed=17, N=1000, D=200, V=3)),
+    ("few_labels", dict(seed=17, N=1000, D=200, V=12)),
     ("few_labels_d64_fp16", dict(seed=18, N=900, D=64, V=5, dtype="fp16")),
 ]
 
