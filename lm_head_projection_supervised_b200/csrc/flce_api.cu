@@ -218,7 +218,9 @@ GemmKernel gemm_kernel(int feat) {
 }
 template <int MODE, int... F, class Fn>
 void each_kernel(std::integer_sequence<int, F...>, Fn&& fn) {
-  (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>), ModeCfg<MODE>::SMEM_BYTES), ...);
+  (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>), ModeCfg<MODE>::SMEM_BYTES,
+      kRegsAtLaunch),
+   ...);
 }
 // the single-kernel backward: bias and rounding of the logits
 using FusedFeats = std::integer_sequence<int, 0, kFeatBias, kFeatRound, kFeatBias | kFeatRound>;
@@ -231,7 +233,8 @@ FusedKernel pick_fused(int feat, std::integer_sequence<int, F...>) {
 }
 template <int... F, class Fn>
 void each_fused(std::integer_sequence<int, F...>, Fn&& fn) {
-  (fn(reinterpret_cast<const void*>(flce_fused_bwd_kernel<F>), FB_SMEM_BYTES), ...);
+  (fn(reinterpret_cast<const void*>(flce_fused_bwd_kernel<F>), FB_SMEM_BYTES, FB_REGS_AT_LAUNCH),
+   ...);
 }
 
 // ---- per-device set-up
@@ -259,7 +262,7 @@ flce_status device_setup(DevInfo* out) {
     d.ok = (major == 10 && minor == 0) && encode_fn() != nullptr;
     if (d.ok) {
       bool fail = false;
-      auto setup = [&](const void* fn, size_t smem) {
+      auto setup = [&](const void* fn, size_t smem, uint32_t regs_needed) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess) {
           fail = true;
@@ -269,7 +272,7 @@ flce_status device_setup(DevInfo* out) {
         // the split only fits if the block was launched with enough of them.
         cudaFuncAttributes fa{};
         if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) fail = true;
-        else if (fa.numRegs < static_cast<int>(kRegsAtLaunch)) d.ok = false;
+        else if (fa.numRegs < static_cast<int>(regs_needed)) d.ok = false;
       };
       each_kernel<kModeFwd>(FwdFeats{}, setup);
       each_kernel<kModeBwd>(BwdFeats{}, setup);
@@ -685,7 +688,7 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
         FusedFeats{});
     if (kern == nullptr) return FLCE_ERR_ARG;
     FLCE_CK(timed_launch(kProfBwd, s, [&] {
-      kern<<<static_cast<unsigned>(di.sms), NUM_THREADS, FB_SMEM_BYTES, s>>>(fa);
+      kern<<<static_cast<unsigned>(di.sms), FB_THREADS, FB_SMEM_BYTES, s>>>(fa);
     }));
     const int64_t D4 = D / 4;
     const int64_t dw_blocks = cdiv64(V * D4, 256) < 8LL * di.sms ? cdiv64(V * D4, 256) : 8LL * di.sms;

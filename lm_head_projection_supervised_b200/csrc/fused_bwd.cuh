@@ -26,13 +26,16 @@
 // drains one while the next accumulates.  D > 64 does not fit: dH of 256 rows
 // and a dW tile need 2 D + D columns beside the 256 of the scores.
 //
-// Roles (384 threads): warp 0 schedules items and loads H (once per row
-// block) and the W tiles (a ring); warp 1 issues the MMAs; warps 4..11 are two
-// epilogue warpgroups, warpgroup h on row half h (thread = TMEM lane = row),
-// which also drain the dW tiles (lane = vocabulary id, 32 columns each) and
-// the dH halves, each warp its 32 TMEM lanes through its own 4 KiB staging
-// box and TMA, so that the epilogue warps meet only once per row block.
-// Every wait is bounded (see mbar_wait).
+// Roles (640 threads): warp 0 schedules items and loads H (once per row
+// block) and the W tiles (a ring); warp 1 issues the MMAs; warps 4..19 are
+// four epilogue warpgroups, warpgroup (h, s) on row half h and the 64 ids s
+// of the tile (thread = TMEM lane = row): the epilogue is bound by its
+// per-entry arithmetic and latency, and four warps per scheduler hide more
+// of it than two.  They also drain the dW tiles (lane = vocabulary id; the
+// two warpgroups of row half t % 2 take tile t, 32 columns each) and the dH
+// halves, each warp its 32 TMEM lanes through its own 4 KiB staging box and
+// TMA, so that the epilogue warps meet only once per row block.  Every wait
+// is bounded (see mbar_wait).
 #pragma once
 
 #include "gemm.cuh"
@@ -42,7 +45,18 @@ namespace flce {
 constexpr int FB_MAX_D = 64;        // hidden sizes the fused backward takes
 constexpr int FB_ROWS = 256;        // rows per work item
 constexpr int FB_COLS = 128;        // vocabulary ids per tile
-constexpr int FB_WSTAGES = 4;       // W tile ring depth
+constexpr int FB_WSTAGES = 2;       // W tile ring depth (a tile lasts thousands of cycles)
+constexpr int FB_EPI_WG = 4;        // epilogue warpgroups
+constexpr int FB_EPI_THREADS = FB_EPI_WG * EPI_WG_THREADS;
+constexpr int FB_THREADS = EPI_WARP0 * 32 + FB_EPI_THREADS;
+// registers per thread after the split (the first warpgroup only schedules,
+// loads and issues), and at launch
+constexpr uint32_t FB_REGS_LOW = 64;
+constexpr uint32_t FB_REGS_HIGH = 104;
+static_assert(128 * FB_REGS_LOW + FB_EPI_THREADS * FB_REGS_HIGH <= 65536, "register split");
+constexpr uint32_t FB_REGS_AT_LAUNCH =
+    (128 * FB_REGS_LOW + FB_EPI_THREADS * FB_REGS_HIGH + FB_THREADS - 1) / FB_THREADS;
+constexpr uint32_t FB_STG_BYTES = 32 * 128;  // 4 KiB staging box per epilogue warp
 constexpr int FB_NCH_MAX = 160;     // vocabulary chunks (slabs of dH partials) at most
 constexpr int FB_NG_MAX = 8;        // groups of row blocks (slabs of dW partials) at most
 constexpr uint32_t FB_H_BYTES = BM * 64 * 2;        // 16 KiB: one 128-row half of H
@@ -53,7 +67,7 @@ constexpr uint32_t FB_TM_Z = 0;     // TMEM column of Z_0 (Z_1 at +128)
 constexpr uint32_t FB_TM_DH = 256;  // dH_0 (dH_1 at +64)
 constexpr uint32_t FB_TM_DW = 384;  // dW buffer 0 (buffer 1 at +64)
 constexpr size_t FB_SMEM_BYTES = 1024 + 2 * FB_HB_BYTES + FB_WSTAGES * FB_W_BYTES +
-                                 2 * FB_G_BYTES + NUM_EPI_WG * STG_BYTES + 512;
+                                 2 * FB_G_BYTES + (FB_EPI_THREADS / 32) * FB_STG_BYTES + 512;
 static_assert(FB_SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // The split of the work: nch vocabulary chunks (one per CTA or more, at most
@@ -90,7 +104,7 @@ struct FusedArgs {
 };
 
 template <int FEAT>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(FB_THREADS, 1)
     flce_fused_bwd_kernel(const __grid_constant__ FusedArgs fa) {
   const GemmArgs& g = fa.g;
   extern __shared__ uint8_t smem_raw[];
@@ -99,8 +113,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sH = smem;                              // [2 buffers][2 halves][16 KiB]
   uint8_t* sW = sH + 2 * FB_HB_BYTES;              // [FB_WSTAGES][16 KiB]
   uint8_t* sG = sW + FB_WSTAGES * FB_W_BYTES;      // [2 halves][2 boxes][16 KiB]
-  uint8_t* sStg = sG + 2 * FB_G_BYTES;             // [8 epilogue warps][4 KiB]
-  uint64_t* w_full = reinterpret_cast<uint64_t*>(sStg + NUM_EPI_WG * STG_BYTES);
+  uint8_t* sStg = sG + 2 * FB_G_BYTES;             // [16 epilogue warps][4 KiB]
+  uint64_t* w_full =
+      reinterpret_cast<uint64_t*>(sStg + (FB_EPI_THREADS / 32) * FB_STG_BYTES);
   uint64_t* w_empty = w_full + FB_WSTAGES;
   uint64_t* h_full = w_empty + FB_WSTAGES;  // [2]
   uint64_t* h_empty = h_full + 2;           // [2]
@@ -122,7 +137,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr uint32_t kEpiWarps = NUM_EPI_THREADS / 32;
+  constexpr uint32_t kEpiWarps = FB_EPI_THREADS / 32;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < FB_WSTAGES; ++s) {
@@ -139,7 +154,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(g_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dw_full[b], 1);
-      mbar_init(&dw_empty[b], kEpiWarps);
+      mbar_init(&dw_empty[b], kEpiWarps / 2);  // the eight warps that drain the tile
     }
     mbar_init(dh_full, 1);
     mbar_init(dh_empty, kEpiWarps);
@@ -188,7 +203,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (warp < EPI_WARP0) {
-    setmaxnreg_dec<kRegsLow>();
+    setmaxnreg_dec<FB_REGS_LOW>();
     if (warp == 0) {
       // ------------------------------------------------------------ scheduler + loads
       if (lane == 0) {
@@ -346,20 +361,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    setmaxnreg_inc<kRegsHigh>();
+    setmaxnreg_inc<FB_REGS_HIGH>();
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;  // TMEM lane: a row of the half, or a vocabulary id of a dW tile
     const int epi_tid = threadIdx.x - EPI_WARP0 * 32;
-    const int wg = epi_tid / EPI_WG_THREADS;  // row half; 32-column slice of a dW tile
-    uint8_t* stg = sStg + (epi_tid / 32) * (STG_BYTES / 4);  // this warp's 32 x 128-byte box
-    uint8_t* gbox = sG + wg * FB_G_BYTES;
+    const int wg = epi_tid / EPI_WG_THREADS;
+    const int hh = wg >> 1;  // row half: Z_hh, G_hh, dH_hh; drains the dW tiles t with t % 2 == hh
+    const int ss = wg & 1;   // ids [64 ss, 64 ss + 64) of a tile (G box ss); columns
+                             // [32 ss, 32 ss + 32) of the dW tiles and of dH_hh
+    uint8_t* stg = sStg + (epi_tid / 32) * FB_STG_BYTES;  // this warp's 32 x 128-byte box
+    uint8_t* gbox = sG + hh * FB_G_BYTES + ss * STG_BYTES;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int round = 0;
     auto decide_abort = [&]() -> bool {
-      named_bar_sync(1, NUM_EPI_THREADS);
+      named_bar_sync(1, FB_EPI_THREADS);
       if (epi_tid == 0) decision[round & 1] = *abort_flag;
-      named_bar_sync(1, NUM_EPI_THREADS);
+      named_bar_sync(1, FB_EPI_THREADS);
       return decision[(round++) & 1] != 0;
     };
     // this warp's 32 rows x 32 f32 columns through its staging box, stored
@@ -389,17 +407,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     };
     // dW of tile t (TMEM buffer buf) -> slab sg, stored or added: this warp's
-    // 32 vocabulary ids x its warpgroup's 32 columns.  TMEM is handed back as
-    // soon as it has been read.
-    auto drain_dw = [&](uint32_t buf, int sg, int t, bool add, bool order) {
+    // 32 vocabulary ids x its 32 columns.  TMEM is handed back as soon as it
+    // has been read.  A warp drains the same ids and columns of a tile in
+    // every pass, so waiting for its own earlier additions orders them.
+    bool first_drain = false;
+    auto drain_dw = [&](uint32_t buf, int sg, int t, bool add) {
       uint32_t w[32];
-      tmem_ld32(lane_base + FB_TM_DW + 64 * buf + 32 * wg, w);
+      tmem_ld32(lane_base + FB_TM_DW + 64 * buf + 32 * ss, w);
       tmem_wait_ld(w);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dw_empty[buf]);
-      emit_box(w, &g.tmDW, 32 * wg, sg * fa.Vp + t * FB_COLS + 32 * q, 32 * wg < g.D, add,
-               order);
+      emit_box(w, &g.tmDW, 32 * ss, sg * fa.Vp + t * FB_COLS + 32 * q, 32 * ss < g.D, add,
+               add && first_drain);
+      first_drain = false;
     };
 
     uint32_t n_t = 0;
@@ -415,11 +436,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int t0 = itm.t0, t1 = itm.t1;
       bool aborted = false;
       for (int rb = itm.rb0; !aborted && rb < itm.rb1; ++rb) {
-        // dW: the group's later row blocks add to the slab, each pass's first
-        // addition after the previous pass's have all been written, so that
-        // every element receives its terms in row-block order
+        // dW: the group's later row blocks add to the slab, each warp's first
+        // addition of a pass after its additions of the previous pass have
+        // all been written, so that every element receives its terms in
+        // row-block order
         const bool add = rb > itm.rb0;
-        const int row = rb * FB_ROWS + wg * BM + r;
+        first_drain = true;
+        const int row = rb * FB_ROWS + hh * BM + r;
         const bool valid = row < C;
         int yabs = 0;
         float krow = 0.f, rrow = 0.f;
@@ -441,26 +464,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int vglob0 = t * FB_COLS;
           const int vlim = g.V - vglob0;
           const int yl = valid ? yabs - vglob0 : -1000000;
-          const uint32_t t_z = lane_base + FB_TM_Z + 128 * wg;
-          uint32_t za[32], zb[32], pk[16];
+          const uint32_t t_z = lane_base + FB_TM_Z + 128 * hh + 64 * ss;
+          uint32_t za[32], pk[16];
           bool big = false;
-          tmem_ld32(t_z, za);
-          tmem_wait_ld(za);
 #pragma unroll 1
-          for (int c = 0; c < 4; c += 2) {
-            uint8_t* box = gbox + (c >> 1) * STG_BYTES;
-            tmem_ld32(t_z + (c + 1) * 32, zb);
-            grad_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
-                             big);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(t_z + c * 32, za);
+            tmem_wait_ld(za);
+            grad_chunk<FEAT>(g, za, 64 * ss + c * 32, vglob0, vlim, yl, valid, krow, rrow, row,
+                             lane, pk, big);
             // G of tile t - 1 has been read by its contractions
             if (c == 0) mbar_wait(g_empty, (n_t & 1) ^ 1, abort_flag, g.err);
-            stage_row128(box, r, 0, pk);
-            tmem_wait_ld(zb);
-            if (c + 2 < 4) tmem_ld32(t_z + (c + 2) * 32, za);
-            grad_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane,
-                             pk, big);
-            stage_row128(box, r, 4, pk);
-            if (c + 2 < 4) tmem_wait_ld(za);
+            stage_row128(gbox, r, 4 * c, pk);
           }
           // Z read (TMEM free for the next tile's scores) and G written
           // (visible to the tensor core's reads)
@@ -471,29 +486,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_arrive(z_empty);
             mbar_arrive(g_full);
           }
-          if (t > t0) {
-            mbar_wait(&dw_full[(n_t - 1) & 1], ((n_t - 1) >> 1) & 1, abort_flag, g.err);
+          if (t > t0 && ((t - 1) & 1) == hh) {
+            const uint32_t np = n_t - 1;
+            mbar_wait(&dw_full[np & 1], (np >> 1) & 1, abort_flag, g.err);
             tc_fence_after();
-            drain_dw((n_t - 1) & 1, itm.g, t - 1, add, add && t == t0 + 1);
+            drain_dw(np & 1, itm.g, t - 1, add);
           }
         }
         // the last dW tile, then the row block's dH halves -> the slab of chunk ch
         const uint32_t nl = n_t - 1;
-        mbar_wait(&dw_full[nl & 1], (nl >> 1) & 1, abort_flag, g.err);
+        if (((t1 - 1) & 1) == hh) {
+          mbar_wait(&dw_full[nl & 1], (nl >> 1) & 1, abort_flag, g.err);
+          tc_fence_after();
+          drain_dw(nl & 1, itm.g, t1 - 1, add);
+        }
         mbar_wait(dh_full, n_item & 1, abort_flag, g.err);
         tc_fence_after();
-        drain_dw(nl & 1, itm.g, t1 - 1, add, add && t1 == t0 + 1);
-        uint32_t w0[32], w1[32];
-        tmem_ld32(lane_base + FB_TM_DH + 64 * wg, w0);
-        tmem_ld32(lane_base + FB_TM_DH + 64 * wg + 32, w1);
+        uint32_t w0[32];
+        tmem_ld32(lane_base + FB_TM_DH + 64 * hh + 32 * ss, w0);
         tmem_wait_ld(w0);
-        tmem_wait_ld(w1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dh_empty);
-        const int ydh = itm.ch * fa.Np + rb * FB_ROWS + wg * BM + 32 * q;
-        emit_box(w0, &g.tmDH, 0, ydh, true, false, false);
-        emit_box(w1, &g.tmDH, 32, ydh, 32 < g.D, false, false);
+        const int ydh = itm.ch * fa.Np + rb * FB_ROWS + hh * BM + 32 * q;
+        emit_box(w0, &g.tmDH, 32 * ss, ydh, 32 * ss < g.D, false, false);
         ++n_item;
         if (decide_abort()) {
           aborted = true;
