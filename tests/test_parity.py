@@ -104,6 +104,11 @@ CASES = [
     # few labels: each label's rows span many windows of the dW target-term sums
     ("few_labels", dict(seed=17, N=1000, D=200, V=12)),
     ("few_labels_d64_fp16", dict(seed=18, N=900, D=64, V=5, dtype="fp16")),
+    # size extremes: a vocabulary of a million ids (thousands of tiles; 74 chained panel
+    # launches at D = 136) and the largest specified hidden size on a ragged small case
+    ("wide_vocab_d64", dict(seed=19, N=300, D=64, V=1000003)),
+    ("wide_vocab_panels", dict(seed=20, N=260, D=136, V=600011, dtype="fp16")),
+    ("deep_d4096_fp16", dict(seed=21, N=300, D=4096, V=5000, dtype="fp16")),
 ]
 
 
