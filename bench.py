@@ -501,6 +501,14 @@ def main():
     value = weak_scaling_tflops(flop_step, args.steps, total_ms, world)
     peak_mib = torch.cuda.max_memory_allocated(dev) / 2**20
     launches = sum(n for _, n in prof.values())
+    # The library allocates no device memory: every buffer of the step is one
+    # of these.  None may be the size of the N x V logits in 16 bits (checked
+    # where that size is what the method avoids: 1 GiB and up).
+    bufs = [t for t in (H, W, b, y, mk, dH, dW, db) if t is not None] + [ws.buf]
+    largest = max(t.numel() * t.element_size() for t in bufs)
+    logits_bytes = inp.N * inp.V * 2
+    if logits_bytes >= 2**30 and largest >= logits_bytes:
+        raise RuntimeError(f"a {largest} B buffer is as large as the {logits_bytes} B logits")
 
     # e2e: every step's inputs copied from pinned host memory and its loss read
     # back, all inside the timed region.  The inputs of step k+1 are copied on
@@ -636,7 +644,7 @@ def main():
                 "bf16_tflops_sustained"),
             "peak_note": f"bf16 peak {burst} TFLOP/s burst, {peak_src}",
             "peak_mib": peak_mib, "input_mib": in_mib,
-            "logits_mib_avoided": inp.N * inp.V * 2 / 2**20,
+            "logits_mib_avoided": inp.N * inp.V * 2 / 2**20, "largest_alloc_mib": largest / 2**20,
             "clocks": clocks, "e2e": e2e, "gpu_launches": launches,
             "roofline": roofline, "cpu_baseline": cpu_baseline}
     if rank == 0:
