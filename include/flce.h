@@ -84,7 +84,8 @@ typedef void* flce_stream;
 /* Bytes of device workspace needed for problem size (N, D, V).  Returns 0
  * when the sizes are out of range (same limits as FLCE_ERR_SHAPE).  For
  * D <= 64 it includes the single-kernel backward's partial sums (see
- * flce_backward), about ceil(N / 256) * V * D * 4 bytes. */
+ * flce_backward): (8 * V + 160 * N) * D * 4 bytes, rounded up, in the space
+ * the panel form's buffers take otherwise. */
 FLCE_API size_t flce_workspace_bytes(int64_t N, int64_t D, int64_t V, int dtype);
 
 /*
@@ -134,8 +135,9 @@ FLCE_API flce_status flce_forward(const void* H, const void* W, const void* b,
  * 8192 ids at a time, and read by the dW and dH contractions.  D <= 64: one
  * kernel per call does the score tile, the gradient and both contractions
  * per 256-row x 128-id tile (§04's single fused pass: dH of the row block
- * accumulates across the vocabulary on chip, dW is summed from one partial
- * per 256-row block in a fixed order by a second kernel).
+ * accumulates across the vocabulary on chip; dW is added up per group of
+ * row blocks in row-block order, and the groups' sums by a second kernel in
+ * a fixed order).
  */
 FLCE_API flce_status flce_backward(const void* H, const void* W, const void* b,
                           const int64_t* labels, const uint8_t* mask, int64_t ignore_index,
