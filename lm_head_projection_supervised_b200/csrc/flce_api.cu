@@ -194,32 +194,45 @@ bool make_map(CUtensorMap* m, const void* base, MapType t, uint64_t inner, uint6
 // optional features that mode can use (bias, rounding of the logits, and the
 // forward's polynomial exponentials or the backward's gradient filtering)
 using GemmKernel = void (*)(GemmArgs);
-using FwdFeats = std::integer_sequence<int, 0, kFeatBias, kFeatPolyExp, kFeatBias | kFeatPolyExp,
+// (at D <= kPolyExpMaxD the forward takes the polynomial exponentials and four
+// epilogue warpgroups together)
+constexpr int kFeatSmallD = kFeatPolyExp | kFeatWide;
+using FwdFeats = std::integer_sequence<int, 0, kFeatBias, kFeatSmallD, kFeatBias | kFeatSmallD,
                                        kFeatRound, kFeatRound | kFeatBias,
-                                       kFeatRound | kFeatPolyExp,
-                                       kFeatRound | kFeatBias | kFeatPolyExp>;
+                                       kFeatRound | kFeatSmallD,
+                                       kFeatRound | kFeatBias | kFeatSmallD>;
 using BwdFeats = std::integer_sequence<int, 0, kFeatBias, kFeatFilter, kFeatBias | kFeatFilter,
                                        kFeatRound, kFeatRound | kFeatBias,
                                        kFeatRound | kFeatFilter,
                                        kFeatRound | kFeatBias | kFeatFilter>;
 using PlainFeats = std::integer_sequence<int, 0>;
 
+// an instantiation with its launch shape
+struct GemmKernelInfo {
+  GemmKernel fn;
+  int threads;
+  size_t smem;
+};
 template <int MODE, int... F>
-GemmKernel pick_kernel(int feat, std::integer_sequence<int, F...>) {
-  GemmKernel k = nullptr;
-  ((feat == F ? (k = flce_gemm_kernel<MODE, F>, 0) : 0), ...);
+GemmKernelInfo pick_kernel(int feat, std::integer_sequence<int, F...>) {
+  GemmKernelInfo k{nullptr, 0, 0};
+  ((feat == F ? (k = GemmKernelInfo{flce_gemm_kernel<MODE, F>, Shape<MODE, F>::THREADS,
+                                    Shape<MODE, F>::Cfg::SMEM_BYTES},
+                 0)
+              : 0),
+   ...);
   return k;
 }
 template <int MODE>
-GemmKernel gemm_kernel(int feat) {
+GemmKernelInfo gemm_kernel(int feat) {
   if constexpr (MODE == kModeFwd) return pick_kernel<MODE>(feat, FwdFeats{});
   else if constexpr (MODE == kModeBwd) return pick_kernel<MODE>(feat, BwdFeats{});
   else return pick_kernel<MODE>(feat, PlainFeats{});
 }
 template <int MODE, int... F, class Fn>
 void each_kernel(std::integer_sequence<int, F...>, Fn&& fn) {
-  (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>), ModeCfg<MODE>::SMEM_BYTES,
-      kRegsAtLaunch),
+  (fn(reinterpret_cast<const void*>(flce_gemm_kernel<MODE, F>),
+      Shape<MODE, F>::Cfg::SMEM_BYTES, Shape<MODE, F>::REGS_AT_LAUNCH),
    ...);
 }
 // the single-kernel backward: bias and rounding of the logits
@@ -377,8 +390,8 @@ void prof_span_end(ProfRec* r, int launches, cudaStream_t s) {
 template <int MODE>
 cudaError_t launch_gemm(const GemmArgs& a, int feat, int64_t units_upper, int pairs,
                         cudaStream_t s, bool pdl = false, bool timed = true) {
-  const GemmKernel kernel = gemm_kernel<MODE>(feat);
-  if (kernel == nullptr) return cudaErrorInvalidValue;
+  const GemmKernelInfo kernel = gemm_kernel<MODE>(feat);
+  if (kernel.fn == nullptr) return cudaErrorInvalidValue;
   if (units_upper <= 0) return cudaSuccess;
   const int npairs = static_cast<int>(units_upper < pairs ? units_upper : pairs);
   const int kind = MODE == kModeFwd ? kProfFwd : MODE == kModeBwd ? kProfBwd : kProfPlain;
@@ -392,12 +405,12 @@ cudaError_t launch_gemm(const GemmArgs& a, int feat, int64_t units_upper, int pa
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * npairs));
-    cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = ModeCfg<MODE>::SMEM_BYTES;
+    cfg.blockDim = dim3(static_cast<unsigned>(kernel.threads));
+    cfg.dynamicSmemBytes = kernel.smem;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    cudaLaunchKernelEx(&cfg, kernel, a);
+    cudaLaunchKernelEx(&cfg, kernel.fn, a);
   };
   if (!timed) {
     launch();
@@ -554,7 +567,7 @@ flce_status forward_impl(const void* H, const void* W, const void* b, const int6
   a.err = p.err;
   const int feat = (b != nullptr ? kFeatBias : 0) |
                    ((flags & FLCE_FLAG_ROUND_LOGITS) ? kFeatRound : 0) |
-                   (D <= kPolyExpMaxD ? kFeatPolyExp : 0);
+                   (D <= kPolyExpMaxD ? kFeatSmallD : 0);
   FLCE_CK(launch_gemm<kModeFwd>(a, feat, cdiv64(N, PAIR_M) * L.nvt, di.pairs, s));
 
   // 32 rows per block pass, at most 8 blocks per SM

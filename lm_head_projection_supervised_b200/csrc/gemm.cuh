@@ -12,9 +12,9 @@
 // accumulators (512 columns).  In each CTA, warp 0 streams that CTA's halves
 // of the operands (in the backward warp 0 the A boxes and warp 2 the B
 // boxes), and two epilogue warpgroups (warps 4..7 and 8..11, each on half of
-// the columns) read a finished accumulator with tcgen05.ld (thread = TMEM
-// lane = tile row) and run the epilogue while the next unit accumulates in
-// the other.
+// the columns; four in the small-D forward) read a finished accumulator with
+// tcgen05.ld (thread = TMEM lane = tile row) and run the epilogue while the
+// next unit accumulates in the other.
 //
 // Modes (one launch = one mode; each mode is instantiated once per
 // combination of its optional features FEAT, see Feature):
@@ -73,13 +73,14 @@ constexpr uint32_t STG_BYTES = BM * 128;         // 16 KiB: 128 rows x 128 bytes
 // Warps 0-3 form the first warpgroup: scheduler + producer (warp 0), MMA
 // issuer (warp 1), two idle warps.  Warps 4-11 are the epilogue: two
 // warpgroups, each draining half of the accumulator's columns (warp w reads
-// TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, the rows of its quadrant).
+// TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, the rows of its quadrant).  The
+// small-D forward has four epilogue warpgroups, warps 4-19, a quarter of the
+// columns each (see Shape).
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WG = 2;
 constexpr int EPI_WG_THREADS = 128;
 constexpr int NUM_EPI_THREADS = NUM_EPI_WG * EPI_WG_THREADS;
-constexpr int EPI_CHUNKS = BN / 32 / NUM_EPI_WG;  // 32-column chunks per epilogue warpgroup
 // Registers per thread after the split: the first warpgroup gives up what the
 // epilogue takes.  The block is launched with at least kRegsAtLaunch per
 // thread (checked on the host before any launch), which covers the split.
@@ -96,14 +97,15 @@ enum GemmMode : int { kModeFwd = 0, kModeBwd = 1, kModePlain = 2 };
 
 // Ring depth per mode: the backward epilogue stages TMA stores through one
 // 16 KiB box per epilogue warpgroup, the other modes use that shared memory
-// for a 7th stage.
-template <int MODE>
+// for a 7th stage (6 with four epilogue warpgroups, whose (m, s) merge takes
+// more room).
+template <int MODE, bool WIDE = false>
 struct ModeCfg {
-  static constexpr int STAGES = (MODE == kModeBwd) ? 6 : 7;
+  static constexpr int STAGES = (MODE == kModeBwd || WIDE) ? 6 : 7;
   static constexpr uint32_t STAGING = (MODE == kModeBwd) ? NUM_EPI_WG * STG_BYTES : 0;
-  // forward: one (m, s) pair per row of the CTA's half tile, to merge the two
-  // epilogue warpgroups' column halves
-  static constexpr uint32_t MERGE = (MODE == kModeFwd) ? BM * 8 : 0;
+  // forward: one (m, s) pair per row of the CTA's half tile from each
+  // epilogue warpgroup but the first, to merge their column slices
+  static constexpr uint32_t MERGE = (MODE == kModeFwd) ? (WIDE ? 3 : 1) * BM * 8 : 0;
   static constexpr size_t SMEM_BYTES =
       1024 + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + STAGING + 512 + MERGE;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -116,7 +118,31 @@ enum UnitClass : int { kClsDW = 0, kClsDH = 1, kClsGrad = 2 };
 // (its add to the logits, and in the backward its column sums) and the
 // rounding of the logits to the input type.  Backward: gradient filtering.
 // Forward: one exponential in four on the FMA pipe.
-enum Feature : int { kFeatBias = 1, kFeatFilter = 2, kFeatPolyExp = 4, kFeatRound = 8 };
+enum Feature : int {
+  kFeatBias = 1,
+  kFeatFilter = 2,
+  kFeatPolyExp = 4,
+  kFeatRound = 8,
+  kFeatWide = 16  // forward: four epilogue warpgroups (small D, where the epilogue is the bound)
+};
+
+// Thread layout of an instantiation: the first warpgroup (scheduler,
+// producers, MMA issuer) and two epilogue warpgroups, or four for kFeatWide
+// (640 threads; registers 64 / 104 after the split, 96 at launch).
+template <int MODE, int FEAT>
+struct Shape {
+  static constexpr bool WIDE = MODE == kModeFwd && (FEAT & kFeatWide) != 0;
+  static constexpr int EPI_WG = WIDE ? 4 : NUM_EPI_WG;
+  static constexpr int EPI_THREADS = EPI_WG * EPI_WG_THREADS;
+  static constexpr int THREADS = EPI_WARP0 * 32 + EPI_THREADS;
+  static constexpr int CHUNKS = BN / 32 / EPI_WG;  // 32-column chunks per epilogue warpgroup
+  static constexpr uint32_t REGS_LOW = WIDE ? 64 : kRegsLow;
+  static constexpr uint32_t REGS_HIGH = WIDE ? 104 : kRegsHigh;
+  static constexpr uint32_t REGS_AT_LAUNCH =
+      (128 * REGS_LOW + EPI_THREADS * REGS_HIGH + THREADS - 1) / THREADS;
+  static_assert(128 * REGS_LOW + EPI_THREADS * REGS_HIGH <= 65536, "register split");
+  using Cfg = ModeCfg<MODE, WIDE>;
+};
 
 struct GemmArgs {
   CUtensorMap tmA[3];  // A operand map per unit class (fwd / plain use [0])
@@ -605,16 +631,21 @@ __device__ __forceinline__ void stage_row128(uint8_t* stg, int r, int chunk0,
 // The kernel (launched as clusters of 2 CTAs)
 // ---------------------------------------------------------------------------
 template <int MODE, int FEAT = 0>
-__global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_constant__ GemmArgs g) {
-  constexpr int STAGES = ModeCfg<MODE>::STAGES;
+__global__ void __launch_bounds__((Shape<MODE, FEAT>::THREADS), 1)
+    flce_gemm_kernel(const __grid_constant__ GemmArgs g) {
+  using SH = Shape<MODE, FEAT>;
+  using CFG = typename SH::Cfg;
+  constexpr int STAGES = CFG::STAGES;
+  constexpr int EPI_THREADS = SH::EPI_THREADS;
+  constexpr int CHUNKS = SH::CHUNKS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_STAGE_BYTES;
   uint8_t* sStg = sB + STAGES * B_STAGE_BYTES;
-  float2* sMerge = reinterpret_cast<float2*>(sStg + ModeCfg<MODE>::STAGING);  // forward only
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + ModeCfg<MODE>::STAGING + ModeCfg<MODE>::MERGE);
+  float2* sMerge = reinterpret_cast<float2*>(sStg + CFG::STAGING);  // forward only
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + CFG::STAGING + CFG::MERGE);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -625,7 +656,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* decision = abort_flag + 1;  // [2]
   volatile int* s_unit = decision + 2;      // [UQ]
-  volatile int* s_keep = s_unit + UQ;       // [NUM_EPI_THREADS / 32]: filtering votes per warp
+  volatile int* s_keep = s_unit + UQ;       // [EPI_THREADS / 32]: filtering votes per warp
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -650,13 +681,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);                           // one multicast MMA commit
-      mbar_init(&tempty[a], 2 * NUM_EPI_THREADS / 32);   // one lane per epilogue warp, both CTAs
+      mbar_init(&tempty[a], 2 * EPI_THREADS / 32);   // one lane per epilogue warp, both CTAs
     }
     for (int q = 0; q < UQ; ++q) {
       mbar_init(&uq_full[q], 1);
       // even CTA: its MMA lane and epilogue warps; odd CTA: its producer and epilogue warps
       // + the second producer of each CTA when the loads are split
-      mbar_init(&uq_empty[q], 2 * (1 + NUM_EPI_THREADS / 32) + (LoadSplit<MODE>::kSplit ? 2 : 0));
+      mbar_init(&uq_empty[q], 2 * (1 + EPI_THREADS / 32) + (LoadSplit<MODE>::kSplit ? 2 : 0));
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -690,7 +721,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
   const UnitSpace us = make_unit_space<MODE>(g, C);
 
   if (warp < EPI_WARP0) {
-    setmaxnreg_dec<kRegsLow>();  // the whole first warpgroup
+    setmaxnreg_dec<SH::REGS_LOW>();  // the whole first warpgroup
     if (warp == 0 || (LoadSplit<MODE>::kSplit && warp == 2)) {
       // ------------------------------------------------------------ scheduler + producers
       // warp 0: the scheduler (even CTA) and the A loads (all loads when not split);
@@ -833,15 +864,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       }
     }
   } else {
-    setmaxnreg_inc<kRegsHigh>();  // each epilogue warpgroup
+    setmaxnreg_inc<SH::REGS_HIGH>();  // each epilogue warpgroup
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;              // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;         // row within this CTA's half of the tile
     const int rbase = static_cast<int>(rank) * BM;
     const int epi_tid = threadIdx.x - EPI_WARP0 * 32;
-    const int wg = epi_tid / EPI_WG_THREADS;   // epilogue warpgroup: columns [128 wg, 128 wg + 128)
+    const int wg = epi_tid / EPI_WG_THREADS;   // epilogue warpgroup: its CHUNKS 32-column chunks
     const int wtid = epi_tid % EPI_WG_THREADS;
-    const int c0 = wg * EPI_CHUNKS;            // first 32-column chunk of this warpgroup
+    const int c0 = wg * CHUNKS;                // first 32-column chunk of this warpgroup
     const uint32_t wg_bar = 2 + static_cast<uint32_t>(wg);  // named barrier of this warpgroup
     uint8_t* stg = sStg + wg * STG_BYTES;      // this warpgroup's staging box (backward)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -849,13 +880,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
     uint32_t acc_phase = 0;
     float wh_scale = 0.f;
     if (MODE == kModeBwd) wh_scale = (C > 0) ? *g.scal * g.inv_sigma : 0.f;
-    // Shared decision of the eight epilogue warps (they pass named barriers
+    // Shared decision of the epilogue warps (they pass named barriers
     // together, so they leave the loop together).
     int round = 0;
     auto decide_abort = [&]() -> bool {
-      named_bar_sync(1, NUM_EPI_THREADS);
+      named_bar_sync(1, EPI_THREADS);
       if (epi_tid == 0) decision[round & 1] = *abort_flag;
-      named_bar_sync(1, NUM_EPI_THREADS);
+      named_bar_sync(1, EPI_THREADS);
       return decision[(round++) & 1] != 0;
     };
     // Stages one 128 x 128-byte box in this warpgroup's staging buffer and
@@ -916,41 +947,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
       const uint32_t t_acc = lane_base + static_cast<uint32_t>(acc * BN);
 
       if (MODE == kModeFwd) {
-        // (m, s) of this warpgroup's 128 columns.  Chunks stream out of TMEM
+        // (m, s) of this warpgroup's columns.  Chunks stream out of TMEM
         // two at a time (one loading while the other is reduced); the
         // accumulator goes back to the MMA issuer after the last chunk's
         // arithmetic.  (Measured slower: reading all four chunks first, 8 %
         // on the forward at D = 64 and 128; releasing the accumulator right
         // after its last read, 2 % here and 2 % on the backward.)
         FwdRowState st{-INFINITY, 0.f, 0.f, false};
-        uint32_t za[32], zb[32];
-        tmem_ld32(t_acc + c0 * 32, za);
-        tmem_wait_ld(za);
+        uint32_t za[32];
+        if constexpr (SH::WIDE) {
+          // four warpgroups: one chunk in flight per thread (the other warps
+          // hide the load), which keeps the epilogue within its registers
 #pragma unroll 1
-        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
-          tmem_ld32(t_acc + (c + 1) * 32, zb);
-          fwd_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, st);
-          tmem_wait_ld(zb);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
-          fwd_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
+          for (int c = c0; c < c0 + CHUNKS; ++c) {
+            tmem_ld32(t_acc + c * 32, za);
+            tmem_wait_ld(za);
+            fwd_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, st);
+          }
+        } else {
+          uint32_t zb[32];
+          tmem_ld32(t_acc + c0 * 32, za);
+          tmem_wait_ld(za);
+#pragma unroll 1
+          for (int c = c0; c < c0 + CHUNKS; c += 2) {
+            tmem_ld32(t_acc + (c + 1) * 32, zb);
+            fwd_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, st);
+            tmem_wait_ld(zb);
+            if (c + 2 < c0 + CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
+            fwd_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, st);
+            if (c + 2 < c0 + CHUNKS) tmem_wait_ld(za);
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) arrive_on_leader(&tempty[acc]);
         if (valid && st.have_tgt) g.tgt[row] = st.tgt;
-        // the second warpgroup's half of the row joins the first's: one
-        // partial per row and tile, stored tile-major (coalesced per warp).
-        // The buffer is reused only after the next unit's decide_abort, which
-        // both warpgroups pass together.
-        if (wg == 1) sMerge[r] = make_float2(st.m, st.s);
-        named_bar_sync(4, NUM_EPI_THREADS);
+        // the other warpgroups' slices of the row join the first's, in
+        // warpgroup order: one partial per row and tile, stored tile-major
+        // (coalesced per warp).  The buffer is reused only after the next
+        // unit's decide_abort, which all warpgroups pass together.
+        if (wg > 0) sMerge[(wg - 1) * BM + r] = make_float2(st.m, st.s);
+        named_bar_sync(8, EPI_THREADS);
         if (wg == 0) {
-          const float2 o = sMerge[r];
-          const float mn = fmaxf(st.m, o.x);
-          if (mn != -INFINITY) {
-            st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + o.y * ex2_approx((o.x - mn) * kLog2e);
-            st.m = mn;
+#pragma unroll
+          for (int k = 0; k < SH::EPI_WG - 1; ++k) {
+            const float2 o = sMerge[k * BM + r];
+            const float mn = fmaxf(st.m, o.x);
+            if (mn != -INFINITY) {
+              st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + o.y * ex2_approx((o.x - mn) * kLog2e);
+              st.m = mn;
+            }
           }
           if (valid)
             g.part[static_cast<size_t>(un.n0 / BN) * g.part_ld + row] = make_float2(st.m, st.s);
@@ -962,7 +1008,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         tmem_ld32(t_acc + c0 * 32, za);
         tmem_wait_ld(za);
 #pragma unroll 1
-        for (int c = c0; c < c0 + EPI_CHUNKS; c += 2) {
+        for (int c = c0; c < c0 + CHUNKS; c += 2) {
           // chunks c, c+1 form one 64-column box of the 16-bit panel
           if (wtid == 0) bulk_wait_group_read<0>();  // the previous box has left the buffer
           named_bar_sync(wg_bar, EPI_WG_THREADS);
@@ -972,11 +1018,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
           grad_chunk<FEAT>(g, za, c * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk, big);
           stage_row128(stg, r, 0, pk);
           tmem_wait_ld(zb);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
+          if (c + 2 < c0 + CHUNKS) tmem_ld32(t_acc + (c + 2) * 32, za);
           grad_chunk<FEAT>(g, zb, (c + 1) * 32, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk,
                      big);
           stage_row128(stg, r, 4, pk);
-          if (c + 2 < c0 + EPI_CHUNKS) tmem_wait_ld(za);
+          if (c + 2 < c0 + CHUNKS) tmem_wait_ld(za);
           fence_proxy_async_smem();
           if (FEAT & kFeatFilter) {
             const bool any = __any_sync(0xffffffffu, big);
@@ -1030,7 +1076,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         // adding a zero tile to dH changes nothing
         const bool issue = (!is_dw || tm0 < g.w_wh) && !(zero && reduce);
         // this warpgroup's chunks [c0, ce) of the ones inside D
-        const int ce = min(c0 + EPI_CHUNKS, cdiv_i(g.D - un.n0, 32));
+        const int ce = min(c0 + CHUNKS, cdiv_i(g.D - un.n0, 32));
         const int nch = ce;
         uint32_t za[32], zb[32], w[32];
         if (!zero && c0 < ce) {
@@ -1060,7 +1106,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) flce_gemm_kernel(const __grid_
         if (lane == 0) arrive_on_leader(&tempty[acc]);
       } else {  // kModePlain
 #pragma unroll 1
-        for (int c = c0; c < c0 + EPI_CHUNKS; ++c) {
+        for (int c = c0; c < c0 + CHUNKS; ++c) {
           const int col0 = un.n0 + c * 32;
           if (col0 >= g.ncols) break;
           uint32_t z[32];
