@@ -12,22 +12,20 @@ import torch.multiprocessing as mp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _free_port():
-    """A TCP port on 127.0.0.1 that the OS reports free (for the rendezvous)."""
-    import socket
-    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
-        sk.bind(("127.0.0.1", 0))
-        return sk.getsockname()[1]
+def _store_path():
+    """A fresh file for the ranks' rendezvous (a file store: no TCP port that
+    another process could take between choosing it and binding it)."""
+    import tempfile
+    return os.path.join(tempfile.mkdtemp(prefix="flce_pg_"), "store")
 
 
-def _worker(rank, world, port, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _worker(rank, world, store, q):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     import bench
-    dist.init_process_group("gloo", rank=rank, world_size=world,
-                            timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("gloo", init_method="file://" + store, rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         dist.barrier()
         t = bench.max_over_ranks(10.0 + 5.0 * rank)
@@ -40,14 +38,16 @@ def _worker(rank, world, port, q):
 def test_max_over_ranks_two_gloo_ranks():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    store = _store_path()
+    procs = [ctx.Process(target=_worker, args=(r, 2, store, q)) for r in range(2)]
     for p in procs:
         p.start()
+    # results first (a child that has put to the queue exits once it is read),
+    # with room for slow process start-up on a loaded host
+    res = sorted(q.get(timeout=300) for _ in range(2))
     for p in procs:
-        p.join(120)
+        p.join(300)
         assert p.exitcode == 0
-    res = sorted(q.get(timeout=10) for _ in range(2))
     assert [r[1] for r in res] == [15.0, 15.0]
     # 2 ranks x 4 steps x 1 TFLOP in 15 ms
     assert abs(res[0][2] - 2 * 4 * 1.0 / 15e-3) < 1e-9

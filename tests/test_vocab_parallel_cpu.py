@@ -16,12 +16,11 @@ from lm_head_projection_supervised_b200 import vocab_parallel as vp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _free_port():
-    """A TCP port on 127.0.0.1 that the OS reports free (for the rendezvous)."""
-    import socket
-    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
-        sk.bind(("127.0.0.1", 0))
-        return sk.getsockname()[1]
+def _store_path():
+    """A fresh file for the ranks' rendezvous (a file store: no TCP port that
+    another process could take between choosing it and binding it)."""
+    import tempfile
+    return os.path.join(tempfile.mkdtemp(prefix="flce_pg_"), "store")
 
 
 @pytest.mark.parametrize("V,P", [(248320, 8), (248320, 3), (32000, 8), (1000, 7), (9, 9),
@@ -101,14 +100,13 @@ def _inputs(seed=11, N=37, D=9, V=611):
     return H, W, b, y, mask, w
 
 
-def _worker(rank, world, port, reduction, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _worker(rank, world, store, reduction, q):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from lm_head_projection_supervised_b200 import vocab_parallel as vpar
-    dist.init_process_group("gloo", rank=rank, world_size=world,
-                            timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("gloo", init_method="file://" + store, rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         H, W, b, y, mask, w = [torch.from_numpy(a) for a in _inputs()]
         V = W.shape[0]
@@ -130,8 +128,8 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
     from oracle import flce_oracle as orc
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, reduction, q))
+    store = _store_path()
+    procs = [ctx.Process(target=_worker, args=(r, world, store, reduction, q))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -158,14 +156,13 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
     assert sum(r[2] for r in res) == W.shape[0]
 
 
-def _autograd_worker(rank, world, port, reduction, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+def _autograd_worker(rank, world, store, reduction, q):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     from lm_head_projection_supervised_b200 import vocab_parallel as vpar
-    dist.init_process_group("gloo", rank=rank, world_size=world,
-                            timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("gloo", init_method="file://" + store, rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         H, W, b, y, mask, w = [torch.from_numpy(a) for a in _inputs(seed=13)]
         V = W.shape[0]
@@ -193,8 +190,8 @@ def test_gloo_autograd_wrapper(reduction):
     from oracle import flce_oracle as orc
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_autograd_worker, args=(r, 2, port, reduction, q))
+    store = _store_path()
+    procs = [ctx.Process(target=_autograd_worker, args=(r, 2, store, reduction, q))
              for r in range(2)]
     for p in procs:
         p.start()
