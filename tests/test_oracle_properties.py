@@ -12,7 +12,9 @@ from hypothesis import strategies as st
 from oracle import flce_oracle as orc
 from oracle import flce_shards as sh
 
-SETTINGS = dict(max_examples=25, deadline=None,
+# derandomize: the same examples on every run, so that the suite's outcome does
+# not depend on the run (a failing example would fail every time)
+SETTINGS = dict(max_examples=25, deadline=None, derandomize=True,
                 suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
 
 
