@@ -16,6 +16,15 @@ from lm_head_projection_supervised_b200 import vocab_parallel as vp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _close(got, want, rel=1e-11):
+    """fp64 agreement up to summation order: each rank's BLAS adds in its own
+    order (several threads), which moves fp64 results by ~1e-13 relative."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    scale = max(1.0, float(np.max(np.abs(want)))) if want.size else 1.0
+    return float(np.max(np.abs(got - want))) <= rel * scale if want.size else True
+
+
 def _store_path():
     """A fresh file for the ranks' rendezvous (a file store: no TCP port that
     another process could take between choosing it and binding it)."""
@@ -147,12 +156,12 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
     for r in res:
         _, v0, n, loss, m, logs, dH, dW, db = r
         want = ref["loss_vec"] if reduction == "none" else ref["loss"]
-        assert np.max(np.abs(loss - want)) < 1e-12                    # same loss on every rank
-        assert np.max(np.abs(m[idx] - ref["m"][idx])) < 1e-13
-        assert np.max(np.abs(logs[idx] - ref["logs"][idx])) < 1e-12
-        assert np.max(np.abs(dH - ref["dH"])) < 1e-12                 # all-reduced dH
-        assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12     # local slice of dW
-        assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
+        assert _close(loss, want)                                      # same loss on every rank
+        assert _close(m[idx], ref["m"][idx])
+        assert _close(logs[idx], ref["logs"][idx])
+        assert _close(dH, ref["dH"])                                   # all-reduced dH
+        assert _close(dW, ref["dW"][v0:v0 + n])                        # local slice of dW
+        assert _close(db, ref["db"][v0:v0 + n])
     assert sum(r[2] for r in res) == W.shape[0]
 
 
@@ -205,7 +214,7 @@ def test_gloo_autograd_wrapper(reduction):
                                grad_rows=0.8 * g if reduction == "none" else None)
     for _, v0, n, loss, dH, dW, db in res:
         want = ref["loss_vec"] if reduction == "none" else ref["loss"]
-        assert np.max(np.abs(loss - want)) < 1e-12
-        assert np.max(np.abs(dH - ref["dH"])) < 1e-12
-        assert np.max(np.abs(dW - ref["dW"][v0:v0 + n])) < 1e-12
-        assert np.max(np.abs(db - ref["db"][v0:v0 + n])) < 1e-12
+        assert _close(loss, want)
+        assert _close(dH, ref["dH"])
+        assert _close(dW, ref["dW"][v0:v0 + n])
+        assert _close(db, ref["db"][v0:v0 + n])
