@@ -704,7 +704,8 @@ flce_status backward_impl(const void* H, const void* W, const void* b, const int
       kern<<<static_cast<unsigned>(di.sms), FB_THREADS, FB_SMEM_BYTES, s>>>(fa);
     }));
     const int64_t D4 = D / 4;
-    const int64_t dw_blocks = cdiv64(V * D4, 256) < 8LL * di.sms ? cdiv64(V * D4, 256) : 8LL * di.sms;
+    const int64_t dw_blocks =
+        cdiv64(V * D4, 256) < 8LL * di.sms ? cdiv64(V * D4, 256) : 8LL * di.sms;
     FLCE_CK(timed_launch(kProfAux, s, [&] {
       fused_reduce_dw_kernel<<<static_cast<unsigned>(dw_blocks), 256, 0, s>>>(
           reinterpret_cast<const float4*>(p.dwp), L.Vp * D4, static_cast<int>(V),

@@ -21,10 +21,11 @@
 // for the next ones, each pass over the chunk starting after the previous
 // pass's writes have completed, so the additions come in row-block order; the
 // chunk's slice of the slab (about 0.4 MB) stays in L2 meanwhile.  After each
-// row block dH_h goes to the slab of chunk ch.  TMEM (512 columns): Z of both halves [0, 256), dH of
-// both halves [256, 384), dW in two buffers [384, 512) so that the epilogue
-// drains one while the next accumulates.  D > 64 does not fit: dH of 256 rows
-// and a dW tile need 2 D + D columns beside the 256 of the scores.
+// row block dH_h goes to the slab of chunk ch.  TMEM (512 columns): Z of both
+// halves [0, 256), dH of both halves [256, 384), dW in two buffers [384, 512)
+// so that the epilogue drains one while the next accumulates.  D > 64 does
+// not fit: dH of 256 rows and a dW tile need 2 D + D columns beside the 256
+// of the scores.
 //
 // Roles (640 threads): warp 0 schedules items and loads H (once per row
 // block) and the W tiles (a ring); warp 1 issues the MMAs; warps 4..19 are
@@ -43,7 +44,7 @@
 namespace flce {
 
 constexpr int FB_MAX_D = 64;        // hidden sizes the fused backward takes
-constexpr int FB_ROWS = 256;        // rows per work item
+constexpr int FB_ROWS = 256;        // rows per row block (two 128-row halves)
 constexpr int FB_COLS = 128;        // vocabulary ids per tile
 constexpr int FB_WSTAGES = 2;       // W tile ring depth (a tile lasts thousands of cycles)
 constexpr int FB_EPI_WG = 4;        // epilogue warpgroups

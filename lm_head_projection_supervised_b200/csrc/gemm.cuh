@@ -1001,7 +1001,8 @@ __global__ void __launch_bounds__((Shape<MODE, FEAT>::THREADS), 1)
             const float2 o = sMerge[k * BM + r];
             const float mn = fmaxf(st.m, o.x);
             if (mn != -INFINITY) {
-              st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + o.y * ex2_approx((o.x - mn) * kLog2e);
+              st.s = st.s * ex2_approx((st.m - mn) * kLog2e) +
+                     o.y * ex2_approx((o.x - mn) * kLog2e);
               st.m = mn;
             }
           }
