@@ -268,10 +268,9 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         uint32_t n_w = 0, n_t = 0;
         int n_item = 0;
         // Z of the tile with global index ti, from W tile wi of the ring.  The
-        // scores of tile t + 1 are issued as soon as G of tile t is in shared
-        // memory (its Z has been read by then), ahead of tile t's
-        // contractions, so that the epilogue finds them ready after it has
-        // drained the previous dW.
+        // scores of tile t + 1 are issued as soon as the epilogue has read
+        // those of tile t (while it still forms G of tile t), ahead of tile
+        // t's contractions, so that they are ready when it moves on.
         auto issue_z = [&](uint32_t wi, uint32_t ti) -> bool {
           if (!mbar_wait(&w_full[wi % FB_WSTAGES], (wi / FB_WSTAGES) & 1u, abort_flag, g.err) ||
               !mbar_wait(z_empty, (ti & 1) ^ 1, abort_flag, g.err))
@@ -308,6 +307,9 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
                  issue_z(n_w, n_t);
             for (int t = t0; ok && t < t1; ++t) {
               const uint32_t stage = n_w % FB_WSTAGES;
+              // the next tile's scores as soon as this tile's have been read
+              // (the epilogue is still forming G)
+              if (t + 1 < t1 && !(ok = issue_z(n_w + 1, n_t + 1))) break;
               if (!mbar_wait(g_full, n_t & 1, abort_flag, g.err)) {
                 ok = false;
                 break;
@@ -315,7 +317,6 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
               tc_fence_after();
               const uint32_t sw = smem_addr(sW + stage * FB_W_BYTES);
               const uint32_t buf = n_t & 1;
-              if (t + 1 < t1 && !(ok = issue_z(n_w + 1, n_t + 1))) break;
               if (t == t0 && !(ok = mbar_wait(dh_empty, (n_item & 1) ^ 1, abort_flag, g.err)))
                 break;
               // dH_h += G_h W_t: G K-major (rows x ids), W_t MN-major (ids x D)
@@ -472,21 +473,22 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           for (int c = 0; c < 2; ++c) {
             tmem_ld32(t_z + c * 32, za);
             tmem_wait_ld(za);
+            if (c == 1) {
+              // Z read: its TMEM is free for the next tile's scores
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(z_empty);
+            }
             grad_chunk<FEAT>(g, za, 64 * ss + c * 32, vglob0, vlim, yl, valid, krow, rrow, row,
                              lane, pk, big);
             // G of tile t - 1 has been read by its contractions
             if (c == 0) mbar_wait(g_empty, (n_t & 1) ^ 1, abort_flag, g.err);
             stage_row128(gbox, r, 4 * c, pk);
           }
-          // Z read (TMEM free for the next tile's scores) and G written
-          // (visible to the tensor core's reads)
-          tc_fence_before();
+          // G written (visible to the tensor core's reads)
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(z_empty);
-            mbar_arrive(g_full);
-          }
+          if (lane == 0) mbar_arrive(g_full);
           if (t > t0 && ((t - 1) & 1) == hh) {
             const uint32_t np = n_t - 1;
             mbar_wait(&dw_full[np & 1], (np >> 1) & 1, abort_flag, g.err);
