@@ -277,14 +277,18 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
             return false;
           tc_fence_after();
           const uint32_t sw = smem_addr(sW + (wi % FB_WSTAGES) * FB_W_BYTES);
+          // descriptors: the low words once, each MMA adds its offset (40 MMAs
+          // a tile, issued by one thread that shares its scheduler with four
+          // epilogue warps: the issue cost is on the tile's critical path)
+          const uint32_t za = desc_lo_sw128(sh, 16), zb = desc_lo_sw128(sw, 16);
           // K = 64 (the hidden size, zero-padded)
-#pragma unroll 1
+#pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               umma_f16(tmem_base + FB_TM_Z + 128 * h,
-                       smem_desc_sw128(sh + h * FB_H_BYTES + kk * 32, 16, 1024),
-                       smem_desc_sw128(sw + kk * 32, 16, 1024), idesc_z, kk > 0 ? 1u : 0u);
+                       desc_sw128_sbo1k(za + ((h * FB_H_BYTES + kk * 32) >> 4)),
+                       desc_sw128_sbo1k(zb + ((kk * 32) >> 4)), idesc_z, kk > 0 ? 1u : 0u);
           umma_commit(z_full);
           return true;
         };
@@ -319,32 +323,34 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
               const uint32_t buf = n_t & 1;
               if (t == t0 && !(ok = mbar_wait(dh_empty, (n_item & 1) ^ 1, abort_flag, g.err)))
                 break;
+              const uint32_t ga = desc_lo_sw128(sg, 16), wb = desc_lo_sw128(sw, 8192);
+              const uint32_t acc0 = t > t0 ? 1u : 0u;
               // dH_h += G_h W_t: G K-major (rows x ids), W_t MN-major (ids x D)
-#pragma unroll 1
+#pragma unroll
               for (int h = 0; h < 2; ++h)
-#pragma unroll 1
+#pragma unroll
                 for (int j = 0; j < 2; ++j)
 #pragma unroll
                   for (int kk = 0; kk < 4; ++kk)
                     umma_f16(tmem_base + FB_TM_DH + 64 * h,
-                             smem_desc_sw128(sg + h * FB_G_BYTES + j * STG_BYTES + kk * 32, 16,
-                                             1024),
-                             smem_desc_sw128(sw + j * 8192 + kk * 2048, 8192, 1024), idesc_dh,
-                             (t > t0 || j > 0 || kk > 0) ? 1u : 0u);
+                             desc_sw128_sbo1k(ga + ((h * FB_G_BYTES + j * STG_BYTES + kk * 32) >> 4)),
+                             desc_sw128_sbo1k(wb + ((j * 8192 + kk * 2048) >> 4)), idesc_dh,
+                             (j > 0 || kk > 0) ? 1u : acc0);
               if (!mbar_wait(&dw_empty[buf], ((n_t >> 1) & 1) ^ 1, abort_flag, g.err)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
+              const uint32_t gm = desc_lo_sw128(sg, STG_BYTES), hm = desc_lo_sw128(sh, 8192);
+              const uint32_t tdw = tmem_base + FB_TM_DW + 64 * buf;
               // dW_t = sum_h G_h^T H_h: G MN-major (ids x rows), H_h MN-major (D x rows)
-#pragma unroll 1
+#pragma unroll
               for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                  umma_f16(tmem_base + FB_TM_DW + 64 * buf,
-                           smem_desc_sw128(sg + h * FB_G_BYTES + kk * 2048, STG_BYTES, 1024),
-                           smem_desc_sw128(sh + h * FB_H_BYTES + kk * 2048, 8192, 1024),
-                           idesc_dw, (h > 0 || kk > 0) ? 1u : 0u);
+                  umma_f16(tdw, desc_sw128_sbo1k(gm + ((h * FB_G_BYTES + kk * 2048) >> 4)),
+                           desc_sw128_sbo1k(hm + ((h * FB_H_BYTES + kk * 2048) >> 4)), idesc_dw,
+                           (h > 0 || kk > 0) ? 1u : 0u);
               umma_commit(&dw_full[buf]);
               umma_commit(g_empty);
               umma_commit(&w_empty[stage]);
@@ -467,24 +473,27 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           const int vlim = g.V - vglob0;
           const int yl = valid ? yabs - vglob0 : -1000000;
           const uint32_t t_z = lane_base + FB_TM_Z + 128 * hh + 64 * ss;
-          uint32_t za[32], pk[16];
+          // both 32-id chunks are formed before the wait for the previous
+          // tile's contractions to release G, so that only the stores into
+          // shared memory wait for them
+          uint32_t za[32], pk0[16], pk1[16];
           bool big = false;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(t_z + c * 32, za);
-            tmem_wait_ld(za);
-            if (c == 1) {
-              // Z read: its TMEM is free for the next tile's scores
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(z_empty);
-            }
-            grad_chunk<FEAT>(g, za, 64 * ss + c * 32, vglob0, vlim, yl, valid, krow, rrow, row,
-                             lane, pk, big);
-            // G of tile t - 1 has been read by its contractions
-            if (c == 0) mbar_wait(g_empty, (n_t & 1) ^ 1, abort_flag, g.err);
-            stage_row128(gbox, r, 4 * c, pk);
-          }
+          tmem_ld32(t_z, za);
+          tmem_wait_ld(za);
+          grad_chunk<FEAT>(g, za, 64 * ss, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk0,
+                           big);
+          tmem_ld32(t_z + 32, za);
+          tmem_wait_ld(za);
+          // Z read: its TMEM is free for the next tile's scores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(z_empty);
+          grad_chunk<FEAT>(g, za, 64 * ss + 32, vglob0, vlim, yl, valid, krow, rrow, row, lane,
+                           pk1, big);
+          // G of tile t - 1 has been read by its contractions
+          mbar_wait(g_empty, (n_t & 1) ^ 1, abort_flag, g.err);
+          stage_row128(gbox, r, 0, pk0);
+          stage_row128(gbox, r, 4, pk1);
           // G written (visible to the tensor core's reads)
           fence_proxy_async_smem();
           __syncwarp();

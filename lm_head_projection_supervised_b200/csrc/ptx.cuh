@@ -356,6 +356,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The same descriptor in two parts, for issuers that step through a tile:
+// the low word (start address and leading byte offset) computed once, and a
+// descriptor per MMA from it plus the start offset in 16-byte units (which
+// stays inside the 14-bit field for shared-memory addresses below 256 KiB),
+// with a 1024-byte stride byte offset.
+__device__ __forceinline__ uint32_t desc_lo_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc_sw128_sbo1k(uint32_t lo) {
+  constexpr uint32_t hi = ((1024u >> 4) & 0x3FFFu) | (1u << (46 - 32)) | (2u << (61 - 32));
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // Instruction descriptor of tcgen05.mma.kind::f16: f32 accumulator,
 // A/B both bf16 (or both fp16), per-operand major-ness, shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc_f16(bool bf16, bool a_mn, bool b_mn, int M,
