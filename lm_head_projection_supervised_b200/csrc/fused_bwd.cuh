@@ -461,6 +461,12 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
                       g.log2_sigma - __ldg(g.logs_saved + o) * kLog2e);
           rrow = __ldg(g.row_scale + row);
         }
+        // a warp whose 32 rows are all supervised with a positive scale takes
+        // the scale into the exponent (two operations an entry fewer); the
+        // bias variants keep the general form, which needs fewer registers
+        const bool fold =
+            (FEAT & kFeatBias) == 0 && __all_sync(0xffffffffu, valid && rrow > 0.f);
+        const float krow_f = fold ? krow + log2f(rrow) : krow;
         // The epilogue warps decide together whether to stop once per row
         // block (at its end): a wait that gives up raises the abort flag and
         // returns, the later waits return at once, and the warps run on to
@@ -480,16 +486,24 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           bool big = false;
           tmem_ld32(t_z, za);
           tmem_wait_ld(za);
-          grad_chunk<FEAT>(g, za, 64 * ss, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk0,
-                           big);
+          if (fold)
+            grad_chunk<FEAT, true>(g, za, 64 * ss, vglob0, vlim, yl, true, krow_f, rrow, row, lane,
+                                   pk0, big);
+          else
+            grad_chunk<FEAT>(g, za, 64 * ss, vglob0, vlim, yl, valid, krow, rrow, row, lane, pk0,
+                             big);
           tmem_ld32(t_z + 32, za);
           tmem_wait_ld(za);
           // Z read: its TMEM is free for the next tile's scores
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(z_empty);
-          grad_chunk<FEAT>(g, za, 64 * ss + 32, vglob0, vlim, yl, valid, krow, rrow, row, lane,
-                           pk1, big);
+          if (fold)
+            grad_chunk<FEAT, true>(g, za, 64 * ss + 32, vglob0, vlim, yl, true, krow_f, rrow, row,
+                                   lane, pk1, big);
+          else
+            grad_chunk<FEAT>(g, za, 64 * ss + 32, vglob0, vlim, yl, valid, krow, rrow, row, lane,
+                             pk1, big);
           // G of tile t - 1 has been read by its contractions
           mbar_wait(g_empty, (n_t & 1) ^ 1, abort_flag, g.err);
           stage_row128(gbox, r, 0, pk0);

@@ -535,8 +535,11 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
 // Epilogue: gradient-panel values of one 32-column chunk, packed to 16 bits.
 // ---------------------------------------------------------------------------
 // krow is log2(sigma) - (log s) log2(e) - m log2(e) for the row, so that
-// sigma p = 2^(z log2(e) + krow) takes one FMA per entry.
-template <int FEAT>
+// sigma p = 2^(z log2(e) + krow) takes one FMA per entry.  FOLDED: the row is
+// supervised and its scale r positive, and krow already holds log2(r) as
+// well, so that the entry is r sigma p at once (no selection on `valid`, no
+// product with r) and the one-hot term is r sigma.
+template <int FEAT, bool FOLDED = false>
 __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32], int cb,
                                            int vglob0, int vlim, int yl, bool valid,
                                            float krow, float rrow, int row, int lane,
@@ -555,7 +558,7 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
 #pragma unroll
   for (int j = 0; j < 32; ++j) gv[j] = ex2_approx(fmaf(x[j], kLog2e, krow));
-  if (!valid) {
+  if (!FOLDED && !valid) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) gv[j] = 0.f;
   }
@@ -566,17 +569,20 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   }
   const int jt = yl - cb;
   if (static_cast<unsigned>(jt) < 32u) {
+    const float onehot = FOLDED ? g.sigma * rrow : g.sigma;
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (j == jt) gv[j] -= g.sigma;
+      if (j == jt) gv[j] -= onehot;
   }
   if (FEAT & kFeatFilter) {
     // gradient filtering: does this row hold an entry that is not negligible?
 #pragma unroll
     for (int j = 0; j < 32; ++j) big |= fabsf(gv[j]) >= g.filter_eps_sigma;
   }
+  if (!FOLDED) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) gv[j] *= rrow;  // the row's scale relative to S
+    for (int j = 0; j < 32; ++j) gv[j] *= rrow;  // the row's scale relative to S
+  }
   // The target entry r (p - 1) sigma dominates its row of dH; keep what the
   // 16-bit rounding takes off it so that dH can add it back in fp32.
   if (valid && static_cast<unsigned>(jt) < 32u) {
