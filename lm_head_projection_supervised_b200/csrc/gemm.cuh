@@ -480,15 +480,14 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
     for (int j = 0; j < 32; ++j)
       if (cb + j >= vlim) x[j] = -INFINITY;
   }
-  // chunk max as a tree (depth 5 instead of a chain of 31)
-  float t[16];
+  // chunk max as a tree of three-input maxima (17 operations, depth 4)
+  float t[11];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) t[j] = fmaxf(x[j], x[j + 16]);
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
-  const float cm = t[0];
+  for (int j = 0; j < 10; ++j) t[j] = fmax3(x[3 * j], x[3 * j + 1], x[3 * j + 2]);
+  t[10] = fmaxf(x[30], x[31]);
+  const float u0 = fmax3(t[0], t[1], t[2]), u1 = fmax3(t[3], t[4], t[5]),
+              u2 = fmax3(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
+  const float cm = fmaxf(fmax3(u0, u1, u2), u3);
   const float mn = fmaxf(st.m, cm);
   // nothing seen yet and this chunk is all padding (a half tile past V): the
   // state stays (-inf, 0) instead of exp(-inf + inf)

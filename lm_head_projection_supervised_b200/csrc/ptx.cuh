@@ -378,6 +378,13 @@ __host__ __device__ constexpr uint32_t make_idesc_f16(bool bf16, bool a_mn, bool
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the special-function unit.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
