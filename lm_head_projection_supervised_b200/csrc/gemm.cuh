@@ -493,16 +493,18 @@ __device__ __forceinline__ void fwd_chunk(const GemmArgs& g, uint32_t (&z)[32], 
   // state stays (-inf, 0) instead of exp(-inf + inf)
   if (mn == -INFINITY) return;
   const float nb = -mn * kLog2e;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  // four running sums, two per packed pair
+  const float2 l2 = make_float2(kLog2e, kLog2e), nb2 = make_float2(nb, nb);
+  float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
-    a0 += ex2_approx(fmaf(x[j], kLog2e, nb));
-    a1 += ex2_approx(fmaf(x[j + 1], kLog2e, nb));
-    a2 += ex2_approx(fmaf(x[j + 2], kLog2e, nb));
-    a3 += ex2_elem<POLY>(fmaf(x[j + 3], kLog2e, nb), j + 3);
+    const float2 y01 = ffma2(make_float2(x[j], x[j + 1]), l2, nb2);
+    const float2 y23 = ffma2(make_float2(x[j + 2], x[j + 3]), l2, nb2);
+    a01 = fadd2(a01, make_float2(ex2_approx(y01.x), ex2_approx(y01.y)));
+    a23 = fadd2(a23, make_float2(ex2_approx(y23.x), ex2_elem<POLY>(y23.y, j + 3)));
   }
   // first chunk: st.m = -inf, the old sum is scaled by exp(-inf) = 0
-  st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + ((a0 + a1) + (a2 + a3));
+  st.s = st.s * ex2_approx((st.m - mn) * kLog2e) + ((a01.x + a01.y) + (a23.x + a23.y));
   st.m = mn;
   const int jt = yl - cb;
   if (static_cast<unsigned>(jt) < 32u) {
@@ -555,8 +557,18 @@ __device__ __forceinline__ void grad_chunk(const GemmArgs& g, uint32_t (&z)[32],
   if (FEAT & kFeatRound) round_to_input_type(g, x);
   float gv[32];
   // sigma * p = 2^( ((z - m) - log s) * log2(e) + log2(sigma) )
+  if (FOLDED) {
+    const float2 l2 = make_float2(kLog2e, kLog2e), k2 = make_float2(krow, krow);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) gv[j] = ex2_approx(fmaf(x[j], kLog2e, krow));
+    for (int j = 0; j < 32; j += 2) {
+      const float2 y = ffma2(make_float2(x[j], x[j + 1]), l2, k2);
+      gv[j] = ex2_approx(y.x);
+      gv[j + 1] = ex2_approx(y.y);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) gv[j] = ex2_approx(fmaf(x[j], kLog2e, krow));
+  }
   if (!FOLDED && !valid) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) gv[j] = 0.f;
