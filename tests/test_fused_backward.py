@@ -71,6 +71,38 @@ def test_fused_and_panel_backward_match_the_oracle(name, kw):
             assert np.abs(out["fused"][q] - out["panel"][q]).max() <= 1e-3 * scale
 
 
+def test_fused_backward_mixed_row_scales():
+    """Per-row upstream gradients that are positive for the first rows and of
+    mixed sign (some zero) after them: warps whose rows all have a positive
+    scale take it into the exponent, the others scale each entry, and both
+    must agree with the oracle."""
+    inp = wl.random_case(seed=80, N=700, D=64, V=6000, bias=False, ignore_frac=0.0,
+                         mask_false_frac=0.0)
+    rng = np.random.default_rng(80)
+    g = 10.0 ** rng.uniform(-2, 1, inp.N)
+    tail = np.arange(inp.N) >= 256
+    g[tail] *= rng.choice([-1.0, 0.0, 1.0], int(tail.sum()))
+    g32 = torch.tensor(g, dtype=torch.float32).numpy().astype(np.float64)
+    H, W, b, y, mk = to_device(inp)
+    ws = binding.Workspace(inp.N, inp.D, inp.V, H.dtype)
+    _, m, logs = binding.forward(H, W, b, y, mk, -100, ws=ws, reduction="none")
+    grads = torch.tensor(g32, dtype=torch.float32, device="cuda")
+    out = {}
+    for form, panel in (("fused", False), ("panel", True)):
+        dH, dW, _ = binding.backward(H, W, b, y, mk, -100, m, logs, lam=1.0, ws=ws,
+                                     reduction="none", grad_rows=grads, panel_backward=panel)
+        assert binding.device_status(ws) == 0
+        out[form] = (dH.cpu().numpy(), dW.cpu().numpy())
+    ref = orc.forward_backward(inp.H64(), inp.W64(), inp.b64(), inp.labels, inp.mask, lam=1.0,
+                               reduction="none", grad_rows=g32)
+    for form in ("fused", "panel"):
+        check_grad(f"dH_{form}", out[form][0], ref["dH"])
+        check_grad(f"dW_{form}", out[form][1], ref["dW"])
+    # rows with a zero upstream gradient get a zero dH row
+    zero = np.flatnonzero(g32 == 0.0)
+    assert zero.size > 0 and not out["fused"][0][zero].any()
+
+
 def test_fused_backward_rounded_logits():
     inp = wl.random_case(seed=77, N=500, D=64, V=4000)
     loss, out = _both_forms(inp, round_logits=True)
