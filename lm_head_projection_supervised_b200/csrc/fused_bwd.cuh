@@ -70,6 +70,11 @@ constexpr uint32_t FB_TM_DW = 384;  // dW buffer 0 (buffer 1 at +64)
 constexpr size_t FB_SMEM_BYTES = 1024 + 2 * FB_HB_BYTES + FB_WSTAGES * FB_W_BYTES +
                                  2 * FB_G_BYTES + (FB_EPI_THREADS / 32) * FB_STG_BYTES + 512;
 static_assert(FB_SMEM_BYTES <= 232448, "shared memory per CTA");
+// The MMA issuer adds operand offsets to a descriptor's 14-bit start-address
+// field (desc_sw128_sbo1k): every shared-memory address of the CTA (this
+// kernel's dynamic shared memory after at most 1 KiB reserved ahead of it),
+// in 16-byte units, stays below 2^14.
+static_assert(1024 + FB_SMEM_BYTES <= (size_t(1) << 18), "descriptor start-address field");
 
 // The split of the work: nch vocabulary chunks (one per CTA or more, at most
 // FB_NCH_MAX: a chunk's dW slice stays small enough for L2) times ng groups
