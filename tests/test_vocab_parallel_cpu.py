@@ -16,13 +16,21 @@ from lm_head_projection_supervised_b200 import vocab_parallel as vp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _close(got, want, rel=1e-11):
+def _check(name, got, want, rel=1e-11):
     """fp64 agreement up to summation order: each rank's BLAS adds in its own
-    order (several threads), which moves fp64 results by ~1e-13 relative."""
+    order (several threads), which moves fp64 results by ~1e-13 relative.  A
+    failure names the quantity, the largest error, where it is and the bar."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
-    scale = max(1.0, float(np.max(np.abs(want)))) if want.size else 1.0
-    return float(np.max(np.abs(got - want))) <= rel * scale if want.size else True
+    assert got.shape == want.shape, f"{name}: shape {got.shape} against {want.shape}"
+    if not want.size:
+        return
+    scale = max(1.0, float(np.max(np.abs(want))))
+    err = np.abs(got - want)
+    k = int(np.argmax(err))
+    assert err.flat[k] <= rel * scale, (
+        f"{name}: max error {err.flat[k]:.3e} at flat index {k} (got {got.flat[k]!r}, "
+        f"want {want.flat[k]!r}; bar {rel * scale:.3e})")
 
 
 def _store_path():
@@ -156,12 +164,12 @@ def test_gloo_ranks_reproduce_the_dense_oracle(world, reduction):
     for r in res:
         _, v0, n, loss, m, logs, dH, dW, db = r
         want = ref["loss_vec"] if reduction == "none" else ref["loss"]
-        assert _close(loss, want)                                      # same loss on every rank
-        assert _close(m[idx], ref["m"][idx])
-        assert _close(logs[idx], ref["logs"][idx])
-        assert _close(dH, ref["dH"])                                   # all-reduced dH
-        assert _close(dW, ref["dW"][v0:v0 + n])                        # local slice of dW
-        assert _close(db, ref["db"][v0:v0 + n])
+        _check("loss", loss, want)                                     # same loss on every rank
+        _check("m", m[idx], ref["m"][idx])
+        _check("logs", logs[idx], ref["logs"][idx])
+        _check("dH", dH, ref["dH"])                                    # all-reduced dH
+        _check("dW", dW, ref["dW"][v0:v0 + n])                         # local slice of dW
+        _check("db", db, ref["db"][v0:v0 + n])
     assert sum(r[2] for r in res) == W.shape[0]
 
 
@@ -214,7 +222,7 @@ def test_gloo_autograd_wrapper(reduction):
                                grad_rows=0.8 * g if reduction == "none" else None)
     for _, v0, n, loss, dH, dW, db in res:
         want = ref["loss_vec"] if reduction == "none" else ref["loss"]
-        assert _close(loss, want)
-        assert _close(dH, ref["dH"])
-        assert _close(dW, ref["dW"][v0:v0 + n])
-        assert _close(db, ref["db"][v0:v0 + n])
+        _check("loss", loss, want)
+        _check("dH", dH, ref["dH"])
+        _check("dW", dW, ref["dW"][v0:v0 + n])
+        _check("db", db, ref["db"][v0:v0 + n])
