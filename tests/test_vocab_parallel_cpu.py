@@ -19,9 +19,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _check(name, got, want, rel=1e-9):
     """fp64 agreement up to summation order.  Usually the ranks agree with the
     dense oracle to ~1e-15 relative; about one run in fifty on a loaded host a
-    single entry differs by up to ~4e-10 relative (seen on log s and on dH), a
-    rounding-level effect of the CPU libraries' thread splits, nine orders of
-    magnitude below what a wrong cut or exchange produces.  A failure names the
+    single entry differs by up to ~4e-10 relative (seen on log s and on dH;
+    the cause is not identified), nine orders of magnitude below what a wrong
+    cut or exchange produces.  A failure names the
     quantity, the largest error, where it is and the bar."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
